@@ -1,0 +1,370 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test would fail for a plausible mistake in the oracle: a /16 instead of
+/15, a sign flip of the zero point, rint taken after adding z, a swapped
+nibble order, a transposed operand, a dropped bias, a wrong group index.
+None of these tests calls the CUDA library.
+"""
+from fractions import Fraction
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from gemv_w4a16_groupwise_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16(vals):
+    return synth.f64_to_bf16_bits(np.asarray(vals, dtype=np.float64))
+
+
+def f16_value(bits):
+    return float(np.asarray(bits, dtype=np.uint16).view(np.float16))
+
+
+def bf16_value(bits):
+    return synth.bf16_bits_to_f32(np.asarray(bits, dtype=np.uint16)).astype(np.float64)
+
+
+# ----------------------------------------------------------------------------
+# Hand-derived closed-form examples (derivations in the comments).
+# Reading of the quantizer (llm-quantization, Objective 1, no formula printed):
+#   s = fp16((max-min)/15); z = clamp(rint(-min/s), 0, 15); q = clamp(rint(w/s) + z, 0, 15)
+# ----------------------------------------------------------------------------
+ROW_A = [-1.0, -0.5, 0.0, 0.5, 1.0, 2.0, 1.5, -0.25]
+# min -1, max 2: (2+1)/15 = 0.2 -> fp16 1.599609375*2^-3 = 0.199951171875 (0x3266)
+# z = rint(1/0.19995...) = rint(5.0012) = 5 (0x4500)
+# w/s = -5.0012, -2.5006, 0, 2.5006, 5.0012, 10.0024, 7.5018, -1.2503
+# rint + 5 = 0, 2, 5, 8, 10, 15, 13, 4
+ROW_A_Q = [0, 2, 5, 8, 10, 15, 13, 4]
+ROW_B = [-1.75, 2.0, 0.125, 0.375, -0.125, -0.375, 0.625, 1.125]
+# min -1.75, max 2: 3.75/15 = 0.25 exactly (0x3400); z = 7 (0x4700)
+# w/s = -7, 8, 0.5, 1.5, -0.5, -1.5, 2.5, 4.5 -> ties go to even: 0, 2, -0, -2, 2, 4
+ROW_B_Q = [0, 15, 7, 9, 7, 5, 9, 11]
+
+
+def test_golden_groupwise_example():
+    q, s, z = oracle.quantize(bf16([ROW_A, ROW_B]), "groupwise", 8)
+    assert q.tolist() == [ROW_A_Q, ROW_B_Q]
+    assert s.ravel().tolist() == [0x3266, 0x3400]
+    assert z.ravel().tolist() == [0x4500, 0x4700]
+    p = oracle.pack(q)
+    # nibble i of the word holds code i: A -> 4,D,F,A,8,5,2,0 ; B -> B,9,5,7,9,7,F,0
+    assert p.ravel().tolist() == [0x4DFA8520, 0xB95797F0]
+
+
+def test_golden_rowwise_and_global():
+    W = bf16([ROW_A, ROW_B])
+    q, s, z = oracle.quantize(W, "rowwise", 0)
+    assert s.shape == (2, 1) and q.tolist() == [ROW_A_Q, ROW_B_Q]
+    assert s.ravel().tolist() == [0x3266, 0x3400]
+    # GLOBAL: one group over both rows -> min -1.75, max 2 -> s 0.25, z 7;
+    # row A: w/s = -4, -2, 0, 2, 4, 8, 6, -1 -> +7 = 3, 5, 7, 9, 11, 15, 13, 6
+    q, s, z = oracle.quantize(W, "global", 0)
+    assert s.shape == (1, 1) and s[0, 0] == 0x3400 and z[0, 0] == 0x4700
+    assert q.tolist() == [[3, 5, 7, 9, 11, 15, 13, 6], ROW_B_Q]
+
+
+def test_golden_degenerate_groups():
+    rows = [[0.5] * 8, [0.0] * 8, [-3.0] * 8, [1.0, 1.5, 2.0, 1.25, 1.75, 1.0, 2.0, 1.5]]
+    q, s, z = oracle.quantize(bf16(rows), "groupwise", 8)
+    # constant 0.5: s = 0 -> s = max(|min|, 2^-14) = 0.5; z = clamp(rint(-1)) = 0; q = 1
+    assert (q[0] == 1).all() and s[0, 0] == 0x3800 and z[0, 0] == 0
+    # all zero: s = 2^-14 (0x0400), z = 0, q = 0 -> w_hat = 0 exactly
+    assert (q[1] == 0).all() and s[1, 0] == 0x0400 and z[1, 0] == 0
+    # constant -3: s = 3 (0x4200), z = 1 (0x3C00), q = rint(-1) + 1 = 0 -> w_hat = -3
+    assert (q[2] == 0).all() and s[2, 0] == 0x4200 and z[2, 0] == 0x3C00
+    # all positive, min 1 max 2: s = fp16(1/15) = 0.066650390625 (0x2C44); z clamps to 0;
+    # every w/s >= 15 so every code clamps to 15 (the clamped integer zero point cannot
+    # reach a group that does not straddle zero)
+    assert (q[3] == 15).all() and s[3, 0] == 0x2C44 and z[3, 0] == 0
+    wh = oracle.dequant(oracle.pack(q), s, z, "groupwise", 8, 8)
+    assert wh[0].tolist() == [0.5] * 8 and wh[1].tolist() == [0.0] * 8
+    assert wh[2].tolist() == [-3.0] * 8 and wh[3].tolist() == [0.999755859375] * 8
+
+
+def test_golden_matmul_example():
+    W = bf16([ROW_A, ROW_B])
+    p, s, z = oracle.quantize_pack(W, "groupwise", 8)
+    X = bf16([[1, 0, 0, 0, 0, 0, 0, 0], [1] * 8, [0.5, -1, 2, 0, 0, 0, 0, 1]])
+    y64, ybf = oracle.linear(X, p, s, z, "groupwise", 8, 2, 8)
+    sA = 0.199951171875
+    # row 0 picks w_hat[:,0]: (0-5)*sA and (0-7)*0.25
+    # row 1 sums the codes: A: sum(q-z) = 17 -> 17*sA ; B: sum(q-z) = 7 -> 1.75
+    # row 2: A: 0.5*(-5) - (-3) + 2*0 + (-1) = -0.5 -> -0.5*sA ; B: -3.5 - 8 + 4 = -7.5 -> -1.875
+    expect = [[-5 * sA, -1.75], [17 * sA, 1.75], [-0.5 * sA, -1.875]]
+    assert y64.tolist() == expect
+    # bf16: -0.99976 -> -1.0 ; 3.39917 -> 218*2^-6 = 3.40625 ; -0.09998 -> -205*2^-11
+    assert bf16_value(ybf).tolist() == [[-1.0, -1.75], [3.40625, 1.75], [-0.10009765625, -1.875]]
+    # bias epilogue adds bias[n] once before the single rounding
+    y64b, _ = oracle.linear(X, p, s, z, "groupwise", 8, 2, 8, bias=bf16([0.25, -1.0]))
+    assert (y64b - y64).tolist() == [[0.25, -1.0]] * 3
+    # transposed: one-hot dY rows return the dequantized rows, a sum returns their sum
+    dY = bf16([[1, 0], [0, 1], [1, 1]])
+    x64, _ = oracle.linear_t(dY, p, s, z, "groupwise", 8, 2, 8)
+    wa = [(q - 5) * sA for q in ROW_A_Q]
+    wb = [(q - 7) * 0.25 for q in ROW_B_Q]
+    assert x64.tolist() == [wa, wb, [a + b for a, b in zip(wa, wb)]]
+
+
+# ----------------------------------------------------------------------------
+# bf16 rounding (used for every output)
+# ----------------------------------------------------------------------------
+def test_bf16_rounding_ties_and_cross_check():
+    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: ties to the even mantissa -> 1.0
+    assert oracle.f64_to_bf16(1 + 2.0 ** -8) == 0x3F80
+    # 1 + 3*2^-8 is halfway between 1 + 2^-7 (odd) and 1 + 2^-6 (even)
+    assert oracle.f64_to_bf16(1 + 3 * 2.0 ** -8) == 0x3F82
+    assert oracle.f64_to_bf16(-2.0) == 0xC000
+    assert oracle.f64_to_bf16(0.0) == 0x0000 and oracle.f64_to_bf16(-0.0) == 0x8000
+    # a value a hair above the tie rounds up (no fp32 double rounding)
+    assert oracle.f64_to_bf16(1 + 2.0 ** -8 + 2.0 ** -40) == 0x3F81
+    # the C routine and the input generator's independent bit trick agree
+    rng = np.random.default_rng(5)
+    v = rng.standard_normal(20000) * np.exp(rng.uniform(-20, 20, 20000))
+    ref = synth.f64_to_bf16_bits(v)
+    got = np.array([oracle.f64_to_bf16(x) for x in v], np.uint16)
+    assert (ref == got).all()
+
+
+# ----------------------------------------------------------------------------
+# Quantizer: exact round trip, brute force, error bound
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("g", [8, 16, 64])
+def test_exact_round_trip_power_of_two_scales(g):
+    """w = (q - z) * 2^-e is exactly representable; quantize must return q, z, 2^-e."""
+    rng = np.random.default_rng(11 + g)
+    N, G = 24, 5
+    K = G * g
+    q = rng.integers(0, 16, size=(N, K))
+    q[:, ::g] = 0            # every group reaches both ends of the code range
+    q[:, 1::g] = 15
+    z = rng.integers(0, 16, size=(N, G))
+    e = rng.integers(-3, 20, size=(N, G))
+    zk = np.repeat(z, g, axis=1)
+    ek = np.repeat(e, g, axis=1)
+    w = (q - zk) * np.ldexp(1.0, -ek)
+    W = bf16(w)
+    assert (bf16_value(W) == w).all()
+    q2, s2, z2 = oracle.quantize(W, "groupwise", g)
+    assert (q2 == q).all()
+    assert (z2.view(np.float16).astype(np.float64) == z).all()
+    assert (s2.view(np.float16).astype(np.float64) == np.ldexp(1.0, -e)).all()
+    wh = oracle.dequant(oracle.pack(q2), s2, z2, "groupwise", g, K)
+    assert (wh == w).all()
+
+
+def _brute_force_group(w_vals, s, z):
+    """Nearest code by exact rational distance, ties to even (q - z)."""
+    out = []
+    sF = Fraction(s)
+    for w in w_vals:
+        t = Fraction(w) / sF
+        best = None
+        for cand in range(16):
+            d = abs(t - (cand - z))
+            key = (d, (cand - z) % 2)
+            if best is None or key < best[0]:
+                best = (key, cand)
+        out.append(best[1])
+    return out
+
+
+def test_brute_force_codes_and_zero_point():
+    rng = np.random.default_rng(3)
+    g = 16
+    W = synth.normal_bf16((40, 4 * g), 0.0, 0.02, seed=7, stream=2)
+    W[5, :g] = bf16(rng.uniform(-1, 1, g) * 3)         # wider groups
+    W[6, g:2 * g] = bf16(np.round(rng.uniform(-8, 8, g)) * 0.125)   # many exact ties
+    q, s, z = oracle.quantize(W, "groupwise", g)
+    wv = bf16_value(W)
+    for n in range(W.shape[0]):
+        for gi in range(4):
+            sl = slice(gi * g, (gi + 1) * g)
+            sv = f16_value(s[n, gi])
+            zv = int(f16_value(z[n, gi]))
+            mn = Fraction(float(wv[n, sl].min()))
+            # z is the integer nearest -min/s (ties to even), clamped to [0, 15]
+            t = -mn / Fraction(sv)
+            zf = int(np.floor(t))
+            rem = t - zf
+            zr = zf + (1 if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and zf % 2) else 0)
+            assert zv == min(max(zr, 0), 15)
+            assert q[n, sl].tolist() == _brute_force_group(wv[n, sl], sv, zv)
+
+
+@pytest.mark.parametrize("mode,g", [("groupwise", 32), ("groupwise", 128), ("rowwise", 0),
+                                    ("global", 0)])
+def test_error_bound_half_step(mode, g):
+    """|w - w_hat| <= 0.51 s wherever the group straddles zero."""
+    W = synth.normal_bf16((64, 512), 0.0, 0.02, seed=21, stream=2)
+    q, s, z = oracle.quantize(W, mode, g)
+    K = 512
+    wh = oracle.dequant(oracle.pack(q), s, z, mode, g, K)
+    sv = s.view(np.float16).astype(np.float64)
+    gl = {"groupwise": g, "rowwise": K, "global": K}[mode]
+    if mode == "global":
+        sk = np.full(W.shape, sv[0, 0])
+    else:
+        sk = np.repeat(sv, gl, axis=1)
+    err = np.abs(bf16_value(W) - wh)
+    assert (err <= 0.51 * sk).all()
+    # and the scale is the smallest that spans the group: max error is at least s/4 somewhere
+    assert err.max() >= 0.25 * sk.min()
+
+
+def test_groups_are_independent_and_row_local():
+    """Quantizing a row subset gives the same codes as quantizing the full matrix."""
+    W = synth.normal_bf16((32, 256), 0.0, 0.02, seed=4, stream=2)
+    q, s, z = oracle.quantize(W, "groupwise", 64)
+    q2, s2, z2 = oracle.quantize(W[10:20], "groupwise", 64)
+    assert (q2 == q[10:20]).all() and (s2 == s[10:20]).all() and (z2 == z[10:20]).all()
+    # each group only sees its own columns
+    W3 = W.copy()
+    W3[:, 64:128] = bf16(np.zeros((32, 64)))
+    q3, s3, _ = oracle.quantize(W3, "groupwise", 64)
+    assert (q3[:, :64] == q[:, :64]).all() and (s3[:, 2:] == s[:, 2:]).all()
+
+
+def test_invalid_arguments():
+    W = synth.normal_bf16((4, 64), 0.0, 0.02, seed=1, stream=2)
+    with pytest.raises(ValueError):
+        oracle.quantize(W, "groupwise", 48)   # K % g != 0
+    with pytest.raises(ValueError):
+        oracle.quantize(W, "groupwise", 0)
+
+
+# ----------------------------------------------------------------------------
+# Packing
+# ----------------------------------------------------------------------------
+def test_pack_golden_words_and_byte_view():
+    q = np.array([[0, 1, 2, 3, 4, 5, 6, 7], [15, 0, 0, 0, 0, 0, 0, 0],
+                  [0, 0, 0, 0, 0, 0, 0, 15]], np.uint8)
+    p = oracle.pack(q)
+    assert p.ravel().tolist() == [0x76543210, 0x0000000F, 0xF0000000]
+    rng = np.random.default_rng(2)
+    q = rng.integers(0, 16, size=(17, 96)).astype(np.uint8)
+    p = oracle.pack(q)
+    # two codes per byte, low nibble = even k (little-endian byte order of the words)
+    by = p.view(np.uint8).reshape(17, 48)
+    assert (by == (q[:, 0::2] | (q[:, 1::2] << 4))).all()
+    assert (oracle.unpack(p, 96) == q).all()
+
+
+# ----------------------------------------------------------------------------
+# Matmul: brute force, one-hot rows, adjoint identity, bias, column subsets
+# ----------------------------------------------------------------------------
+@pytest.fixture(scope="module")
+def tiny_case():
+    """The tiny correctness workload: M=4, K=512, N=256, g=64, seed 0."""
+    seed = 0
+    X = synth.activations(4, 512, seed)
+    W = synth.weights(256, 512, seed)
+    dY = synth.grads(4, 256, seed)
+    p, s, z = oracle.quantize_pack(W, "groupwise", 64)
+    return X, W, dY, p, s, z
+
+
+def test_matmul_matches_fp64_library_matmul(tiny_case):
+    X, W, dY, p, s, z = tiny_case
+    wh = oracle.dequant(p, s, z, "groupwise", 64, 512)
+    y64, ybf = oracle.linear(X, p, s, z, "groupwise", 64, 256, 512)
+    ref = bf16_value(X) @ wh.T
+    assert np.allclose(y64, ref, rtol=1e-12, atol=1e-12)
+    x64, _ = oracle.linear_t(dY, p, s, z, "groupwise", 64, 256, 512)
+    assert np.allclose(x64, bf16_value(dY) @ wh, rtol=1e-12, atol=1e-12)
+    assert (ybf == synth.f64_to_bf16_bits(y64)).all()
+
+
+def test_one_hot_rows_reproduce_dequantized_weights(tiny_case):
+    X, W, dY, p, s, z = tiny_case
+    wh = oracle.dequant(p, s, z, "groupwise", 64, 512)
+    ks = [0, 7, 63, 64, 200, 511]
+    E = np.zeros((len(ks), 512))
+    E[np.arange(len(ks)), ks] = 1.0
+    y64, ybf = oracle.linear(bf16(E), p, s, z, "groupwise", 64, 256, 512)
+    assert (y64 == wh[:, ks].T).all()
+    assert (ybf == synth.f64_to_bf16_bits(wh[:, ks].T)).all()
+    ns = [0, 1, 128, 255]
+    D = np.zeros((len(ns), 256))
+    D[np.arange(len(ns)), ns] = 1.0
+    x64, _ = oracle.linear_t(bf16(D), p, s, z, "groupwise", 64, 256, 512)
+    assert (x64 == wh[ns]).all()
+
+
+def test_adjoint_identity(tiny_case):
+    X, W, dY, p, s, z = tiny_case
+    y64, _ = oracle.linear(X, p, s, z, "groupwise", 64, 256, 512)
+    x64, _ = oracle.linear_t(dY, p, s, z, "groupwise", 64, 256, 512)
+    lhs = float(np.sum(y64 * bf16_value(dY)))
+    rhs = float(np.sum(bf16_value(X) * x64))
+    assert abs(lhs - rhs) <= 1e-9 * (abs(lhs) + 1.0)
+
+
+def test_bias_and_column_subsets(tiny_case):
+    X, W, dY, p, s, z = tiny_case
+    b = synth.bias(256, 0)
+    y0, _ = oracle.linear(X, p, s, z, "groupwise", 64, 256, 512)
+    yb, _ = oracle.linear(X, p, s, z, "groupwise", 64, 256, 512, bias=b)
+    assert np.allclose(yb - y0, bf16_value(b)[None, :], rtol=0, atol=1e-12)
+    cols = np.array([255, 3, 3, 100])
+    ys, _ = oracle.linear(X, p, s, z, "groupwise", 64, 256, 512, bias=b, cols=cols)
+    assert (ys == yb[:, cols]).all()
+    bk = synth.bias(512, 1)
+    x0, _ = oracle.linear_t(dY, p, s, z, "groupwise", 64, 256, 512)
+    xb, _ = oracle.linear_t(dY, p, s, z, "groupwise", 64, 256, 512, bias=bk)
+    assert np.allclose(xb - x0, bf16_value(bk)[None, :], rtol=0, atol=1e-12)
+    kc = np.array([511, 0, 64])
+    xs, _ = oracle.linear_t(dY, p, s, z, "groupwise", 64, 256, 512, bias=bk, cols=kc)
+    assert (xs == xb[:, kc]).all()
+
+
+@pytest.mark.parametrize("mode,g", [("groupwise", 64), ("rowwise", 0)])
+def test_fused_qkv_equivalence(mode, g):
+    """Fused Q/K/V weights concatenated along N (torchao "Add fused QKV HQQ
+    triton_mm test"): forward is the concatenation, transposed is the sum."""
+    K = 256
+    parts = [synth.weights(n, K, 30 + i) for i, n in enumerate([64, 32, 32])]
+    qs = [oracle.quantize_pack(Wp, mode, g) for Wp in parts]
+    Wf = np.concatenate(parts, axis=0)
+    pf, sf, zf = oracle.quantize_pack(Wf, mode, g)
+    assert (pf == np.concatenate([t[0] for t in qs])).all()
+    assert (sf == np.concatenate([t[1] for t in qs])).all()
+    X = synth.activations(3, K, 5)
+    yf, _ = oracle.linear(X, pf, sf, zf, mode, g, 128, K)
+    ys = [oracle.linear(X, *t, mode, g, Wp.shape[0], K)[0] for t, Wp in zip(qs, parts)]
+    assert (yf == np.concatenate(ys, axis=1)).all()
+    dY = synth.grads(3, 128, 6)
+    xf, _ = oracle.linear_t(dY, pf, sf, zf, mode, g, 128, K)
+    offs = [0, 64, 96, 128]
+    xs = [oracle.linear_t(dY[:, offs[i]:offs[i + 1]], *qs[i], mode, g, offs[i + 1] - offs[i], K)[0]
+          for i in range(3)]
+    assert np.allclose(xf, xs[0] + xs[1] + xs[2], rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# Soft band: the llm-quantization page's MAE column (not an exact pin)
+# ----------------------------------------------------------------------------
+def test_quantization_mae_soft_band():
+    rows = []
+    with open(os.path.join(GOLDEN, "llm_quantization_mae.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            mode, g, mae = line.split()
+            rows.append((mode, int(g), float(mae)))
+    W = synth.normal_bf16((2048, 2048), 0.0, 1.0, seed=8, stream=2)
+    wv = bf16_value(W)
+    for mode, g, page_mae in rows:
+        # the page's ROWWISE row disagrees with its own 4096-long groups (0.0969 vs
+        # 0.1189), so only GLOBAL and groups up to the row length are compared
+        if mode == "ROWWISE" or g > 2048:
+            continue
+        m = mode.lower()
+        q, s, z = oracle.quantize(W, m, g)
+        wh = oracle.dequant(oracle.pack(q), s, z, m, g, 2048)
+        mae = float(np.mean(np.abs(wv - wh)))
+        assert 0.75 * page_mae <= mae <= 1.25 * page_mae, (mode, g, mae, page_mae)
