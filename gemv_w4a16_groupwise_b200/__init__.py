@@ -1,0 +1,201 @@
+"""B200-native W4A16 weight-only matmul: thin Python binding of ``libw4a16.so``.
+
+Every step of the computation runs in the library's sm_100a kernels; this
+module only checks tensor metadata, passes device pointers and the current
+CUDA stream, and turns status codes into exceptions.  PyTorch provides
+device memory and streams.  There is no CPU fallback: without a CUDA device
+or without the built library every call raises.
+
+Entry points (same names as the C ABI in ``include/w4a16.h``):
+
+* :func:`w4_quantize_pack` -- bf16 W [N, K] -> packed int4 (int32 [N, K/8]),
+  fp16 scales and zeros
+* :func:`w4a16_gemm` -- Y = X . dequant(W)^T (or dX = dY . dequant(W) with
+  ``transposed=True``), optional bias
+* :func:`w4a16_gemv` -- the same for M <= 4 on CUDA cores
+* :func:`w4_workspace_bytes`, :func:`w4_device_error`
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+from . import build as _build
+
+W4_MODE_GLOBAL = 0
+W4_MODE_ROWWISE = 1
+W4_MODE_GROUPWISE = 2
+MODES = {"global": W4_MODE_GLOBAL, "rowwise": W4_MODE_ROWWISE, "groupwise": W4_MODE_GROUPWISE}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class W4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {library().w4_status_string(status).decode()}")
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def library():
+    """Load (building first if needed) the in-tree CUDA library."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.build()
+            lib = ctypes.CDLL(path)
+            P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+            lib.w4_status_string.argtypes = [I]
+            lib.w4_status_string.restype = ctypes.c_char_p
+            lib.w4_quantize_workspace_bytes.argtypes = [I, I, I]
+            lib.w4_quantize_workspace_bytes.restype = Z
+            lib.w4_quantize_pack.argtypes = [P, I, I, I, I, P, P, P, P, Z, P]
+            lib.w4_quantize_pack.restype = I
+            lib.w4_workspace_bytes.argtypes = [I, I, I, I]
+            lib.w4_workspace_bytes.restype = Z
+            for name in ("w4a16_gemm", "w4a16_gemv"):
+                f = getattr(lib, name)
+                f.argtypes = [P, I, I, I, P, P, P, I, I, P, I, P, P, Z, P]
+                f.restype = I
+            lib.w4_device_error.argtypes = [ctypes.POINTER(I)]
+            lib.w4_device_error.restype = I
+            lib.w4_launch_count.argtypes = []
+            lib.w4_launch_count.restype = ctypes.c_uint64
+            _lib = lib
+    return _lib
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _mode(mode) -> int:
+    return MODES[mode] if isinstance(mode, str) else int(mode)
+
+
+def _check_cuda(t, name, dtype, shape=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must live on a CUDA device (no CPU path exists)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _stream_ptr(device):
+    torch = _torch()
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def meta_shape(N: int, K: int, mode, group_size: int):
+    m = _mode(mode)
+    if m == W4_MODE_GLOBAL:
+        return (1, 1)
+    if m == W4_MODE_ROWWISE:
+        return (N, 1)
+    if group_size <= 0 or K % group_size:
+        raise ValueError(f"group_size {group_size} must divide K={K}")
+    return (N, K // group_size)
+
+
+def w4_quantize_workspace_bytes(N: int, K: int, mode) -> int:
+    return int(library().w4_quantize_workspace_bytes(N, K, _mode(mode)))
+
+
+def w4_workspace_bytes(M: int, N: int, K: int, transposed: bool = False) -> int:
+    return int(library().w4_workspace_bytes(M, N, K, int(bool(transposed))))
+
+
+def w4_quantize_pack(W, mode="groupwise", group_size: int = 128, out=None):
+    """Quantize bf16 W [N, K] (CUDA) -> (packed int32 [N, K/8], scales fp16, zeros fp16)."""
+    torch = _torch()
+    _check_cuda(W, "W", torch.bfloat16)
+    N, K = W.shape
+    shape = meta_shape(N, K, mode, group_size)
+    dev = W.device
+    if out is None:
+        packed = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
+        scales = torch.empty(shape, dtype=torch.float16, device=dev)
+        zeros = torch.empty(shape, dtype=torch.float16, device=dev)
+    else:
+        packed, scales, zeros = out
+    nws = w4_quantize_workspace_bytes(N, K, mode)
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = library().w4_quantize_pack(W.data_ptr(), N, K, _mode(mode), int(group_size),
+                                        packed.data_ptr(), scales.data_ptr(), zeros.data_ptr(),
+                                        ws.data_ptr(), nws, _stream_ptr(dev))
+    if st != 0:
+        raise W4Error(st, "w4_quantize_pack")
+    return packed, scales, zeros
+
+
+def _matmul(fname, A, packed, scales, zeros, mode, group_size, N, K, bias, transposed, out):
+    torch = _torch()
+    _check_cuda(A, "A", torch.bfloat16)
+    _check_cuda(packed, "packed", torch.int32, (N, K // 8))
+    _check_cuda(scales, "scales", torch.float16, meta_shape(N, K, mode, group_size))
+    _check_cuda(zeros, "zeros", torch.float16, meta_shape(N, K, mode, group_size))
+    if A.dim() != 2:
+        raise ValueError("A must be 2-D")
+    M = A.shape[0]
+    in_len, out_len = (N, K) if transposed else (K, N)
+    if A.shape[1] != in_len:
+        raise ValueError(f"A must have {in_len} columns, got {A.shape[1]}")
+    if bias is not None:
+        _check_cuda(bias, "bias", torch.bfloat16, (out_len,))
+    dev = A.device
+    if out is None:
+        out = torch.empty((M, out_len), dtype=torch.bfloat16, device=dev)
+    else:
+        _check_cuda(out, "out", torch.bfloat16, (M, out_len))
+    nws = w4_workspace_bytes(M, N, K, transposed)
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev) if nws else None
+    with torch.cuda.device(dev):
+        st = getattr(library(), fname)(
+            A.data_ptr(), M, N, K, packed.data_ptr(), scales.data_ptr(), zeros.data_ptr(),
+            _mode(mode), int(group_size), None if bias is None else bias.data_ptr(),
+            int(bool(transposed)), out.data_ptr(), None if ws is None else ws.data_ptr(), nws,
+            _stream_ptr(dev))
+    if st != 0:
+        raise W4Error(st, fname)
+    return out
+
+
+def w4a16_gemm(A, packed, scales, zeros, mode="groupwise", group_size: int = 128, *, N: int,
+               K: int, bias=None, transposed: bool = False, out=None):
+    """Y = A . dequant(W)^T  (A [M, K])  or, transposed, dX = A . dequant(W)  (A [M, N])."""
+    return _matmul("w4a16_gemm", A, packed, scales, zeros, mode, group_size, N, K, bias,
+                   transposed, out)
+
+
+def w4a16_gemv(A, packed, scales, zeros, mode="groupwise", group_size: int = 128, *, N: int,
+               K: int, bias=None, transposed: bool = False, out=None):
+    """Small-batch (M <= 4) path of :func:`w4a16_gemm` on CUDA cores."""
+    return _matmul("w4a16_gemv", A, packed, scales, zeros, mode, group_size, N, K, bias,
+                   transposed, out)
+
+
+def w4_launch_count() -> int:
+    """Kernel launches issued by the library in this process (host counter)."""
+    return int(library().w4_launch_count())
+
+
+def w4_device_error() -> int:
+    """Read and clear the device error word (synchronizes); 0 = no kernel gave up."""
+    code = ctypes.c_int(0)
+    st = library().w4_device_error(ctypes.byref(code))
+    if st not in (0, 6):
+        raise W4Error(st, "w4_device_error")
+    return int(code.value)

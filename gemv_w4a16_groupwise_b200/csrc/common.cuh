@@ -1,0 +1,76 @@
+// Shared device helpers of the W4A16 library (sm_100a only).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "this library targets sm_100a (B200) only"
+#endif
+
+namespace w4 {
+
+// Device-side error word: kernels whose waits are bounded record why they
+// gave up here instead of hanging (read and cleared by w4_device_error).
+__device__ unsigned int g_error_word;
+
+enum DeviceError : unsigned int {
+    kErrNone = 0,
+    kErrTimeoutTmaFull = 1,     // a consumer waited too long for a TMA stage
+    kErrTimeoutDequant = 2,     // the MMA issuer waited too long for dequantized tiles
+    kErrTimeoutEmpty = 3,       // the producer waited too long for a free stage
+    kErrTimeoutAccum = 4,       // the epilogue waited too long for the accumulator
+};
+
+__device__ __forceinline__ void record_error(unsigned int code) {
+    atomicCAS(&g_error_word, 0u, code);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
+    // (a & mask) | orv in one instruction
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(orv));
+    return r;
+}
+
+// Byte permute: result byte i = byte sel_i of {b:a} (PTX prmt default mode).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ldg_stream_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    return __ffma2_rn(a, b, c);
+}
+
+// Two codes of a packed word as bf16 "magic" values 128 + q: the low half
+// carries code i (bits 4i..4i+3 of w >> (4i)), the high half code i + 4.
+// Returned as the float pair (128 + q_i, 128 + q_{i+4}), both exact.
+template <int I>
+__device__ __forceinline__ float2 magic_pair(uint32_t w) {
+    const uint32_t v = lop3_and_or(w >> (4 * I), 0x000F000Fu, 0x43004300u);
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+
+}  // namespace w4

@@ -1,0 +1,204 @@
+// Quantize bf16 W [N, K] to uint4 codes and pack eight codes per uint32
+// along K (llm-quantization, "Objectives" 1; modes GLOBAL / ROWWISE /
+// GROUPWISE from its mode table).  Memory bound: W is read once (twice for
+// groups that do not fit a warp segment, the second read hitting L2), the
+// packed words and the fp16 scale / zero are written once.
+//
+// Per group, in IEEE fp32 with round-half-even and no contraction:
+//     s = fp16((max - min) / 15); if s == 0: s = fp16(max(|min|, 2^-14))
+//     z = clamp(rint(-min / s), 0, 15)
+//     q = clamp(rint(w / s) + z, 0, 15)
+// Clamps use fmaxf/fminf (a NaN lands on 0) and then convert to int, so a
+// negative zero never reaches the stored fp16 zero point.
+#pragma once
+
+#include "common.cuh"
+
+namespace w4 {
+
+struct GroupParams {
+    __half s;
+    float sf;   // float(s)
+    int z;
+};
+
+__device__ __forceinline__ GroupParams group_params_from_range(float mn, float mx) {
+    GroupParams p;
+    const float range = __fsub_rn(mx, mn);
+    __half s = __float2half_rn(__fdiv_rn(range, 15.0f));
+    if (__half2float(s) == 0.0f) s = __float2half_rn(fmaxf(fabsf(mn), 0x1p-14f));
+    p.s = s;
+    p.sf = __half2float(s);
+    const float zf = fminf(fmaxf(rintf(__fdiv_rn(-mn, p.sf)), 0.0f), 15.0f);
+    p.z = static_cast<int>(zf);
+    return p;
+}
+
+__device__ __forceinline__ uint32_t quantize_code(float w, const GroupParams& p) {
+    float t = __fadd_rn(rintf(__fdiv_rn(w, p.sf)), static_cast<float>(p.z));
+    t = fminf(fmaxf(t, 0.0f), 15.0f);
+    return static_cast<uint32_t>(static_cast<int>(t));
+}
+
+__device__ __forceinline__ void unpack8_bf16(const uint4 raw, float (&v)[8]) {
+    const uint32_t r[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(r[i] << 16);
+        v[2 * i + 1] = __uint_as_float(r[i] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack8(const float (&v)[8], const GroupParams& p) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) word |= quantize_code(v[i], p) << (4 * i);
+    return word;
+}
+
+// Groups of g = 8 * LPG elements, LPG a power of two <= 32: each thread owns
+// one 16-byte chunk (8 values, one packed word); the LPG lanes of a group
+// reduce min / max with shuffles inside their aligned lane segment.
+template <int LPG>
+__global__ void __launch_bounds__(256) quantize_segmented_kernel(
+    const uint16_t* __restrict__ W, long long total_words, uint32_t* __restrict__ packed,
+    __half* __restrict__ scales, __half* __restrict__ zeros) {
+    const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const bool active = t < total_words;
+    const long long tw = active ? t : (total_words - 1);
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(W) + tw);
+    float v[8];
+    unpack8_bf16(raw, v);
+    float mn = v[0], mx = v[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) {
+        mn = fminf(mn, v[i]);
+        mx = fmaxf(mx, v[i]);
+    }
+#pragma unroll
+    for (int off = 1; off < LPG; off <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    }
+    const GroupParams p = group_params_from_range(mn, mx);
+    if (!active) return;
+    packed[t] = pack8(v, p);
+    if ((threadIdx.x & (LPG - 1)) == 0) {
+        const long long grp = t / LPG;
+        scales[grp] = p.s;
+        zeros[grp] = __int2half_rn(p.z);
+    }
+}
+
+// Any group length g (multiple of 8): one warp per group, lanes stride over
+// the group's 16-byte chunks; min / max first, then a second pass quantizes
+// (the re-read is an L2 hit for all but the longest rows).
+__global__ void __launch_bounds__(256) quantize_warp_group_kernel(
+    const uint16_t* __restrict__ W, long long num_groups, int words_per_group,
+    uint32_t* __restrict__ packed, __half* __restrict__ scales, __half* __restrict__ zeros) {
+    const int lane = threadIdx.x & 31;
+    const long long grp =
+        static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (grp >= num_groups) return;
+    const long long base = grp * words_per_group;
+    const uint4* src = reinterpret_cast<const uint4*>(W) + base;
+    float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
+    for (int c = lane; c < words_per_group; c += 32) {
+        float v[8];
+        unpack8_bf16(__ldg(src + c), v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            mn = fminf(mn, v[i]);
+            mx = fmaxf(mx, v[i]);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    }
+    const GroupParams p = group_params_from_range(mn, mx);
+    for (int c = lane; c < words_per_group; c += 32) {
+        float v[8];
+        unpack8_bf16(__ldg(src + c), v);
+        packed[base + c] = pack8(v, p);
+    }
+    if (lane == 0) {
+        scales[grp] = p.s;
+        zeros[grp] = __int2half_rn(p.z);
+    }
+}
+
+// GLOBAL mode, pass 1: grid-stride min / max, one partial pair per block.
+__global__ void __launch_bounds__(256) global_minmax_kernel(const uint16_t* __restrict__ W,
+                                                            long long total_words,
+                                                            float2* __restrict__ partial) {
+    __shared__ float smn[8], smx[8];
+    float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
+    for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+         t < total_words; t += static_cast<long long>(gridDim.x) * blockDim.x) {
+        float v[8];
+        unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(W) + t), v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            mn = fminf(mn, v[i]);
+            mx = fmaxf(mx, v[i]);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        smn[warp] = mn;
+        smx[warp] = mx;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) {
+            mn = fminf(mn, smn[w]);
+            mx = fmaxf(mx, smx[w]);
+        }
+        partial[blockIdx.x] = make_float2(mn, mx);
+    }
+}
+
+// GLOBAL mode, pass 2: every block folds the partials (min / max are exact
+// and order-free, so all blocks agree), derives (s, z), quantizes a
+// grid-stride share of W; block 0 stores s and z.
+__global__ void __launch_bounds__(256) global_quantize_kernel(
+    const uint16_t* __restrict__ W, long long total_words, const float2* __restrict__ partial,
+    int num_partial, uint32_t* __restrict__ packed, __half* __restrict__ scales,
+    __half* __restrict__ zeros) {
+    __shared__ GroupParams sp;
+    if (threadIdx.x < 32) {
+        float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
+        for (int i = threadIdx.x; i < num_partial; i += 32) {
+            const float2 pm = partial[i];
+            mn = fminf(mn, pm.x);
+            mx = fmaxf(mx, pm.y);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
+            mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+        }
+        if (threadIdx.x == 0) sp = group_params_from_range(mn, mx);
+    }
+    __syncthreads();
+    const GroupParams p = sp;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        scales[0] = p.s;
+        zeros[0] = __int2half_rn(p.z);
+    }
+    for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+         t < total_words; t += static_cast<long long>(gridDim.x) * blockDim.x) {
+        float v[8];
+        unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(W) + t), v);
+        packed[t] = pack8(v, p);
+    }
+}
+
+}  // namespace w4

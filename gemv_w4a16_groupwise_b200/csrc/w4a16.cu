@@ -1,0 +1,588 @@
+// C-ABI entry points of the W4A16 library: argument validation, launch
+// planning, TMA descriptors, dispatch.  Declared in include/w4a16.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "quantize.cuh"
+#include "w4a16.h"
+
+namespace {
+
+using namespace w4;
+
+// ----------------------------------------------------------------- device info
+struct DeviceInfo {
+    int sms = 0;
+    int max_smem_optin = 0;
+};
+
+DeviceInfo device_info(int dev) {
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    static bool have[64] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < 64 && have[dev]) return cache[dev];
+    DeviceInfo d;
+    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (d.sms <= 0) {  // no usable device: keep the planners well defined
+        cudaGetLastError();
+        d.sms = 1;
+        d.max_smem_optin = 0;
+        return d;
+    }
+    if (dev >= 0 && dev < 64) {
+        cache[dev] = d;
+        have[dev] = true;
+    }
+    return d;
+}
+
+int current_device() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return dev;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per (device, kernel).
+cudaError_t ensure_smem(const void* fn, size_t bytes) {
+    static std::mutex mu;
+    struct Entry {
+        int dev;
+        const void* fn;
+        size_t bytes;
+    };
+    static Entry table[512];
+    static int count = 0;
+    const int dev = current_device();
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < count; ++i)
+        if (table[i].dev == dev && table[i].fn == fn && table[i].bytes >= bytes) return cudaSuccess;
+    cudaError_t e =
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    if (e != cudaSuccess) return e;
+    if (count < 512) table[count++] = Entry{dev, fn, bytes};
+    return cudaSuccess;
+}
+
+// ------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `esize`-byte elements, box [box_rows,
+// box_cols], swizzle span 0 (none), 64 or 128 bytes.  Out-of-range elements
+// read as 0.
+bool make_map_2d(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, int esize,
+                 uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+                 int swizzle) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[2] = {cols, rows};
+    cuuint64_t gstride[1] = {cols * static_cast<uint64_t>(esize)};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dt, 2, const_cast<void*>(ptr), gdim, gstride, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                    : swizzle == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                    : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ validation
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Meta {
+    int g;       // group length along K (K for ROWWISE / GLOBAL)
+    int G;       // groups per row
+    int sz_row;  // row stride of the scale / zero arrays
+};
+
+w4_status check_mode(int K, int mode, int group_size, Meta* meta) {
+    if (mode == W4_MODE_GLOBAL) {
+        *meta = Meta{K, 1, 0};
+        return W4_OK;
+    }
+    if (mode == W4_MODE_ROWWISE) {
+        *meta = Meta{K, 1, 1};
+        return W4_OK;
+    }
+    if (mode == W4_MODE_GROUPWISE) {
+        if (group_size < 8 || group_size % 8 != 0 || K % group_size != 0) return W4_ERR_INVALID_ARG;
+        *meta = Meta{group_size, K / group_size, K / group_size};
+        return W4_OK;
+    }
+    return W4_ERR_INVALID_ARG;
+}
+
+std::atomic<uint64_t> g_launches{0};
+
+// Called right after every kernel launch: counts it and maps a launch
+// failure to W4_ERR_CUDA.
+w4_status launch_status() {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+int gcd_int(int a, int b) {
+    while (b) {
+        const int t = a % b;
+        a = b;
+        b = t;
+    }
+    return a;
+}
+
+// -------------------------------------------------------- GEMV planning
+struct FwdPlan {
+    bool tma = false;
+    int F = 0, TK = 0, splits = 1, row_tiles = 0, units = 0, grid = 0;
+    size_t smem = 0, ws = 0;
+};
+
+FwdPlan plan_fwd(int M, int N, int K, const Meta& meta, int sms) {
+    FwdPlan p;
+    p.tma = (K % 32 == 0) && (meta.g % 32 == 0);
+    if (!p.tma) return p;
+    p.F = gcd_int(meta.g, kGemvBoxK);
+    p.row_tiles = (N + kGemvTileRows - 1) / kGemvTileRows;
+    const int tk_max = (M == 1) ? 16384 : (M == 2) ? 8192 : (M == 3) ? 5120 : 4096;
+    const int k_pad = (K + kGemvBoxK - 1) / kGemvBoxK * kGemvBoxK;
+    const int s_min = (k_pad + tk_max - 1) / tk_max;
+    const int s_max = std::max(s_min, k_pad / kGemvBoxK);
+    double best = -1.0;
+    for (int s = s_min; s <= std::min(s_max, s_min * 16); ++s) {
+        int tk = (k_pad + s - 1) / s;
+        tk = (tk + kGemvBoxK - 1) / kGemvBoxK * kGemvBoxK;
+        const int se = (K + tk - 1) / tk;
+        const long long units = static_cast<long long>(p.row_tiles) * se;
+        const long long waves = (units + sms - 1) / sms;
+        // per-SM serial bytes vs the ideal even share of the weights
+        const double ideal = static_cast<double>(N) * K / 2.0 / sms;
+        const double real = static_cast<double>(waves) * tk * kGemvTileRows / 2.0;
+        double eff = ideal / real;
+        const int nb = tk / kGemvBoxK;
+        if (nb < kGemvConsumerWarps) eff *= 0.5 + 0.5 * nb / kGemvConsumerWarps;  // idle warps
+        if (se > 1) eff *= 1.0 - std::min(0.5, 16.0 * se * M / K);               // partials
+        if (eff > best * 1.02) {
+            best = eff;
+            p.TK = tk;
+            p.splits = se;
+            p.units = static_cast<int>(units);
+        }
+    }
+    p.grid = std::min(p.units, sms);
+    p.smem = gemv_fwd_smem_bytes(M, p.TK, p.F);
+    p.ws = p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * sizeof(float) : 0;
+    return p;
+}
+
+struct TPlan {
+    int splits = 1, rows_per_split = 0;
+    size_t ws = 0;
+};
+
+TPlan plan_t(int M, int N, int K, int sms) {
+    TPlan p;
+    const int W8 = K / 8;
+    const int col_tiles = (W8 + kGemvTWordsPerCta - 1) / kGemvTWordsPerCta;
+    int splits = (sms * 6 + col_tiles - 1) / col_tiles;
+    splits = std::min(splits, std::max(1, N / (320 * M)));  // partial traffic <= ~5%
+    splits = std::max(1, std::min(splits, (N + 31) / 32));
+    p.rows_per_split = (N + splits - 1) / splits;
+    p.splits = (N + p.rows_per_split - 1) / p.rows_per_split;
+    p.ws = p.splits > 1 ? static_cast<size_t>(p.splits) * M * K * sizeof(float) : 0;
+    return p;
+}
+
+size_t gemv_workspace(int M, int N, int K, int transposed, int sms) {
+    if (transposed) return plan_t(M, N, K, sms).ws;
+    // the group structure only changes the fold granule, not the split
+    Meta meta{K, 1, 1};
+    FwdPlan p = plan_fwd(M, N, K, meta, sms);
+    size_t ws = p.ws;
+    Meta meta32{32, K / 32, K / 32};
+    if (K % 32 == 0) ws = std::max(ws, plan_fwd(M, N, K, meta32, sms).ws);
+    return ws;
+}
+
+template <int M>
+w4_status launch_gemv_fwd(const FwdPlan& p, const CUtensorMap& map, const GemvFwdArgs& a,
+                          cudaStream_t st) {
+    const void* fn = nullptr;
+    switch (p.F) {
+        case 32: fn = reinterpret_cast<const void*>(gemv_fwd_tma_kernel<M, 32>); break;
+        case 64: fn = reinterpret_cast<const void*>(gemv_fwd_tma_kernel<M, 64>); break;
+        case 128: fn = reinterpret_cast<const void*>(gemv_fwd_tma_kernel<M, 128>); break;
+        default: return W4_ERR_UNSUPPORTED;
+    }
+    if (ensure_smem(fn, p.smem) != cudaSuccess) return W4_ERR_CUDA;
+    switch (p.F) {
+        case 32: gemv_fwd_tma_kernel<M, 32><<<p.grid, kGemvThreads, p.smem, st>>>(map, a); break;
+        case 64: gemv_fwd_tma_kernel<M, 64><<<p.grid, kGemvThreads, p.smem, st>>>(map, a); break;
+        case 128: gemv_fwd_tma_kernel<M, 128><<<p.grid, kGemvThreads, p.smem, st>>>(map, a); break;
+    }
+    return launch_status();
+}
+
+w4_status run_gemv_fwd(const void* A, int M, int N, int K, const uint32_t* packed, const void* S,
+                       const void* Z, const Meta& meta, const void* bias, void* Y, void* ws,
+                       size_t ws_bytes, cudaStream_t st) {
+    const DeviceInfo di = device_info(current_device());
+    const FwdPlan p = plan_fwd(M, N, K, meta, di.sms);
+    GemvFwdArgs a;
+    a.X = static_cast<const uint16_t*>(A);
+    a.S = static_cast<const __half*>(S);
+    a.Z = static_cast<const __half*>(Z);
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.Y = static_cast<uint16_t*>(Y);
+    a.partial = static_cast<float*>(ws);
+    a.N = N;
+    a.K = K;
+    a.g = meta.g;
+    a.G = meta.G;
+    a.sz_row = meta.sz_row;
+    a.TK = p.TK;
+    a.splits = p.splits;
+    a.row_tiles = p.row_tiles;
+    a.units = p.units;
+    if (!p.tma) {
+        const int blocks = (N * 32 + 255) / 256;
+        switch (M) {
+            case 1: gemv_fwd_simple_kernel<1><<<blocks, 256, 0, st>>>(a, packed); break;
+            case 2: gemv_fwd_simple_kernel<2><<<blocks, 256, 0, st>>>(a, packed); break;
+            case 3: gemv_fwd_simple_kernel<3><<<blocks, 256, 0, st>>>(a, packed); break;
+            case 4: gemv_fwd_simple_kernel<4><<<blocks, 256, 0, st>>>(a, packed); break;
+        }
+        return launch_status();
+    }
+    if (p.ws > ws_bytes || (p.ws > 0 && ws == nullptr)) return W4_ERR_WORKSPACE;
+    if (p.smem > static_cast<size_t>(di.max_smem_optin)) return W4_ERR_UNSUPPORTED;
+    CUtensorMap map;
+    if (!make_map_2d(&map, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, kGemvTileRows,
+                     kGemvBoxWords, 64))
+        return W4_ERR_CUDA;
+    w4_status s = W4_OK;
+    switch (M) {
+        case 1: s = launch_gemv_fwd<1>(p, map, a, st); break;
+        case 2: s = launch_gemv_fwd<2>(p, map, a, st); break;
+        case 3: s = launch_gemv_fwd<3>(p, map, a, st); break;
+        case 4: s = launch_gemv_fwd<4>(p, map, a, st); break;
+    }
+    if (s != W4_OK) return s;
+    if (p.splits > 1) {
+        const long long total = static_cast<long long>(M) * N;
+        const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, di.sms * 8));
+        splits_finalize_kernel<<<blocks, 256, 0, st>>>(a.partial, p.splits, M, N, a.bias, a.Y);
+        return launch_status();
+    }
+    return W4_OK;
+}
+
+w4_status run_gemv_t(const void* A, int M, int N, int K, const uint32_t* packed, const void* S,
+                     const void* Z, const Meta& meta, const void* bias, void* Y, void* ws,
+                     size_t ws_bytes, cudaStream_t st) {
+    const DeviceInfo di = device_info(current_device());
+    const TPlan p = plan_t(M, N, K, di.sms);
+    if (p.ws > ws_bytes || (p.ws > 0 && ws == nullptr)) return W4_ERR_WORKSPACE;
+    GemvTArgs a;
+    a.dY = static_cast<const uint16_t*>(A);
+    a.packed = packed;
+    a.S = static_cast<const __half*>(S);
+    a.Z = static_cast<const __half*>(Z);
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.dX = static_cast<uint16_t*>(Y);
+    a.partial = static_cast<float*>(ws);
+    a.N = N;
+    a.K = K;
+    a.g = meta.g;
+    a.G = meta.G;
+    a.sz_row = meta.sz_row;
+    a.rows_per_split = p.rows_per_split;
+    a.splits = p.splits;
+    const dim3 grid((K / 8 + kGemvTWordsPerCta - 1) / kGemvTWordsPerCta, p.splits);
+    switch (M) {
+        case 1: gemv_t_kernel<1><<<grid, kGemvTThreads, 0, st>>>(a); break;
+        case 2: gemv_t_kernel<2><<<grid, kGemvTThreads, 0, st>>>(a); break;
+        case 3: gemv_t_kernel<3><<<grid, kGemvTThreads, 0, st>>>(a); break;
+        case 4: gemv_t_kernel<4><<<grid, kGemvTThreads, 0, st>>>(a); break;
+    }
+    w4_status s = launch_status();
+    if (s != W4_OK) return s;
+    if (p.splits > 1) {
+        const long long total = static_cast<long long>(M) * K;
+        const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, di.sms * 8));
+        splits_finalize_kernel<<<blocks, 256, 0, st>>>(a.partial, p.splits, M, K, a.bias, a.dX);
+        return launch_status();
+    }
+    return W4_OK;
+}
+
+// Common argument checks of the matmul entry points, in the documented order.
+w4_status check_matmul(const void* A, int M, int N, int K, const uint32_t* packed, const void* S,
+                       const void* Z, int mode, int group_size, const void* bias, void* Y,
+                       Meta* meta) {
+    if (M <= 0 || N <= 0 || K <= 0) return W4_ERR_INVALID_ARG;
+    if (K % 8 != 0) return W4_ERR_INVALID_ARG;
+    w4_status s = check_mode(K, mode, group_size, meta);
+    if (s != W4_OK) return s;
+    if (!A || !packed || !S || !Z || !Y) return W4_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(packed) || !aligned16(S) || !aligned16(Z) || !aligned16(Y) ||
+        (bias && !aligned16(bias)))
+        return W4_ERR_ALIGNMENT;
+    return W4_OK;
+}
+
+w4_status run_gemv(const void* A, int M, int N, int K, const uint32_t* packed, const void* S,
+                   const void* Z, const Meta& meta, const void* bias, int transposed, void* Y,
+                   void* ws, size_t ws_bytes, cudaStream_t st) {
+    return transposed ? run_gemv_t(A, M, N, K, packed, S, Z, meta, bias, Y, ws, ws_bytes, st)
+                      : run_gemv_fwd(A, M, N, K, packed, S, Z, meta, bias, Y, ws, ws_bytes, st);
+}
+
+
+// ---------------------------------------------------------- tensor-core GEMM
+size_t gemm_tc_workspace_bytes(int M, int N, int K, int transposed, int sms) {
+    (void)M;
+    (void)N;
+    (void)K;
+    (void)transposed;
+    (void)sms;
+    return 0;
+}
+
+int tc_pick_bn(int M) {
+    if (M <= 16) return 16;
+    if (M <= 32) return 32;
+    if (M <= 64) return 64;
+    if (M <= 128) return 128;
+    return 256;
+}
+
+template <bool TR, int BN, bool PWG>
+w4_status launch_tc(const CUtensorMap& pm, const CUtensorMap& bm, const TcArgs& a, dim3 grid,
+                    size_t smem, cudaStream_t st) {
+    const void* fn = reinterpret_cast<const void*>(gemm_tc_kernel<TR, BN, PWG>);
+    if (ensure_smem(fn, smem) != cudaSuccess) return W4_ERR_CUDA;
+    gemm_tc_kernel<TR, BN, PWG><<<grid, kTcThreads, smem, st>>>(pm, bm, a);
+    return launch_status();
+}
+
+template <bool TR, bool PWG>
+w4_status launch_tc_bn(int BN, const CUtensorMap& pm, const CUtensorMap& bm, const TcArgs& a,
+                       dim3 grid, size_t smem, cudaStream_t st) {
+    switch (BN) {
+        case 16: return launch_tc<TR, 16, PWG>(pm, bm, a, grid, smem, st);
+        case 32: return launch_tc<TR, 32, PWG>(pm, bm, a, grid, smem, st);
+        case 64: return launch_tc<TR, 64, PWG>(pm, bm, a, grid, smem, st);
+        case 128: return launch_tc<TR, 128, PWG>(pm, bm, a, grid, smem, st);
+        default: return launch_tc<TR, 256, PWG>(pm, bm, a, grid, smem, st);
+    }
+}
+
+w4_status run_gemm_tc(const TcProblem& p, cudaStream_t st) {
+    if (p.K % 32 != 0) return W4_ERR_UNSUPPORTED;      // packed rows must be 16-byte strided
+    if (p.transposed && p.N % 8 != 0) return W4_ERR_UNSUPPORTED;  // dY rows 16-byte strided
+    const DeviceInfo di = device_info(current_device());
+    const int BN = tc_pick_bn(p.M);
+    const int stage = tc_stage_bytes(BN);
+    const size_t fixed = 1024 + 64;
+    int stages = static_cast<int>((static_cast<size_t>(di.max_smem_optin) - fixed - 64) / (stage + 24));
+    stages = std::min(stages, 8);
+    if (stages < 2) return W4_ERR_UNSUPPORTED;
+    const size_t smem = fixed + static_cast<size_t>(stages) * stage + static_cast<size_t>(3 * stages + 1) * 8 + 16;
+    const bool tr = p.transposed != 0;
+    CUtensorMap pm, bm;
+    // packed weights [N, K/8] uint32: box 8 words x 128 rows (forward) or
+    // 16 words x 64 rows (transposed); activations [M, K] or dY [M, N] bf16,
+    // box 64 x BN with the 128-byte swizzle the MMA descriptors expect
+    bool ok = tr ? make_map_2d(&pm, p.packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, p.N, p.K / 8, 64, 16, 0)
+                 : make_map_2d(&pm, p.packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, p.N, p.K / 8, 128, 8, 0);
+    ok = ok && make_map_2d(&bm, p.A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.M, tr ? p.N : p.K, BN, 64, 128);
+    if (!ok) return W4_ERR_CUDA;
+    TcArgs a;
+    a.S = static_cast<const __half*>(p.S);
+    a.Z = static_cast<const __half*>(p.Z);
+    a.bias = static_cast<const uint16_t*>(p.bias);
+    a.Y = static_cast<uint16_t*>(p.Y);
+    a.M = p.M;
+    a.N = p.N;
+    a.K = p.K;
+    a.g = p.g;
+    a.G = p.G;
+    a.sz_row = p.sz_row;
+    a.stages = stages;
+    const int L_out = tr ? p.K : p.N;
+    const dim3 grid((p.M + BN - 1) / BN, (L_out + kTcBM - 1) / kTcBM);
+    if (grid.y > 65535) return W4_ERR_UNSUPPORTED;
+    const bool pwg = (p.g % 32) != 0;
+    if (tr) return pwg ? launch_tc_bn<true, true>(BN, pm, bm, a, grid, smem, st)
+                       : launch_tc_bn<true, false>(BN, pm, bm, a, grid, smem, st);
+    return pwg ? launch_tc_bn<false, true>(BN, pm, bm, a, grid, smem, st)
+               : launch_tc_bn<false, false>(BN, pm, bm, a, grid, smem, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* w4_status_string(int status) {
+    switch (status) {
+        case W4_OK: return "W4_OK";
+        case W4_ERR_INVALID_ARG: return "W4_ERR_INVALID_ARG: a size, mode or group size is out of range";
+        case W4_ERR_UNSUPPORTED: return "W4_ERR_UNSUPPORTED: valid arguments that no kernel here handles";
+        case W4_ERR_ALIGNMENT: return "W4_ERR_ALIGNMENT: a pointer is not 16-byte aligned";
+        case W4_ERR_WORKSPACE: return "W4_ERR_WORKSPACE: workspace missing or too small";
+        case W4_ERR_CUDA: return "W4_ERR_CUDA: a CUDA call or kernel launch failed";
+        case W4_ERR_TIMEOUT: return "W4_ERR_TIMEOUT: a kernel abandoned a bounded wait";
+        default: return "unknown w4_status";
+    }
+}
+
+size_t w4_quantize_workspace_bytes(int N, int K, int mode) {
+    (void)N;
+    (void)K;
+    return mode == W4_MODE_GLOBAL ? 1024 * sizeof(float2) : 0;
+}
+
+w4_status w4_quantize_pack(const void* W, int N, int K, int mode, int group_size, uint32_t* packed,
+                           void* scales, void* zeros, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+    if (N <= 0 || K <= 0 || K % 8 != 0) return W4_ERR_INVALID_ARG;
+    Meta meta;
+    w4_status s = check_mode(K, mode, group_size, &meta);
+    if (s != W4_OK) return s;
+    if (!W || !packed || !scales || !zeros) return W4_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(packed) || !aligned16(scales) || !aligned16(zeros))
+        return W4_ERR_ALIGNMENT;
+    const size_t need = w4_quantize_workspace_bytes(N, K, mode);
+    if (workspace_bytes < need || (need > 0 && !workspace)) return W4_ERR_WORKSPACE;
+    if (need > 0 && !aligned16(workspace)) return W4_ERR_ALIGNMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const uint16_t* w = static_cast<const uint16_t*>(W);
+    __half* sc = static_cast<__half*>(scales);
+    __half* ze = static_cast<__half*>(zeros);
+    const long long total_words = static_cast<long long>(N) * (K / 8);
+    const DeviceInfo di = device_info(current_device());
+    if (mode == W4_MODE_GLOBAL) {
+        const int blocks = static_cast<int>(
+            std::min<long long>(1024, std::min<long long>((total_words + 255) / 256, di.sms * 4)));
+        float2* part = static_cast<float2*>(workspace);
+        global_minmax_kernel<<<blocks, 256, 0, st>>>(w, total_words, part);
+        s = launch_status();
+        if (s != W4_OK) return s;
+        const int qblocks =
+            static_cast<int>(std::min<long long>((total_words + 255) / 256, di.sms * 8));
+        global_quantize_kernel<<<qblocks, 256, 0, st>>>(w, total_words, part, blocks, packed, sc, ze);
+        return launch_status();
+    }
+    const int lpg = meta.g / 8;
+    const int blocks = static_cast<int>((total_words + 255) / 256);
+    switch (lpg) {
+        case 1: quantize_segmented_kernel<1><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        case 2: quantize_segmented_kernel<2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        case 4: quantize_segmented_kernel<4><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        case 8: quantize_segmented_kernel<8><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        case 16: quantize_segmented_kernel<16><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        case 32: quantize_segmented_kernel<32><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        default: {
+            const long long groups = total_words / lpg;
+            const int gblocks = static_cast<int>((groups + 7) / 8);
+            quantize_warp_group_kernel<<<gblocks, 256, 0, st>>>(w, groups, lpg, packed, sc, ze);
+        }
+    }
+    return launch_status();
+}
+
+size_t w4_workspace_bytes(int M, int N, int K, int transposed) {
+    if (M <= 0 || N <= 0 || K <= 0 || K % 8 != 0) return 0;
+    const int sms = device_info(current_device()).sms;
+    if (M <= 4) return gemv_workspace(M, N, K, transposed, sms);
+    return gemm_tc_workspace_bytes(M, N, K, transposed, sms);
+}
+
+w4_status w4a16_gemv(const void* A, int M, int N, int K, const uint32_t* packed,
+                     const void* scales, const void* zeros, int mode, int group_size,
+                     const void* bias, int transposed, void* Y, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+    Meta meta;
+    w4_status s = check_matmul(A, M, N, K, packed, scales, zeros, mode, group_size, bias, Y, &meta);
+    if (s != W4_OK) return s;
+    if (M > 4) return W4_ERR_INVALID_ARG;
+    if (workspace && !aligned16(workspace)) return W4_ERR_ALIGNMENT;
+    return run_gemv(A, M, N, K, packed, scales, zeros, meta, bias, transposed, Y, workspace,
+                    workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+w4_status w4a16_gemm(const void* A, int M, int N, int K, const uint32_t* packed,
+                     const void* scales, const void* zeros, int mode, int group_size,
+                     const void* bias, int transposed, void* Y, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+    Meta meta;
+    w4_status s = check_matmul(A, M, N, K, packed, scales, zeros, mode, group_size, bias, Y, &meta);
+    if (s != W4_OK) return s;
+    if (workspace && !aligned16(workspace)) return W4_ERR_ALIGNMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (M <= 4)
+        return run_gemv(A, M, N, K, packed, scales, zeros, meta, bias, transposed, Y, workspace,
+                        workspace_bytes, st);
+    const int sms = device_info(current_device()).sms;
+    if (workspace_bytes < gemm_tc_workspace_bytes(M, N, K, transposed, sms))
+        return W4_ERR_WORKSPACE;
+    TcProblem pr;
+    pr.A = A;
+    pr.M = M;
+    pr.N = N;
+    pr.K = K;
+    pr.packed = packed;
+    pr.S = scales;
+    pr.Z = zeros;
+    pr.g = meta.g;
+    pr.G = meta.G;
+    pr.sz_row = meta.sz_row;
+    pr.bias = bias;
+    pr.transposed = transposed;
+    pr.Y = Y;
+    pr.sms = sms;
+    return run_gemm_tc(pr, st);
+}
+
+uint64_t w4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+w4_status w4_device_error(int* code) {
+    if (!code) return W4_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return W4_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, w4::g_error_word, sizeof v) != cudaSuccess) return W4_ERR_CUDA;
+    if (cudaMemcpyToSymbol(w4::g_error_word, &zero, sizeof zero) != cudaSuccess) return W4_ERR_CUDA;
+    *code = static_cast<int>(v);
+    return v ? W4_ERR_TIMEOUT : W4_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,152 @@
+/*
+ * w4a16.h -- C ABI of the B200 (sm_100a) weight-only int4 matmul library.
+ *
+ * The operation: Y = X_bf16 . dequant(W_int4)^T, where each 4-bit code q
+ * of W carries a per-group fp16 scale s and zero point z and dequantizes as
+ * w = (q - z) * s (llm-quantization, "Objectives" 1 and 2: quantize FP16 to
+ * INT4 and pack into INT8/INT32; Y = X_bf16 @ W_int4^T).  The same packed
+ * weights also serve the transposed product dX = dY . dequant(W) used in
+ * fine-tuning backward ("Re-write HQQ Fused Gemm Transpose": pack once, pass
+ * transposed=True, no repacking and no reshaping of scales or zeros).
+ *
+ * Conventions shared by every entry point
+ *   - All array arguments are DEVICE pointers owned by the caller; the
+ *     library never frees or keeps them.  Calls are asynchronous on
+ *     `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *   - N and K always name W's dimensions: W is [N, K] row-major.
+ *   - packed: uint32 [N, K/8]; code i of word j of row n holds k = 8j + i
+ *     in bits 4i..4i+3 (byte-identical to two codes per byte, low nibble =
+ *     even k).
+ *   - scales / zeros: fp16 [N, K/g] row-major (GROUPWISE), [N, 1]
+ *     (ROWWISE), [1, 1] (GLOBAL).  zeros hold integer values 0..15.
+ *   - Activations, gradients, bias and outputs are bf16, row-major, dense.
+ *   - Accumulation is fp32; each output is rounded to bf16 once, after the
+ *     optional bias has been added in fp32.
+ *   - Arguments are validated before any launch, in the order listed in
+ *     each comment; the first failure is returned and nothing is launched.
+ *     After each launch the library checks cudaGetLastError() and returns
+ *     W4_ERR_CUDA if it reports a launch failure.
+ *   - The library allocates no device memory.  Kernels that need scratch
+ *     take it from the caller's `workspace`; query the size first.
+ *   - Pointers must be 16-byte aligned (W4_ERR_ALIGNMENT otherwise).
+ */
+#ifndef W4A16_H
+#define W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum w4_status {
+    W4_OK = 0,
+    W4_ERR_INVALID_ARG = 1,  /* a size, mode or group size out of range */
+    W4_ERR_UNSUPPORTED = 2,  /* valid, but no kernel here handles it */
+    W4_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned */
+    W4_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
+    W4_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
+    W4_ERR_TIMEOUT = 6       /* a kernel gave up on a bounded wait (see w4_device_error) */
+} w4_status;
+
+typedef enum w4_mode {
+    W4_MODE_GLOBAL = 0,    /* one (s, z) for the whole matrix */
+    W4_MODE_ROWWISE = 1,   /* one (s, z) per row; group_size is ignored (g = K) */
+    W4_MODE_GROUPWISE = 2  /* one (s, z) per g consecutive k of a row */
+} w4_mode;
+
+/*
+ * Workspace bytes w4_quantize_pack needs for (N, K, mode): non-zero only for
+ * GLOBAL, whose min/max runs as a separate grid-wide pass.
+ */
+size_t w4_quantize_workspace_bytes(int N, int K, int mode);
+
+/*
+ * w4_quantize_pack -- quantize bf16 W [N, K] to uint4 and pack eight codes
+ * per uint32 along K (llm-quantization, "Objectives" 1: a kernel that
+ * quantizes a 2-D matrix to INT4 and packs it into INT32; modes GLOBAL,
+ * ROWWISE and GROUPWISE from its mode table).  Per group:
+ *     s = fp16((max - min) / 15); if s == 0: s = fp16(max(|min|, 2^-14))
+ *     z = clamp(rint(-min / s), 0, 15)
+ *     q = clamp(rint(w / s) + z, 0, 15)
+ * in IEEE fp32 with round-half-even; results are bit-exact against the
+ * CPU oracle.  Inputs must be finite and satisfy (max - min) / 15 <= 65504.
+ *
+ * Outputs: packed uint32 [N, K/8]; scales, zeros fp16 (see conventions).
+ * Validation: N, K > 0; K % 8 == 0; mode in range; GROUPWISE needs
+ * group_size >= 8, group_size % 8 == 0, K % group_size == 0; pointers
+ * non-NULL and 16-byte aligned; workspace_bytes >=
+ * w4_quantize_workspace_bytes(N, K, mode).
+ */
+w4_status w4_quantize_pack(const void *W, int N, int K, int mode, int group_size,
+                           uint32_t *packed, void *scales, void *zeros,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Workspace bytes w4a16_gemm / w4a16_gemv need for this problem (0 when the
+ * chosen kernels need none).  Depends only on (M, N, K, transposed).
+ */
+size_t w4_workspace_bytes(int M, int N, int K, int transposed);
+
+/*
+ * w4a16_gemm -- weight-only int4 matmul with in-register dequantization.
+ *   transposed = 0:  A = X  [M, K] -> Y  [M, N]:  Y  = X  . w_hat^T (+ bias[N])
+ *       (llm-quantization, "Objectives" 2: Y = X_bf16 @ W_int4^T)
+ *   transposed = 1:  A = dY [M, N] -> Y = dX [M, K]:  dX = dY . w_hat (+ bias[K])
+ *       ("Re-write HQQ Fused Gemm Transpose": the backward product from the
+ *       same packed weights, scales and zeros)
+ *   bias: bf16 vector over the output columns, or NULL (vLLM "Adding bias
+ *       epilogue support for cutlass_scaled_mm": bias dtype = output dtype).
+ * Fused QKV weights (torchao "Add fused QKV HQQ triton_mm test") are just
+ * the row-wise concatenation of the Q, K and V packed weights, scales and
+ * zeros; they need no special call.
+ * M <= 4 runs the CUDA-core GEMV kernels (same results as w4a16_gemv); M > 4
+ * runs the tcgen05 tensor-core kernel.
+ * Validation: M, N, K > 0; K % 8 == 0; mode/group rules as for
+ * w4_quantize_pack; pointers (bias may be NULL) non-NULL and 16-byte
+ * aligned; workspace_bytes >= w4_workspace_bytes(M, N, K, transposed).
+ * The tensor-core path also needs K % 32 == 0 and, when transposed,
+ * N % 8 == 0 (W4_ERR_UNSUPPORTED otherwise).
+ */
+w4_status w4a16_gemm(const void *A, int M, int N, int K, const uint32_t *packed,
+                     const void *scales, const void *zeros, int mode, int group_size,
+                     const void *bias, int transposed, void *Y,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * w4a16_gemv -- the small-batch path on CUDA cores (TensorRT-LLM "Modify
+ * small-batched weight only quantization": batch <= 4 GEMV bound by global
+ * memory loads).  Same arguments and results as w4a16_gemm; M must be 1..4
+ * (W4_ERR_INVALID_ARG otherwise).
+ */
+w4_status w4a16_gemv(const void *A, int M, int N, int K, const uint32_t *packed,
+                     const void *scales, const void *zeros, int mode, int group_size,
+                     const void *bias, int transposed, void *Y,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *w4_status_string(int status);
+
+/*
+ * w4_device_error -- read and clear the device-side error word of the
+ * current device.  Kernels whose waits are bounded set it instead of
+ * hanging; *code receives 0 when no kernel gave up.  Synchronizes the
+ * device.  Returns W4_ERR_TIMEOUT when *code != 0, W4_ERR_CUDA on a CUDA
+ * failure, W4_OK otherwise.
+ */
+w4_status w4_device_error(int *code);
+
+/*
+ * w4_launch_count -- number of kernel launches this library has issued in
+ * the calling process since it was loaded (all devices, all entry points).
+ * Host-side counter; launches replayed from a captured CUDA graph are not
+ * re-counted.
+ */
+uint64_t w4_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H */

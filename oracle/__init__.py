@@ -74,6 +74,8 @@ def _load():
             lib.oracle_groups_per_row.restype = L
             lib.oracle_f64_to_bf16.argtypes = [ctypes.c_double]
             lib.oracle_f64_to_bf16.restype = ctypes.c_uint16
+            lib.oracle_num_threads.argtypes = []
+            lib.oracle_num_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -104,6 +106,11 @@ def meta_shape(N: int, K: int, mode, g: int):
     if g <= 0 or K % g:
         raise ValueError(f"group size {g} must be positive and divide K={K}")
     return (N, K // g)
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle's parallel loops use."""
+    return int(_load().oracle_num_threads())
 
 
 def f64_to_bf16(x: float) -> int:

@@ -41,12 +41,16 @@
  * thread count.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <string.h>
 
 #define MODE_GLOBAL 0
 #define MODE_ROWWISE 1
 #define MODE_GROUPWISE 2
+
+/* Threads an OpenMP region of this library uses (for reporting). */
+int oracle_num_threads(void) { return omp_get_max_threads(); }
 
 /* ---------------------------------------------------------------- formats */
 
