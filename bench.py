@@ -77,6 +77,21 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(dist, value: float, device) -> float:
+    """Max of a per-rank timing over all ranks (identity without a process group)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_value(world: int, bytes_per_step: int, ms_per_step: float) -> float:
+    """Whole-job GB/s: every rank runs the full sweep, timed by the slowest rank."""
+    return world * bytes_per_step / (ms_per_step * 1e-3) / 1e9
+
+
 def case_bytes(M, N, K, groups_per_row, out_len=None):
     """Algorithmic bytes of one GEMV call: packed W + fp16 s,z + X + Y."""
     out_len = N if out_len is None else out_len
@@ -423,11 +438,8 @@ def run_ours(args):
             graph.replay()
             torch.cuda.synchronize()
     clocks = sampler.stop()
-    if dist:
-        t = torch.tensor([ms_step], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
-    value = ws_ * bytes_step / (ms_step * 1e-3) / 1e9
+    ms_step = max_over_ranks(dist, ms_step, dev)
+    value = weak_value(ws_, bytes_step, ms_step)
 
     # per-case device times (graph of one call, 20 replays; L2 warm for the
     # small sets -- reported for context, the headline is the cold sweep)
@@ -469,12 +481,8 @@ def run_ours(args):
             e2e_step()
         a1.record(stream)
         torch.cuda.synchronize()
-    ms_e2e = a0.elapsed_time(a1) / e2e_steps
-    if dist:
-        t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e_value = ws_ * bytes_step / (ms_e2e * 1e-3) / 1e9
+    ms_e2e = max_over_ranks(dist, a0.elapsed_time(a1) / e2e_steps, dev)
+    e2e_value = weak_value(ws_, bytes_step, ms_e2e)
 
     rows = None
     if not args.no_rows:
