@@ -448,6 +448,36 @@ w4_status run_gemm_tc(const TcProblem& p, cudaStream_t st) {
                : launch_tc_bn<false, false>(BN, pm, bm, a, grid, smem, st);
 }
 
+
+// ------------------------------------------------- allocation-free GEMV
+// Scratch for w4a16_gemv_noalloc: the fp32 split-K partials of the forward
+// GEMV live in this file-scope array instead of a caller workspace.  Every
+// device that loads the library holds one copy until the process exits.
+constexpr size_t kNoAllocScratchBytes = 8u << 20;  // 8 MiB
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+// Device address of the scratch array on the current device.  Host code
+// cannot pass &g_noalloc_scratch to a kernel (that name is a host-side
+// stand-in), so the first call on each device looks the address up with
+// that device current and caches it.
+w4_status noalloc_scratch(void** out) {
+    static std::mutex mu;
+    static void* ptrs[64] = {};
+    const int dev = current_device();
+    if (dev < 0 || dev >= 64) return W4_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return W4_ERR_CUDA;
+        }
+        ptrs[dev] = p;
+    }
+    *out = ptrs[dev];
+    return W4_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -571,6 +601,25 @@ w4_status w4a16_gemm(const void* A, int M, int N, int K, const uint32_t* packed,
     pr.Y = Y;
     pr.sms = sms;
     return run_gemm_tc(pr, st);
+}
+
+// Forward GEMV (M <= 4) that allocates nothing: the split-K partials go to
+// the library's built-in 8 MiB device scratch instead of a caller
+// workspace.  See include/w4a16.h for who needs this and its limits.
+w4_status w4a16_gemv_noalloc(const void* X, int M, int N, int K, const uint32_t* packed,
+                             const void* scales, const void* zeros, int mode, int group_size,
+                             const void* bias, void* Y, void* stream) {
+    Meta meta;
+    w4_status s = check_matmul(X, M, N, K, packed, scales, zeros, mode, group_size, bias, Y, &meta);
+    if (s != W4_OK) return s;
+    if (M > 4) return W4_ERR_INVALID_ARG;
+    void* scratch = nullptr;
+    s = noalloc_scratch(&scratch);
+    if (s != W4_OK) return s;
+    const int sms = device_info(current_device()).sms;
+    if (gemv_workspace(M, N, K, 0, sms) > kNoAllocScratchBytes) return W4_ERR_WORKSPACE;
+    return run_gemv_fwd(X, M, N, K, packed, scales, zeros, meta, bias, Y, scratch,
+                        kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
 }
 
 uint64_t w4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -145,6 +145,38 @@ w4_status w4_device_error(int *code);
  */
 uint64_t w4_launch_count(void);
 
+/*
+ * w4a16_gemv_noalloc -- the forward GEMV of w4a16_gemv (M = 1..4,
+ * transposed = 0) for callers that cannot allocate device memory: code that
+ * runs where cudaMalloc is off limits or unsafe, such as inside an engine
+ * that owns every byte of the GPU through its own pool, a plugin handed
+ * only its input and output buffers, or a path that must not block on the
+ * allocator.  The pages have no counterpart of this call.
+ *
+ * Instead of a caller workspace it uses a scratch array compiled into the
+ * library: 8 MiB of device memory per GPU, held from the moment the library
+ * is loaded on that device until the process exits.  The call allocates
+ * nothing (no cudaMalloc, cudaFree or allocating library routine).  The
+ * caller still passes X [M, K], the packed weights, scales, zeros, the
+ * optional bias [N] and Y [M, N], with the layouts and validation of
+ * w4a16_gemv.
+ *
+ * Limits and sharing:
+ *   - A problem whose split-K partials need more than 8 MiB
+ *     (w4_workspace_bytes(M, N, K, 0) > 8 MiB) returns W4_ERR_WORKSPACE and
+ *     launches nothing.
+ *   - Every call on a device shares the one array.  Calls that may overlap
+ *     on the GPU (other streams, other host threads) race on it and give
+ *     wrong results; order them on one stream.  Each call writes all the
+ *     partials it later reads, so nothing needs clearing between calls.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ */
+w4_status w4a16_gemv_noalloc(const void *X, int M, int N, int K, const uint32_t *packed,
+                             const void *scales, const void *zeros, int mode, int group_size,
+                             const void *bias, void *Y, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
