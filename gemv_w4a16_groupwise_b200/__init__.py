@@ -35,7 +35,10 @@ _lib = None
 class W4Error(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {library().w4_status_string(status).decode()}")
+        msg = f"{what}: {library().w4_status_string(status).decode()}"
+        if status == 5:
+            msg += f" ({library().w4_last_cuda_error().decode()})"
+        super().__init__(msg)
 
 
 def library_path() -> str:
@@ -64,6 +67,8 @@ def library():
                 f.restype = I
             lib.w4_device_error.argtypes = [ctypes.POINTER(I)]
             lib.w4_device_error.restype = I
+            lib.w4_last_cuda_error.argtypes = []
+            lib.w4_last_cuda_error.restype = ctypes.c_char_p
             lib.w4_launch_count.argtypes = []
             lib.w4_launch_count.restype = ctypes.c_uint64
             _lib = lib

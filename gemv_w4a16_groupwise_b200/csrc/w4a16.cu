@@ -19,6 +19,8 @@ namespace {
 
 using namespace w4;
 
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
 // ----------------------------------------------------------------- device info
 struct DeviceInfo {
     int sms = 0;
@@ -69,7 +71,11 @@ cudaError_t ensure_smem(const void* fn, size_t bytes) {
         if (table[i].dev == dev && table[i].fn == fn && table[i].bytes >= bytes) return cudaSuccess;
     cudaError_t e =
         cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        cudaGetLastError();
+        return e;
+    }
     if (count < 512) table[count++] = Entry{dev, fn, bytes};
     return cudaSuccess;
 }
@@ -142,12 +148,14 @@ w4_status check_mode(int K, int mode, int group_size, Meta* meta) {
 }
 
 std::atomic<uint64_t> g_launches{0};
-
 // Called right after every kernel launch: counts it and maps a launch
-// failure to W4_ERR_CUDA.
+// failure to W4_ERR_CUDA (the CUDA error is kept for w4_last_cuda_error).
 w4_status launch_status() {
     g_launches.fetch_add(1, std::memory_order_relaxed);
-    return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) return W4_OK;
+    g_last_cuda_error = e;
+    return W4_ERR_CUDA;
 }
 
 int gcd_int(int a, int b) {
@@ -223,6 +231,8 @@ TPlan plan_t(int M, int N, int K, int sms) {
 
 size_t gemv_workspace(int M, int N, int K, int transposed, int sms) {
     if (transposed) return plan_t(M, N, K, sms).ws;
+    // M <= 2 with K % 32 == 0 normally takes the workspace-free lanes-along-K
+    // kernel; the TMA kernel's split still bounds what may be needed
     // the group structure only changes the fold granule, not the split
     Meta meta{K, 1, 1};
     FwdPlan p = plan_fwd(M, N, K, meta, sms);
@@ -251,10 +261,84 @@ w4_status launch_gemv_fwd(const FwdPlan& p, const CUtensorMap& map, const GemvFw
     return launch_status();
 }
 
+// Lanes-along-K GEMV for M <= 2 (gemv_rows_kernel): chunk = 32 k inside one
+// group, so K % 32 == 0 and g % 32 == 0.  Picks the warps per CTA and the
+// rows per round so that the persistent grid covers the SMs.
+struct RowsPlan {
+    bool ok = false;
+    int NW = 16, KB = 0, RBP = 1, rounds = 0, grid = 0;
+    size_t smem = 0;
+};
+
+RowsPlan plan_rows(int M, int N, int K, const Meta& meta, const DeviceInfo& di) {
+    RowsPlan best;
+    if (M > 2 || K % 32 != 0 || meta.g % 32 != 0) return best;
+    const int KB = (K + 1023) / 1024;
+    const int nrb = (N + kRowsRB - 1) / kRowsRB;
+    double best_score = -1.0;
+    for (int NW : {16, 8, 4}) {
+        RowsPlan p;
+        p.NW = NW;
+        p.KB = KB;
+        p.RBP = NW / gcd_int(KB, NW);
+        p.rounds = (nrb + p.RBP - 1) / p.RBP;
+        p.smem = gemv_rows_smem_bytes(M, KB, p.RBP);
+        if (p.smem > static_cast<size_t>(di.max_smem_optin)) continue;
+        const int by_smem = std::max(1, static_cast<int>((228 * 1024) / (p.smem + 1024)));
+        const int by_threads = 2048 / (NW * 32);
+        const int by_regs = 65536 / (NW * 32 * (M == 1 ? 64 : 128));
+        const int occ = std::max(1, std::min(by_smem, std::min(by_threads, by_regs)));
+        p.grid = std::min(p.rounds, di.sms * occ);
+        const long long per_cta = (p.rounds + p.grid - 1) / p.grid;
+        // warps kept busy, discounted by round imbalance and by the staging
+        // every CTA repeats (M * K activations)
+        const double busy = static_cast<double>(p.grid) * NW * p.rounds / (per_cta * p.grid);
+        const double work = static_cast<double>(per_cta) * p.RBP * kRowsRB * K;  // weights per CTA
+        const double stage = 8.0 * M * K;
+        const double score = busy * work / (work + stage);
+        if (score > best_score) {
+            best_score = score;
+            best = p;
+            best.ok = true;
+        }
+    }
+    return best;
+}
+
+w4_status run_gemv_rows(const RowsPlan& p, int M, int N, int K, const void* A, const uint32_t* packed,
+                        const void* S, const void* Z, const Meta& meta, const void* bias, void* Y,
+                        cudaStream_t st) {
+    GemvRowsArgs a;
+    a.X = static_cast<const uint16_t*>(A);
+    a.packed = packed;
+    a.S = static_cast<const __half*>(S);
+    a.Z = static_cast<const __half*>(Z);
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.Y = static_cast<uint16_t*>(Y);
+    a.N = N;
+    a.K = K;
+    a.g = meta.g;
+    a.G = meta.G;
+    a.sz_row = meta.sz_row;
+    a.KB = p.KB;
+    a.RBP = p.RBP;
+    a.rounds = p.rounds;
+    const void* fn = M == 1 ? reinterpret_cast<const void*>(gemv_rows_kernel<1>)
+                            : reinterpret_cast<const void*>(gemv_rows_kernel<2>);
+    if (ensure_smem(fn, p.smem) != cudaSuccess) return W4_ERR_CUDA;
+    if (M == 1) gemv_rows_kernel<1><<<p.grid, p.NW * 32, p.smem, st>>>(a);
+    else gemv_rows_kernel<2><<<p.grid, p.NW * 32, p.smem, st>>>(a);
+    return launch_status();
+}
+
 w4_status run_gemv_fwd(const void* A, int M, int N, int K, const uint32_t* packed, const void* S,
                        const void* Z, const Meta& meta, const void* bias, void* Y, void* ws,
                        size_t ws_bytes, cudaStream_t st) {
     const DeviceInfo di = device_info(current_device());
+    {
+        const RowsPlan rp = plan_rows(M, N, K, meta, di);
+        if (rp.ok) return run_gemv_rows(rp, M, N, K, A, packed, S, Z, meta, bias, Y, st);
+    }
     const FwdPlan p = plan_fwd(M, N, K, meta, di.sms);
     GemvFwdArgs a;
     a.X = static_cast<const uint16_t*>(A);
@@ -621,6 +705,8 @@ w4_status w4a16_gemv_noalloc(const void* X, int M, int N, int K, const uint32_t*
     return run_gemv_fwd(X, M, N, K, packed, scales, zeros, meta, bias, Y, scratch,
                         kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
 }
+
+const char* w4_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 uint64_t w4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 

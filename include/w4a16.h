@@ -138,6 +138,13 @@ const char *w4_status_string(int status);
 w4_status w4_device_error(int *code);
 
 /*
+ * w4_last_cuda_error -- text of the last CUDA error behind a W4_ERR_CUDA
+ * returned on the calling host thread ("no error" if none).  Static
+ * storage, never NULL.
+ */
+const char *w4_last_cuda_error(void);
+
+/*
  * w4_launch_count -- number of kernel launches this library has issued in
  * the calling process since it was loaded (all devices, all entry points).
  * Host-side counter; launches replayed from a captured CUDA graph are not
