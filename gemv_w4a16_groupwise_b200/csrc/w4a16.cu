@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_stream.cuh"
 #include "quantize.cuh"
 #include "w4a16.h"
 
@@ -229,16 +230,90 @@ TPlan plan_t(int M, int N, int K, int sms) {
     return p;
 }
 
+// Streaming forward GEMV (gemv_stream_kernel): K % 32 == 0 and g % 32 == 0
+// so that every 32-k chunk lies inside one group.  The K slice is the
+// largest whole number of 2048-k boxes whose activation block fits in
+// shared memory next to the TMA ring; the k-parts per round are chosen to
+// even out the work of the persistent CTAs.
+struct StreamPlan {
+    bool ok = false;
+    int TKC = 0, splits = 1, nbs = 0, KP = 1, RBP = kSW, rounds = 0, units = 0, grid = 0, stages = 2;
+    int szw = 0;
+    size_t smem = 0, xbytes = 0, ws = 0, partial_off = 0;
+};
+
+// szw: scale / zero words per stage row (gemv_stream_sz_words of the group
+// length).  Ring depth first: the deepest ring (4, 3, then 2 stages per
+// warp) whose activation block for all of K still fits; if none does, 2
+// stages and K split into slices.
+StreamPlan plan_stream_szw(int M, int N, int K, int szw, const DeviceInfo& di) {
+    StreamPlan p;
+    p.szw = szw;
+    const int nb_total = (K + kSBK - 1) / kSBK;
+    auto nbs_fit = [&](int stages) {
+        int best = 0;
+        for (int nb = 1; nb <= nb_total; ++nb) {
+            if (gemv_stream_smem_bytes(M, nb * kSBK, stages, szw) > static_cast<size_t>(di.max_smem_optin)) break;
+            best = nb;
+        }
+        return best;
+    };
+    int nbs_max = 0;
+    for (int stages : {4, 3, 2}) {
+        p.stages = stages;
+        nbs_max = nbs_fit(stages);
+        if (nbs_max >= nb_total) break;
+    }
+    if (nbs_max == 0) return p;
+    p.splits = (nb_total + nbs_max - 1) / nbs_max;
+    p.nbs = (nb_total + p.splits - 1) / p.splits;
+    p.TKC = p.nbs * kSBK;
+    const int nrb = (N + kSR - 1) / kSR;
+    double best = 1e300;
+    for (int KP : {1, 2, 4, 8}) {
+        if (KP > p.nbs) break;
+        const int RBP = kSW / KP;
+        const int rounds = (nrb + RBP - 1) / RBP;
+        const int units = p.splits * rounds;
+        const int grid = std::min(units, di.sms);
+        const int per_cta = (units + grid - 1) / grid;
+        // boxes the busiest warp streams, plus the round's barrier and
+        // reduction (about half a box)
+        const double cost = per_cta * ((p.nbs + KP - 1) / KP + 0.5);
+        if (cost < best * 0.999) {
+            best = cost;
+            p.KP = KP;
+            p.RBP = RBP;
+            p.rounds = rounds;
+            p.units = units;
+            p.grid = grid;
+        }
+    }
+    p.smem = gemv_stream_smem_bytes(M, p.TKC, p.stages, szw);
+    p.xbytes = gemv_stream_xblock_bytes(M, p.TKC);
+    p.partial_off = (p.splits * p.xbytes + 255) / 256 * 256;
+    p.ws = p.partial_off + (p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * sizeof(float) : 0);
+    p.ok = true;
+    return p;
+}
+
+StreamPlan plan_stream(int M, int N, int K, const Meta& meta, const DeviceInfo& di) {
+    if (K % 32 != 0 || meta.g % 32 != 0) return StreamPlan{};
+    return plan_stream_szw(M, N, K, gemv_stream_sz_words(meta.g), di);
+}
+
 size_t gemv_workspace(int M, int N, int K, int transposed, int sms) {
     if (transposed) return plan_t(M, N, K, sms).ws;
-    // M <= 2 with K % 32 == 0 normally takes the workspace-free lanes-along-K
-    // kernel; the TMA kernel's split still bounds what may be needed
-    // the group structure only changes the fold granule, not the split
-    Meta meta{K, 1, 1};
-    FwdPlan p = plan_fwd(M, N, K, meta, sms);
-    size_t ws = p.ws;
-    Meta meta32{32, K / 32, K / 32};
-    if (K % 32 == 0) ws = std::max(ws, plan_fwd(M, N, K, meta32, sms).ws);
+    if (K % 32 != 0) return 0;
+    // the group length changes the stage size and so possibly the split:
+    // cover every stage size a group length of 32 .. K can give
+    DeviceInfo di = device_info(current_device());
+    di.sms = sms;
+    size_t ws = 0;
+    for (int szw = gemv_stream_sz_words(K); szw <= gemv_stream_sz_words(32); ++szw) {
+        const StreamPlan p = plan_stream_szw(M, N, K, szw, di);
+        if (p.ok) ws = std::max(ws, p.ws);
+    }
     return ws;
 }
 
@@ -331,13 +406,84 @@ w4_status run_gemv_rows(const RowsPlan& p, int M, int N, int K, const void* A, c
     return launch_status();
 }
 
+template <int M, int GK>
+w4_status launch_gemv_stream_gk(const StreamPlan& p, const CUtensorMap& map, const GemvStreamArgs& a,
+                                cudaStream_t st) {
+    const void* fn = reinterpret_cast<const void*>(gemv_stream_kernel<M, GK>);
+    if (ensure_smem(fn, p.smem) != cudaSuccess) return W4_ERR_CUDA;
+    gemv_stream_kernel<M, GK><<<p.grid, kSW * 32, p.smem, st>>>(map, a);
+    return launch_status();
+}
+
+template <int M>
+w4_status launch_gemv_stream(const StreamPlan& p, const CUtensorMap& map, const GemvStreamArgs& a,
+                             cudaStream_t st) {
+    if (a.G == 1) return launch_gemv_stream_gk<M, kGroupsOne>(p, map, a, st);
+    if (kSBK % a.g == 0) return launch_gemv_stream_gk<M, kGroupsPow2>(p, map, a, st);
+    return launch_gemv_stream_gk<M, kGroupsAny>(p, map, a, st);
+}
+
+w4_status run_gemv_stream(const StreamPlan& p, int M, int N, int K, const void* A, const uint32_t* packed,
+                          const void* S, const void* Z, const Meta& meta, const void* bias, void* Y,
+                          void* ws, size_t ws_bytes, cudaStream_t st) {
+    if (p.ws > ws_bytes || ws == nullptr) return W4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return W4_ERR_ALIGNMENT;
+    uint8_t* xb = static_cast<uint8_t*>(ws);
+    const long long chunks = static_cast<long long>(p.splits) * M * (p.TKC / 32);
+    gemv_xprep_kernel<<<static_cast<int>((chunks + 255) / 256), 256, 0, st>>>(
+        static_cast<const uint16_t*>(A), M, K, p.TKC, p.splits, xb);
+    w4_status s = launch_status();
+    if (s != W4_OK) return s;
+    CUtensorMap map;
+    if (!make_map_2d(&map, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, kSR, kSBK / 8, 0))
+        return W4_ERR_CUDA;
+    GemvStreamArgs a;
+    a.xblocks = xb;
+    a.S = static_cast<const __half*>(S);
+    a.Z = static_cast<const __half*>(Z);
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.Y = static_cast<uint16_t*>(Y);
+    a.partial = p.splits > 1 ? reinterpret_cast<float*>(xb + p.partial_off) : nullptr;
+    a.N = N;
+    a.K = K;
+    a.g = meta.g;
+    a.G = meta.G;
+    a.sz_row = meta.sz_row;
+    a.TKC = p.TKC;
+    a.splits = p.splits;
+    a.nbs = p.nbs;
+    a.KP = p.KP;
+    a.RBP = p.RBP;
+    a.rounds = p.rounds;
+    a.units = p.units;
+    a.stages = p.stages;
+    a.szw = p.szw;
+    a.sz_total = meta.sz_row ? static_cast<long long>(N) * meta.sz_row : 1;
+    switch (M) {
+        case 1: s = launch_gemv_stream<1>(p, map, a, st); break;
+        case 2: s = launch_gemv_stream<2>(p, map, a, st); break;
+        case 3: s = launch_gemv_stream<3>(p, map, a, st); break;
+        case 4: s = launch_gemv_stream<4>(p, map, a, st); break;
+        default: return W4_ERR_INVALID_ARG;
+    }
+    if (s != W4_OK) return s;
+    if (p.splits > 1) {
+        const DeviceInfo di = device_info(current_device());
+        const long long total = static_cast<long long>(M) * N;
+        const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, di.sms * 8));
+        splits_finalize_kernel<<<blocks, 256, 0, st>>>(a.partial, p.splits, M, N, a.bias, a.Y);
+        return launch_status();
+    }
+    return W4_OK;
+}
+
 w4_status run_gemv_fwd(const void* A, int M, int N, int K, const uint32_t* packed, const void* S,
                        const void* Z, const Meta& meta, const void* bias, void* Y, void* ws,
                        size_t ws_bytes, cudaStream_t st) {
     const DeviceInfo di = device_info(current_device());
     {
-        const RowsPlan rp = plan_rows(M, N, K, meta, di);
-        if (rp.ok) return run_gemv_rows(rp, M, N, K, A, packed, S, Z, meta, bias, Y, st);
+        const StreamPlan sp = plan_stream(M, N, K, meta, di);
+        if (sp.ok) return run_gemv_stream(sp, M, N, K, A, packed, S, Z, meta, bias, Y, ws, ws_bytes, st);
     }
     const FwdPlan p = plan_fwd(M, N, K, meta, di.sms);
     GemvFwdArgs a;
@@ -534,9 +680,10 @@ w4_status run_gemm_tc(const TcProblem& p, cudaStream_t st) {
 
 
 // ------------------------------------------------- allocation-free GEMV
-// Scratch for w4a16_gemv_noalloc: the fp32 split-K partials of the forward
-// GEMV live in this file-scope array instead of a caller workspace.  Every
-// device that loads the library holds one copy until the process exits.
+// Scratch for w4a16_gemv_noalloc: the forward GEMV's workspace (prepared
+// activations, split-K partials) lives in this file-scope array instead of
+// a caller workspace.  Every device that loads the library holds one copy
+// until the process exits.
 constexpr size_t kNoAllocScratchBytes = 8u << 20;  // 8 MiB
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
@@ -687,7 +834,7 @@ w4_status w4a16_gemm(const void* A, int M, int N, int K, const uint32_t* packed,
     return run_gemm_tc(pr, st);
 }
 
-// Forward GEMV (M <= 4) that allocates nothing: the split-K partials go to
+// Forward GEMV (M <= 4) that allocates nothing: its workspace goes to
 // the library's built-in 8 MiB device scratch instead of a caller
 // workspace.  See include/w4a16.h for who needs this and its limits.
 w4_status w4a16_gemv_noalloc(const void* X, int M, int N, int K, const uint32_t* packed,

@@ -169,13 +169,14 @@ uint64_t w4_launch_count(void);
  * w4a16_gemv.
  *
  * Limits and sharing:
- *   - A problem whose split-K partials need more than 8 MiB
- *     (w4_workspace_bytes(M, N, K, 0) > 8 MiB) returns W4_ERR_WORKSPACE and
- *     launches nothing.
+ *   - A problem whose workspace (the activations in the kernel's
+ *     fixed-point form and, when K is split, the fp32 partials) needs more
+ *     than 8 MiB (w4_workspace_bytes(M, N, K, 0) > 8 MiB) returns
+ *     W4_ERR_WORKSPACE and launches nothing.
  *   - Every call on a device shares the one array.  Calls that may overlap
  *     on the GPU (other streams, other host threads) race on it and give
  *     wrong results; order them on one stream.  Each call writes all the
- *     partials it later reads, so nothing needs clearing between calls.
+ *     scratch it later reads, so nothing needs clearing between calls.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.

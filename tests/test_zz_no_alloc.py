@@ -64,7 +64,7 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_device):
 
 def test_noalloc_rejects_problems_beyond_the_scratch(cuda_device):
     w4, lib = _lib()
-    M, N, K = 4, 1 << 20, 16384
+    M, N, K = 4, 1 << 20, 65536      # K split into slices: fp32 partials of 4 x M x N
     need = w4.w4_workspace_bytes(M, N, K, False)
     assert need > (8 << 20)
     fake = 1 << 20          # never dereferenced: the size check comes before any launch
