@@ -157,6 +157,7 @@ struct GemvStreamArgs {
     int stages;               // TMA stages per warp
     int szw;                  // scale / zero words per row and stage
     long long sz_total;       // halves in each of S and Z (N * sz_row, or 1)
+    int M;                    // activation rows (the tensor-pipe kernel takes it at run time)
 };
 
 // 1-D bulk copy global -> shared, completing on `bar` (16-byte aligned

@@ -13,6 +13,7 @@
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "gemv_stream.cuh"
+#include "gemv_mma.cuh"
 #include "quantize.cuh"
 #include "w4a16.h"
 
@@ -119,6 +120,21 @@ bool make_map_2d(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, int 
                     : swizzle == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                                     : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// n `esize`-byte elements as a one-row 2-D tensor (the row stride is never
+// stepped; it is only rounded up to the 16 bytes the encoder requires), box
+// of `box` elements.
+bool make_map_row(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, int esize, uint64_t n, uint32_t box) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[2] = {n, 1};
+    cuuint64_t gstride[1] = {(n * esize + 15) / 16 * 16};
+    cuuint32_t bx[2] = {box, 1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dt, 2, const_cast<void*>(ptr), gdim, gstride, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -238,7 +254,8 @@ TPlan plan_t(int M, int N, int K, int sms) {
 struct StreamPlan {
     bool ok = false;
     int TKC = 0, splits = 1, nbs = 0, KP = 1, RBP = kSW, rounds = 0, units = 0, grid = 0, stages = 2;
-    int szw = 0;
+    int szw = 0, warps = kSW, sz = 0;
+    bool mma = false;
     size_t smem = 0, xbytes = 0, ws = 0, partial_off = 0;
 };
 
@@ -302,17 +319,90 @@ StreamPlan plan_stream(int M, int N, int K, const Meta& meta, const DeviceInfo& 
     return plan_stream_szw(M, N, K, gemv_stream_sz_words(meta.g), di);
 }
 
+// Tensor-pipe GEMV (gemv_mma_kernel): group length a multiple of 128, or
+// one group per row.  Same slicing as the CUDA-core kernel, but the ring
+// may hold 8, 12 or 16 warps: the deepest ring (warps x stages) whose
+// activation block for all of K fits wins; if none fits, 8 warps x 2
+// stages and K split into slices.
+StreamPlan plan_mma(int M, int N, int K, int sz, int szw, const DeviceInfo& di) {
+    StreamPlan p;
+    p.szw = szw;
+    p.sz = sz;
+    const int nb_total = (K + kSBK - 1) / kSBK;
+    auto nbs_fit = [&](int warps, int stages) {
+        int best = 0;
+        for (int nb = 1; nb <= nb_total; ++nb) {
+            if (gemv_mma_smem_bytes(M, nb * kSBK, warps, stages, sz, szw) > static_cast<size_t>(di.max_smem_optin))
+                break;
+            best = nb;
+        }
+        return best;
+    };
+    static const int kRings[][2] = {{16, 3}, {12, 4}, {16, 2}, {12, 3}, {8, 4}, {12, 2}, {8, 3}, {8, 2}};
+    int nbs_max = 0;
+    for (const auto& r : kRings) {
+        p.warps = r[0];
+        p.stages = r[1];
+        nbs_max = nbs_fit(p.warps, p.stages);
+        if (nbs_max >= nb_total) break;
+    }
+    if (nbs_max == 0) return p;
+    p.splits = (nb_total + nbs_max - 1) / nbs_max;
+    p.nbs = (nb_total + p.splits - 1) / p.splits;
+    p.TKC = p.nbs * kSBK;
+    const int nrb = (N + kSR - 1) / kSR;
+    double best = 1e300;
+    for (int KP = 1; KP <= p.warps && KP <= p.nbs; ++KP) {
+        if (p.warps % KP) continue;
+        const int RBP = p.warps / KP;
+        const int rounds = (nrb + RBP - 1) / RBP;
+        const int units = p.splits * rounds;
+        const int grid = std::min(units, di.sms);
+        const int per_cta = (units + grid - 1) / grid;
+        const double cost = per_cta * ((p.nbs + KP - 1) / KP + 0.5);
+        if (cost < best * 0.999) {
+            best = cost;
+            p.KP = KP;
+            p.RBP = RBP;
+            p.rounds = rounds;
+            p.units = units;
+            p.grid = grid;
+        }
+    }
+    p.smem = gemv_mma_smem_bytes(M, p.TKC, p.warps, p.stages, sz, szw);
+    p.xbytes = gemv_mma_xblock_bytes(M, p.TKC);
+    p.partial_off = (p.splits * p.xbytes + 255) / 256 * 256;
+    p.ws = p.partial_off + (p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * sizeof(float) : 0);
+    p.mma = true;
+    p.ok = true;
+    return p;
+}
+
+bool mma_eligible(int K, const Meta& meta) { return K % 32 == 0 && (meta.G == 1 || meta.g % 128 == 0); }
+
+// How the tensor-pipe GEMV fetches scales and zeros (SzKind).
+int mma_sz_kind(const Meta& meta) {
+    if (meta.sz_row == 0) return kSzConst;
+    if (meta.G == 1) return kSzTma1d;
+    if (meta.G % 8 == 0) return kSzTma2d;
+    return kSzCopy;
+}
+
 size_t gemv_workspace(int M, int N, int K, int transposed, int sms) {
     if (transposed) return plan_t(M, N, K, sms).ws;
     if (K % 32 != 0) return 0;
-    // the group length changes the stage size and so possibly the split:
-    // cover every stage size a group length of 32 .. K can give
+    // the group length picks the kernel and the stage size, and so possibly
+    // the split: cover every choice a group length of 32 .. K can make
     DeviceInfo di = device_info(current_device());
     di.sms = sms;
     size_t ws = 0;
     for (int szw = gemv_stream_sz_words(K); szw <= gemv_stream_sz_words(32); ++szw) {
         const StreamPlan p = plan_stream_szw(M, N, K, szw, di);
         if (p.ok) ws = std::max(ws, p.ws);
+        for (int sz : {kSzConst, kSzTma2d, kSzTma1d, kSzCopy}) {
+            const StreamPlan q = plan_mma(M, N, K, sz, szw, di);
+            if (q.ok) ws = std::max(ws, q.ws);
+        }
     }
     return ws;
 }
@@ -423,15 +513,83 @@ w4_status launch_gemv_stream(const StreamPlan& p, const CUtensorMap& map, const 
     return launch_gemv_stream_gk<M, kGroupsAny>(p, map, a, st);
 }
 
+// The GEMV is launched as a programmatic dependent of the prep kernel just
+// before it: its prologue and first weight loads overlap the prep kernel.
+template <int M, int GK, int SZ>
+w4_status launch_gemv_mma_k(const StreamPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
+                            const CUtensorMap& zm, const GemvStreamArgs& a, cudaStream_t st) {
+    auto* fn = gemv_mma_kernel<M, GK, SZ>;
+    if (ensure_smem(reinterpret_cast<const void*>(fn), p.smem) != cudaSuccess) return W4_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.grid);
+    cfg.blockDim = dim3(p.warps * 32);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, fn, wm, sm, zm, a);
+    return launch_status();
+}
+
+template <int M, int GK>
+w4_status launch_gemv_mma_gk(const StreamPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
+                             const CUtensorMap& zm, const GemvStreamArgs& a, cudaStream_t st) {
+    switch (p.sz) {
+        case kSzConst: return launch_gemv_mma_k<M, GK, kSzConst>(p, wm, sm, zm, a, st);
+        case kSzTma2d: return launch_gemv_mma_k<M, GK, kSzTma2d>(p, wm, sm, zm, a, st);
+        case kSzTma1d: return launch_gemv_mma_k<M, GK, kSzTma1d>(p, wm, sm, zm, a, st);
+        default: return launch_gemv_mma_k<M, GK, kSzCopy>(p, wm, sm, zm, a, st);
+    }
+}
+
+template <int M>
+w4_status launch_gemv_mma_m(const StreamPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
+                            const CUtensorMap& zm, const GemvStreamArgs& a, cudaStream_t st) {
+    if (a.G == 1) return launch_gemv_mma_gk<M, kGroupsOne>(p, wm, sm, zm, a, st);
+    if (kSBK % a.g == 0) return launch_gemv_mma_gk<M, kGroupsPow2>(p, wm, sm, zm, a, st);
+    return launch_gemv_mma_gk<M, kGroupsAny>(p, wm, sm, zm, a, st);
+}
+
+w4_status launch_gemv_mma(const StreamPlan& p, int M, const CUtensorMap& wm, const void* S, const void* Z,
+                          const GemvStreamArgs& a, cudaStream_t st) {
+    CUtensorMap sm, zm;
+    std::memset(&sm, 0, sizeof sm);
+    std::memset(&zm, 0, sizeof zm);
+    bool ok = true;
+    if (p.sz == kSzTma2d) {
+        ok = make_map_2d(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.G, kSR, 16, 0) &&
+             make_map_2d(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.G, kSR, 16, 0);
+    } else if (p.sz == kSzTma1d) {
+        ok = make_map_row(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, 8) &&
+             make_map_row(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, 8);
+    }
+    if (!ok) return W4_ERR_CUDA;
+    switch (M) {
+        case 1: return launch_gemv_mma_m<1>(p, wm, sm, zm, a, st);
+        case 2: return launch_gemv_mma_m<2>(p, wm, sm, zm, a, st);
+        case 3: return launch_gemv_mma_m<3>(p, wm, sm, zm, a, st);
+        default: return launch_gemv_mma_m<4>(p, wm, sm, zm, a, st);
+    }
+}
+
 w4_status run_gemv_stream(const StreamPlan& p, int M, int N, int K, const void* A, const uint32_t* packed,
                           const void* S, const void* Z, const Meta& meta, const void* bias, void* Y,
                           void* ws, size_t ws_bytes, cudaStream_t st) {
     if (p.ws > ws_bytes || ws == nullptr) return W4_ERR_WORKSPACE;
     if (!aligned16(ws)) return W4_ERR_ALIGNMENT;
     uint8_t* xb = static_cast<uint8_t*>(ws);
-    const long long chunks = static_cast<long long>(p.splits) * M * (p.TKC / 32);
-    gemv_xprep_kernel<<<static_cast<int>((chunks + 255) / 256), 256, 0, st>>>(
-        static_cast<const uint16_t*>(A), M, K, p.TKC, p.splits, xb);
+    if (p.mma) {
+        const long long lanes = static_cast<long long>(p.splits) * (p.TKC / 256) * M * 32;
+        gemv_xfrag_kernel<<<static_cast<int>((lanes + 255) / 256), 256, 0, st>>>(
+            static_cast<const uint16_t*>(A), M, K, p.TKC, p.splits, xb);
+    } else {
+        const long long chunks = static_cast<long long>(p.splits) * M * (p.TKC / 32);
+        gemv_xprep_kernel<<<static_cast<int>((chunks + 255) / 256), 256, 0, st>>>(
+            static_cast<const uint16_t*>(A), M, K, p.TKC, p.splits, xb);
+    }
     w4_status s = launch_status();
     if (s != W4_OK) return s;
     CUtensorMap map;
@@ -459,7 +617,10 @@ w4_status run_gemv_stream(const StreamPlan& p, int M, int N, int K, const void* 
     a.stages = p.stages;
     a.szw = p.szw;
     a.sz_total = meta.sz_row ? static_cast<long long>(N) * meta.sz_row : 1;
-    switch (M) {
+    a.M = M;
+    if (p.mma) {
+        s = launch_gemv_mma(p, M, map, S, Z, a, st);
+    } else switch (M) {
         case 1: s = launch_gemv_stream<1>(p, map, a, st); break;
         case 2: s = launch_gemv_stream<2>(p, map, a, st); break;
         case 3: s = launch_gemv_stream<3>(p, map, a, st); break;
@@ -482,7 +643,9 @@ w4_status run_gemv_fwd(const void* A, int M, int N, int K, const uint32_t* packe
                        size_t ws_bytes, cudaStream_t st) {
     const DeviceInfo di = device_info(current_device());
     {
-        const StreamPlan sp = plan_stream(M, N, K, meta, di);
+        StreamPlan sp;
+        if (mma_eligible(K, meta)) sp = plan_mma(M, N, K, mma_sz_kind(meta), gemv_stream_sz_words(meta.g), di);
+        if (!sp.ok) sp = plan_stream(M, N, K, meta, di);
         if (sp.ok) return run_gemv_stream(sp, M, N, K, A, packed, S, Z, meta, bias, Y, ws, ws_bytes, st);
     }
     const FwdPlan p = plan_fwd(M, N, K, meta, di.sms);
