@@ -157,8 +157,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr uint32_t kIdesc = umma_idesc_bf16(BN, TR);
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int NS = a.stages;
     uint64_t* tma_full = reinterpret_cast<uint64_t*>(base + NS * kStageBytes);
     uint64_t* deq_full = tma_full + NS;

@@ -117,8 +117,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     constexpr int FW = F / 8;                // words per granule
     constexpr int GPB = kGemvBoxK / F;       // fold granules per box
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* ring = base;
     // activation record of (m, word j): 8 uint32 = hi(even k), hi(odd k),
     // mid(even), mid(odd), lo(even), lo(odd), 2 unused; byte i of an "even"

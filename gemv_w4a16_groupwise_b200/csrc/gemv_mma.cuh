@@ -165,8 +165,7 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
                     const __grid_constant__ CUtensorMap zmap, const GemvStreamArgs a) {
     static_assert(M >= 1 && M <= 4, "M");
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int NW = blockDim.x >> 5;
     const int NS = a.stages;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
@@ -177,7 +176,7 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
     // bytes the scale / zero boxes add to a stage's transaction count
     constexpr int kSzTx = SZ == kSzTma2d ? 2 * kSR * 16 * 2 : SZ == kSzTma1d ? 2 * 8 * 2 : 0;
     uint8_t* ring = base;                                                    // [warp][stage][SB]
-    float4* table = reinterpret_cast<float4*>(ring + NW * NS * SB);          // [warp][4 rows][8 windows]
+    float4* table = reinterpret_cast<float4*>(ring + NW * NS * SB);          // [warp][8 windows][4 rows]
     uint8_t* xblk = reinterpret_cast<uint8_t*>(table + NW * kSR * 8);
     const uint4* frag = reinterpret_cast<const uint4*>(xblk);                // [qw][t][8M]
     const float4* fsc = reinterpret_cast<const float4*>(xblk + static_cast<size_t>(nqw) * M * 512);  // [qw][2M]
@@ -278,6 +277,12 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
 
     const int wrow = g >> 1, wchunk = (g & 1) * 4 + tig;   // the B chunk this lane loads
     const bool f_lane = g < 2 * M;
+    // lanes without activation rows (g >= 2M) never load: their fragments
+    // and fold constants stay zero for the whole kernel
+    uint4 af[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) af[t] = make_uint4(0u, 0u, 0u, 0u);
+    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
     float s_const = 0.f, z_const = 0.f;
     if (SZ == kSzConst) {
         s_const = __half2float(a.S[0]);
@@ -315,7 +320,8 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
             }
             const uint8_t* sb = ring + st * SB;
             if (SZ != kSzConst) {
-                // fp32 table of (s, z) for row ti, window tq, both halves
+                // fp32 table of (s, z) for window tq, row ti, both halves (the 4
+                // rows of a window are adjacent: the readers hit 4 distinct banks)
                 const int grp_lo = first_group(k0);
                 int o0, o1;
                 if (GK == kGroupsOne) {
@@ -341,23 +347,23 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
                     ps = sh + ti * 2 * a.szw + ((((row0 + ti) & a.sz_row) ^ grp_lo) & 1);
                     pz = ps + kSR * 2 * a.szw;
                 }
-                wtable[ti * 8 + tq] = make_float4(__half2float(ps[o0]), __half2float(pz[o0]), __half2float(ps[o1]),
+                wtable[tq * kSR + ti] = make_float4(__half2float(ps[o0]), __half2float(pz[o0]), __half2float(ps[o1]),
                                                   __half2float(pz[o1]));
                 __syncwarp();
             }
+            // per-box bases: every window below is an immediate offset from them
             const uint8_t* wsrc = sb + wrow * 1024 + wchunk * 16;
             const int qw0 = (b_lo + bi) * (kSBK / 256);
-#pragma unroll 2
+            const uint4* fb = frag + qw0 * (32 * M) + lane;
+            const float4* cb = fsc + qw0 * (2 * M) + g;
+#pragma unroll
             for (int qwl = 0; qwl < kSBK / 256; ++qwl) {
                 const uint4 wv = *reinterpret_cast<const uint4*>(wsrc + qwl * 128);
-                const int qw = qw0 + qwl;
-                uint4 af[4] = {};
-                float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (lane < 8 * M) {
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) af[t] = frag[(qw * 4 + t) * (8 * M) + lane];
+                    for (int t = 0; t < 4; ++t) af[t] = fb[(qwl * 4 + t) * (8 * M)];
                 }
-                if (f_lane) f = fsc[qw * 2 * M + g];
+                if (f_lane) f = cb[qwl * 2 * M];
                 int acc[2][4];
                 mma_s8u8_16832_z(acc[0], af[0], wv.x & 0x0F0F0F0Fu, (wv.x >> 4) & 0x0F0F0F0Fu);
                 mma_s8u8_16832_z(acc[1], af[1], wv.y & 0x0F0F0F0Fu, (wv.y >> 4) & 0x0F0F0F0Fu);
@@ -367,7 +373,7 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
                 const int d1 = acc[0][3] + acc[1][3];   // half 1: A row g + 8, B column (tig, 1)
                 float4 sz;
                 if (SZ == kSzConst) sz = make_float4(s_const, z_const, s_const, z_const);
-                else sz = wtable[tig * 8 + qwl];
+                else sz = wtable[qwl * kSR + tig];
                 y = fmaf(sz.x, fmaf(f.x, static_cast<float>(d0), -sz.y * f.y), y);
                 y = fmaf(sz.z, fmaf(f.z, static_cast<float>(d1), -sz.w * f.w), y);
             }

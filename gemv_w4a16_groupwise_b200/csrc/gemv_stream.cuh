@@ -195,8 +195,7 @@ __global__ void __launch_bounds__(kSW * 32, 1)
     gemv_stream_kernel(const __grid_constant__ CUtensorMap wmap, const GemvStreamArgs a) {
     static_assert(M >= 1 && M <= 4, "M");
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int NS = a.stages;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
     const int nchunk = a.TKC / 32;
