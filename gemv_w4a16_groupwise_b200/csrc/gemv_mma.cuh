@@ -31,8 +31,8 @@
 // tig against (m, p) = (g / 2, g % 2) for both halves, and folds them:
 //   y += s * (f1 * D - z * f2),  f1 = xs * 256^(1 - p),  f2 = [p == 1] xs * sum_k x'
 // with xs = 2^(e - 140), e the granule's largest bf16 exponent.  The two
-// digits meet in one shuffle at the end of the item.  Rounds, k-parts and
-// the output are as in gemv_stream_kernel.
+// digits meet in one shuffle when a row block is done; the work split and
+// the output are described at the kernel.
 #pragma once
 
 #include "gemv_stream.cuh"
@@ -58,9 +58,15 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 
 // One warp per (slice, window, m); lane = 16 h + 4 t + tig converts the 8
 // activations k = 128 h + 32 tig + 8 t .. + 7 of the window (zero past K).
+// The grid also clears the GEMV's row-block counters.
 __global__ void __launch_bounds__(256) gemv_xfrag_kernel(const uint16_t* __restrict__ X, int M, int K,
-                                                         int TKC, int splits, uint8_t* __restrict__ out) {
+                                                         int TKC, int splits, uint8_t* __restrict__ out,
+                                                         int* __restrict__ counters, int ncounters) {
     pdl_launch_dependents();
+    // the GEMV's per-row-block box counters start from zero on every call
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < ncounters;
+         i += static_cast<long long>(gridDim.x) * blockDim.x)
+        counters[i] = 0;
     const int nqw = TKC / 256;
     const long long unit = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     if (unit >= static_cast<long long>(splits) * nqw * M) return;   // whole warps
@@ -154,15 +160,43 @@ __host__ __device__ inline size_t gemv_mma_smem_bytes(int M, int TKC, int warps,
     b += static_cast<size_t>(warps) * stages * gemv_mma_stage_bytes(sz, szw);
     b += static_cast<size_t>(warps) * kSR * 8 * 16;                 // per-box fp32 scale / zero table
     b += gemv_mma_xblock_bytes(M, TKC);
-    b += static_cast<size_t>(warps) * kSR * M * 4;
     b += static_cast<size_t>(warps) * stages * 8 + 8 + 16;
     return b;
 }
 
+// Arguments of gemv_mma_kernel.
+struct GemvMmaArgs {
+    const uint8_t* xblocks;   // [splits] activation blocks from gemv_xfrag_kernel
+    const __half* S;
+    const __half* Z;
+    const uint16_t* bias;
+    uint16_t* Y;
+    float* partial;           // [splits, M, N] when splits > 1
+    float* slots;             // [splits, warps of a slice, 2, 4 rows, M] shared row blocks
+    int* counters;            // [splits, row blocks] boxes finished (zeroed by the prep kernel)
+    int N, K, g, G, sz_row;
+    int TKC;                  // k per slice (a whole number of boxes)
+    int splits;               // slices; CTA c works on slice c / cps
+    int nbs;                  // boxes per slice and row block
+    int nrb;                  // row blocks (4 rows each)
+    int cps;                  // CTAs per slice
+    int stages;               // TMA stages per warp
+    int szw;                  // copy path: scale / zero words per row and stage
+    long long sz_total;       // halves in each of S and Z (N * sz_row, or 1)
+};
+
+// Work split: the boxes of a slice, row block major (box b = row block
+// b / nbs, k box b % nbs), are cut into one contiguous range per warp of
+// the slice's CTAs, so every warp streams the same number of boxes to
+// within one and no warp waits for another.  A row block that one warp
+// covers completely is written at once; a row block shared by neighbouring
+// warps (at most the first and the last of each range) goes through
+// per-warp partial slots, and the warp that completes its box count sums
+// the slots in warp order, so the result does not depend on timing.
 template <int M, int GK, int SZ>
 __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
     gemv_mma_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
-                    const __grid_constant__ CUtensorMap zmap, const GemvStreamArgs a) {
+                    const __grid_constant__ CUtensorMap zmap, const GemvMmaArgs a) {
     static_assert(M >= 1 && M <= 4, "M");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -180,14 +214,13 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
     uint8_t* xblk = reinterpret_cast<uint8_t*>(table + NW * kSR * 8);
     const uint4* frag = reinterpret_cast<const uint4*>(xblk);                // [qw][t][8M]
     const float4* fsc = reinterpret_cast<const float4*>(xblk + static_cast<size_t>(nqw) * M * 512);  // [qw][2M]
-    float* part = reinterpret_cast<float*>(xblk + xbytes);                   // [warp][4 rows][M]
-    uint64_t* full = reinterpret_cast<uint64_t*>(part + NW * kSR * M);
+    uint64_t* full = reinterpret_cast<uint64_t*>(xblk + xbytes);
     uint64_t* xbar = full + NW * NS;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(xbar + 1);
 
     if (tid == 0) {
-        // a stage completes on lane 0's expect-tx arrival and its bytes; the
-        // copy path adds one cp.async arrival per lane
+        // a stage completes on the elected lane's expect-tx arrival and its
+        // bytes; the copy path adds one cp.async arrival per lane
         for (int i = 0; i < NW * NS; ++i) mbar_init(&full[i], SZ == kSzCopy ? 33 : 1);
         mbar_init(xbar, 1);
         *abort_flag = 0;
@@ -202,31 +235,32 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
     }
     __syncthreads();
 
-    const int u_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * a.units / gridDim.x);
-    const int u_end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * a.units / gridDim.x);
-    const int rbl = warp / a.KP, kp = warp - rbl * a.KP;
-    const int b_lo = kp * a.nbs / a.KP;
-    const int BPI = (kp + 1) * a.nbs / a.KP - b_lo;
+    const int slice = blockIdx.x / a.cps;
+    const int W = a.cps * NW;                                   // warps of this slice
+    const int w = (blockIdx.x - slice * a.cps) * NW + warp;
+    const long long T = static_cast<long long>(a.nrb) * a.nbs;  // boxes of the slice
+    auto wstart = [&](int ww) { return static_cast<int>(static_cast<long long>(ww) * T / W); };
+    // the warp whose range holds box b
+    auto warp_of = [&](int b) {
+        return static_cast<int>((static_cast<long long>(b + 1) * W - 1) / T);
+    };
+    const int b_begin = wstart(w), b_end = wstart(w + 1);
     int gshift = 0;
     if (GK == kGroupsPow2) gshift = __ffs(a.g) - 1;
 
     struct Cur {
-        int u, slice, rd, bi;
+        int b, rb, kb;
     };
     auto advance = [&](Cur& c) {
-        if (++c.bi >= BPI) {
-            c.bi = 0;
-            ++c.u;
-            if (++c.rd == a.rounds) {
-                c.rd = 0;
-                ++c.slice;
-            }
+        ++c.b;
+        if (++c.kb == a.nbs) {
+            c.kb = 0;
+            ++c.rb;
         }
     };
-    const int slice0 = u_begin / a.rounds;
-    const Cur start{u_begin, slice0, u_begin - slice0 * a.rounds, 0};
-    auto box_k0 = [&](const Cur& c) { return c.slice * a.TKC + (b_lo + c.bi) * kSBK; };
-    auto box_row0 = [&](const Cur& c) { return (c.rd * a.RBP + rbl) * kSR; };
+    const Cur start{b_begin, b_begin / a.nbs, b_begin - (b_begin / a.nbs) * a.nbs};
+    auto box_k0 = [&](const Cur& c) { return slice * a.TKC + c.kb * kSBK; };
+    auto box_row0 = [&](const Cur& c) { return c.rb * kSR; };
     auto first_group = [&](int k0) {
         if (GK == kGroupsOne) return 0;
         if (GK == kGroupsPow2) return k0 >> gshift;
@@ -237,7 +271,7 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
     int islot = 0;
     Cur ic = start;
     auto issue = [&]() {
-        if (BPI > 0 && ic.u < u_end) {
+        if (ic.b < b_end) {
             const int k0 = box_k0(ic), row0 = box_row0(ic);
             const int st = warp * NS + islot;
             uint8_t* sd = ring + st * SB;
@@ -246,34 +280,40 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
                     (static_cast<long long>(row0 + sz_row_i) * a.sz_row + first_group(k0)) & ~1ll;
                 uint32_t* szd = reinterpret_cast<uint32_t*>(sd + kSBBytes) + (sz_arr * kSR + sz_row_i) * a.szw;
                 const __half* src = sz_arr ? a.Z : a.S;
-                for (int w = lane >> 3; w < a.szw; w += 4) {
-                    const long long hh = h0 + 2 * w;
+                for (int q = lane >> 3; q < a.szw; q += 4) {
+                    const long long hh = h0 + 2 * q;
                     const long long avail = a.sz_total - hh;
                     const uint32_t bytes = avail >= 2 ? 4u : (avail == 1 ? 2u : 0u);
-                    cp_async_4(szd + w, src + (bytes ? hh : 0), bytes);
+                    cp_async_4(szd + q, src + (bytes ? hh : 0), bytes);
                 }
                 cp_async_arrive_noinc(&full[st]);
             }
-            if (lane == 0 && !*abort_flag) {
-                fence_proxy_async_smem();
-                mbar_arrive_expect_tx(&full[st], kSBBytes + kSzTx);
-                tma_load_2d(sd, &wmap, k0 / 8, row0, &full[st]);
-                if (SZ == kSzTma2d) {
-                    const int x = first_group(k0) & ~7;
-                    tma_load_2d(sd + kSBBytes, &smap, x, row0, &full[st]);
-                    tma_load_2d(sd + kSBBytes + 128, &zmap, x, row0, &full[st]);
-                } else if (SZ == kSzTma1d) {
-                    tma_load_2d(sd + kSBBytes, &smap, row0 & ~7, 0, &full[st]);
-                    tma_load_2d(sd + kSBBytes + 128, &zmap, row0 & ~7, 0, &full[st]);
-                }
+            // (after a timed-out wait the loads keep coming; the kernel lets
+            // them land before it exits)
+            if (SZ == kSzTma2d) {
+                const int x = first_group(k0) & ~7;
+                tma_issue_elected<3>(&full[st], kSBBytes + kSzTx, sd, &wmap, k0 / 8, row0, sd + kSBBytes, &smap, x,
+                                     row0, sd + kSBBytes + 128, &zmap, x, row0);
+            } else if (SZ == kSzTma1d) {
+                tma_issue_elected<3>(&full[st], kSBBytes + kSzTx, sd, &wmap, k0 / 8, row0, sd + kSBBytes, &smap,
+                                     row0 & ~7, 0, sd + kSBBytes + 128, &zmap, row0 & ~7, 0);
+            } else {
+                tma_issue_elected<1>(&full[st], kSBBytes, sd, &wmap, k0 / 8, row0);
             }
             if (++islot == NS) islot = 0;
             advance(ic);
         }
     };
-    for (int b = 0; b < NS; ++b) issue();
-    // from here on the prep kernel's activation block is needed
+    // one stage of weights first; then, once the prep kernel is done, the
+    // activation block (so that it does not queue behind the whole ring);
+    // then the rest of the ring
+    issue();
     pdl_wait();
+    if (tid == 0 && b_begin < wstart(NW * (blockIdx.x - slice * a.cps + 1))) {
+        mbar_arrive_expect_tx(xbar, xbytes);
+        bulk_load_1d(xblk, a.xblocks + static_cast<size_t>(slice) * xbytes, xbytes, xbar);
+    }
+    for (int b = 1; b < NS; ++b) issue();
 
     const int wrow = g >> 1, wchunk = (g & 1) * 4 + tig;   // the B chunk this lane loads
     const bool f_lane = g < 2 * M;
@@ -290,120 +330,134 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
     }
     float4* wtable = table + warp * kSR * 8;
     const int tq = lane & 7, ti = lane >> 3;               // table entry this lane builds
+    if (b_begin < b_end) mbar_wait_bounded(xbar, 0, abort_flag, kErrTimeoutTmaFull);
+
+    // the outputs of row block rb: lanes with even g < 2M hold (m = g / 2,
+    // row tig) after the digit shuffle
+    auto store = [&](int m, int n, float v) {
+        if (a.splits == 1) {
+            if (a.bias) v += bf16_bits_to_float(a.bias[n]);
+            a.Y[static_cast<size_t>(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        } else {
+            a.partial[(static_cast<size_t>(slice) * M + m) * a.N + n] = v;
+        }
+    };
+    const int first_rb = start.rb;
+    auto finish = [&](int rb, int nb, float y) {
+        const float v = y + __shfl_xor_sync(0xFFFFFFFFu, y, 4);
+        const bool out_lane = !(g & 1) && f_lane;
+        if (nb == a.nbs) {
+            const int n = rb * kSR + tig;
+            if (out_lane && n < a.N) store(g >> 1, n, v);
+            return;
+        }
+        float* sl = a.slots + ((static_cast<size_t>(slice) * W + w) * 2 + (rb == first_rb ? 0 : 1)) * (kSR * M);
+        if (out_lane) sl[tig * M + (g >> 1)] = v;
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) last = (atomicAdd(&a.counters[slice * a.nrb + rb], nb) + nb == a.nbs);
+        last = __shfl_sync(0xFFFFFFFFu, last, 0);
+        if (!last) return;
+        __threadfence();
+        const int w0 = warp_of(rb * a.nbs), w1 = warp_of(rb * a.nbs + a.nbs - 1);
+        if (lane < kSR * M) {
+            const int r = lane / M, m = lane - (lane / M) * M;
+            float s = 0.0f;
+            for (int ww = w0; ww <= w1; ++ww) {
+                const int ws = wstart(ww);
+                if (ws == wstart(ww + 1)) continue;
+                const int sslot = (ws / a.nbs == rb) ? 0 : 1;
+                s += __ldcg(a.slots + ((static_cast<size_t>(slice) * W + ww) * 2 + sslot) * (kSR * M) + r * M + m);
+            }
+            const int n = rb * kSR + r;
+            if (n < a.N) store(m, n, s);
+        }
+    };
 
     int cslot = 0;
-    uint32_t cpar = 0, xpar = 0;
+    uint32_t cpar = 0;
     Cur cc = start;
-    int cur_slice = -1;
-
-    for (int u = u_begin; u < u_end; ++u) {
-        const int slice = cc.slice, rd = cc.rd;
-        if (slice != cur_slice) {
-            if (tid == 0 && !*abort_flag) {
-                fence_proxy_async_smem();
-                mbar_arrive_expect_tx(xbar, xbytes);
-                bulk_load_1d(xblk, a.xblocks + static_cast<size_t>(slice) * xbytes, xbytes, xbar);
-            }
-            mbar_wait_bounded(xbar, xpar, abort_flag, kErrTimeoutTmaFull);
-            xpar ^= 1u;
-            cur_slice = slice;
+    float y = 0.0f;
+    int nb_rb = 0;
+    for (int b = b_begin; b < b_end; ++b) {
+        const int k0 = box_k0(cc), row0 = box_row0(cc);
+        const int st = warp * NS + cslot;
+        __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[st], cpar, abort_flag, kErrTimeoutTmaFull));
+        if (++cslot == NS) {
+            cslot = 0;
+            cpar ^= 1u;
         }
-        float y = 0.0f;
-
-        for (int bi = 0; bi < BPI; ++bi) {
-            const int k0 = box_k0(cc), row0 = box_row0(cc);
-            const int st = warp * NS + cslot;
-            __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[st], cpar, abort_flag, kErrTimeoutTmaFull));
-            if (++cslot == NS) {
-                cslot = 0;
-                cpar ^= 1u;
+        const uint8_t* sb = ring + st * SB;
+        if (SZ != kSzConst) {
+            // fp32 table of (s, z) for window tq, row ti, both halves (the 4
+            // rows of a window are adjacent: the readers hit 4 distinct banks)
+            const int grp_lo = first_group(k0);
+            int o0, o1;
+            if (GK == kGroupsOne) {
+                o0 = 0;
+                o1 = 0;
+            } else if (GK == kGroupsPow2) {
+                o0 = (tq * 256) >> gshift;
+                o1 = (tq * 256 + 128) >> gshift;
+            } else {
+                const int r0 = k0 - grp_lo * a.g;
+                o0 = (r0 + tq * 256) / a.g;
+                o1 = (r0 + tq * 256 + 128) / a.g;
             }
-            const uint8_t* sb = ring + st * SB;
-            if (SZ != kSzConst) {
-                // fp32 table of (s, z) for window tq, row ti, both halves (the 4
-                // rows of a window are adjacent: the readers hit 4 distinct banks)
-                const int grp_lo = first_group(k0);
-                int o0, o1;
-                if (GK == kGroupsOne) {
-                    o0 = 0;
-                    o1 = 0;
-                } else if (GK == kGroupsPow2) {
-                    o0 = (tq * 256) >> gshift;
-                    o1 = (tq * 256 + 128) >> gshift;
-                } else {
-                    const int r0 = k0 - grp_lo * a.g;
-                    o0 = (r0 + tq * 256) / a.g;
-                    o1 = (r0 + tq * 256 + 128) / a.g;
-                }
-                const __half* sh = reinterpret_cast<const __half*>(sb + kSBBytes);
-                const __half *ps, *pz;
-                if (SZ == kSzTma2d) {
-                    ps = sh + ti * 16 + (grp_lo & 7);
-                    pz = ps + 64;                    // Z box 128 bytes after the S box
-                } else if (SZ == kSzTma1d) {
-                    ps = sh + (row0 & 7) + ti;
-                    pz = ps + 64;
-                } else {
-                    ps = sh + ti * 2 * a.szw + ((((row0 + ti) & a.sz_row) ^ grp_lo) & 1);
-                    pz = ps + kSR * 2 * a.szw;
-                }
-                wtable[tq * kSR + ti] = make_float4(__half2float(ps[o0]), __half2float(pz[o0]), __half2float(ps[o1]),
-                                                  __half2float(pz[o1]));
-                __syncwarp();
+            const __half* sh = reinterpret_cast<const __half*>(sb + kSBBytes);
+            const __half *ps, *pz;
+            if (SZ == kSzTma2d) {
+                ps = sh + ti * 16 + (grp_lo & 7);
+                pz = ps + 64;                    // Z box 128 bytes after the S box
+            } else if (SZ == kSzTma1d) {
+                ps = sh + (row0 & 7) + ti;
+                pz = ps + 64;
+            } else {
+                ps = sh + ti * 2 * a.szw + ((((row0 + ti) & a.sz_row) ^ grp_lo) & 1);
+                pz = ps + kSR * 2 * a.szw;
             }
-            // per-box bases: every window below is an immediate offset from them
-            const uint8_t* wsrc = sb + wrow * 1024 + wchunk * 16;
-            const int qw0 = (b_lo + bi) * (kSBK / 256);
-            const uint4* fb = frag + qw0 * (32 * M) + lane;
-            const float4* cb = fsc + qw0 * (2 * M) + g;
-#pragma unroll
-            for (int qwl = 0; qwl < kSBK / 256; ++qwl) {
-                const uint4 wv = *reinterpret_cast<const uint4*>(wsrc + qwl * 128);
-                if (lane < 8 * M) {
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) af[t] = fb[(qwl * 4 + t) * (8 * M)];
-                }
-                if (f_lane) f = cb[qwl * 2 * M];
-                int acc[2][4];
-                mma_s8u8_16832_z(acc[0], af[0], wv.x & 0x0F0F0F0Fu, (wv.x >> 4) & 0x0F0F0F0Fu);
-                mma_s8u8_16832_z(acc[1], af[1], wv.y & 0x0F0F0F0Fu, (wv.y >> 4) & 0x0F0F0F0Fu);
-                mma_s8u8_16832(acc[0], af[2], wv.z & 0x0F0F0F0Fu, (wv.z >> 4) & 0x0F0F0F0Fu);
-                mma_s8u8_16832(acc[1], af[3], wv.w & 0x0F0F0F0Fu, (wv.w >> 4) & 0x0F0F0F0Fu);
-                const int d0 = acc[0][0] + acc[1][0];   // half 0: A row g, B column (tig, 0)
-                const int d1 = acc[0][3] + acc[1][3];   // half 1: A row g + 8, B column (tig, 1)
-                float4 sz;
-                if (SZ == kSzConst) sz = make_float4(s_const, z_const, s_const, z_const);
-                else sz = wtable[qwl * kSR + tig];
-                y = fmaf(sz.x, fmaf(f.x, static_cast<float>(d0), -sz.y * f.y), y);
-                y = fmaf(sz.z, fmaf(f.z, static_cast<float>(d1), -sz.w * f.w), y);
-            }
+            wtable[tq * kSR + ti] = make_float4(__half2float(ps[o0]), __half2float(pz[o0]), __half2float(ps[o1]),
+                                                __half2float(pz[o1]));
             __syncwarp();
-            issue();
-            advance(cc);
         }
-
-        // end of the item: add the two digits of each (m, row); lanes with
-        // even g < 2M then hold y[m = g / 2][row tig]
-        y += __shfl_xor_sync(0xFFFFFFFFu, y, 4);
-        if (!(g & 1) && f_lane) part[(warp * kSR + tig) * M + (g >> 1)] = y;
-        __syncthreads();
-        for (int o = tid; o < a.RBP * kSR * M; o += NW * 32) {
-            const int rb2 = o / (kSR * M);
-            const int rem = o - rb2 * kSR * M;
-            const int r = rem / M, m = rem - (rem / M) * M;
-            const int n = (rd * a.RBP + rb2) * kSR + r;
-            if (n < a.N) {
-                float sacc = 0.0f;
-                for (int p = 0; p < a.KP; ++p) sacc += part[((rb2 * a.KP + p) * kSR + r) * M + m];
-                if (a.splits == 1) {
-                    if (a.bias) sacc += bf16_bits_to_float(a.bias[n]);
-                    a.Y[static_cast<size_t>(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(sacc));
-                } else {
-                    a.partial[(static_cast<size_t>(slice) * M + m) * a.N + n] = sacc;
-                }
+        // per-box bases: every window below is an immediate offset from them
+        const uint8_t* wsrc = sb + wrow * 1024 + wchunk * 16;
+        const int qw0 = cc.kb * (kSBK / 256);
+        const uint4* fb = frag + qw0 * (32 * M) + lane;
+        const float4* cb = fsc + qw0 * (2 * M) + g;
+#pragma unroll
+        for (int qwl = 0; qwl < kSBK / 256; ++qwl) {
+            const uint4 wv = *reinterpret_cast<const uint4*>(wsrc + qwl * 128);
+            if (lane < 8 * M) {
+#pragma unroll
+                for (int t = 0; t < 4; ++t) af[t] = fb[(qwl * 4 + t) * (8 * M)];
             }
+            if (f_lane) f = cb[qwl * 2 * M];
+            int acc[2][4];
+            mma_s8u8_16832_z(acc[0], af[0], wv.x & 0x0F0F0F0Fu, (wv.x >> 4) & 0x0F0F0F0Fu);
+            mma_s8u8_16832_z(acc[1], af[1], wv.y & 0x0F0F0F0Fu, (wv.y >> 4) & 0x0F0F0F0Fu);
+            mma_s8u8_16832(acc[0], af[2], wv.z & 0x0F0F0F0Fu, (wv.z >> 4) & 0x0F0F0F0Fu);
+            mma_s8u8_16832(acc[1], af[3], wv.w & 0x0F0F0F0Fu, (wv.w >> 4) & 0x0F0F0F0Fu);
+            const int d0 = acc[0][0] + acc[1][0];   // half 0: A row g, B column (tig, 0)
+            const int d1 = acc[0][3] + acc[1][3];   // half 1: A row g + 8, B column (tig, 1)
+            float4 sz;
+            if (SZ == kSzConst) sz = make_float4(s_const, z_const, s_const, z_const);
+            else sz = wtable[qwl * kSR + tig];
+            y = fmaf(sz.x, fmaf(f.x, static_cast<float>(d0), -sz.y * f.y), y);
+            y = fmaf(sz.z, fmaf(f.z, static_cast<float>(d1), -sz.w * f.w), y);
         }
-        __syncthreads();
+        __syncwarp();
+        issue();
+        ++nb_rb;
+        const int rb = cc.rb;
+        const bool rb_done = (cc.kb == a.nbs - 1) || (b == b_end - 1);
+        advance(cc);
+        if (rb_done) {
+            finish(rb, nb_rb, y);
+            y = 0.0f;
+            nb_rb = 0;
+        }
     }
     if (*abort_flag) {
         const unsigned long long t0 = global_timer_ns();

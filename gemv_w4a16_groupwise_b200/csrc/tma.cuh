@@ -90,6 +90,44 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
+// One elected lane of the warp orders the warp's earlier shared-memory
+// reads before the async proxy's writes, arms `bar` for `bytes` and issues
+// N (1 or 3) 2-D TMA loads that complete on it.  Every lane computes the
+// same operands; only the election is predicated, so the warp does not
+// diverge.
+template <int N>
+__device__ __forceinline__ void tma_issue_elected(uint64_t* bar, uint32_t bytes, void* d0, const CUtensorMap* m0,
+                                                  int x0, int y0, void* d1 = nullptr, const CUtensorMap* m1 = nullptr,
+                                                  int x1 = 0, int y1 = 0, void* d2 = nullptr,
+                                                  const CUtensorMap* m2 = nullptr, int x2 = 0, int y2 = 0) {
+    static_assert(N == 1 || N == 3, "N");
+    if (N == 1) {
+        asm volatile(
+            "{\n .reg .pred P;\n elect.sync _|P, 0xffffffff;\n"
+            " @P fence.proxy.async.shared::cta;\n"
+            " @P mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n"
+            " @P cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%2], [%3, {%4, %5}], [%0];\n}\n" ::"r"(smem_u32(bar)),
+            "r"(bytes), "r"(smem_u32(d0)), "l"(reinterpret_cast<uint64_t>(m0)), "r"(x0), "r"(y0)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n .reg .pred P;\n elect.sync _|P, 0xffffffff;\n"
+            " @P fence.proxy.async.shared::cta;\n"
+            " @P mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n"
+            " @P cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%2], [%3, {%4, %5}], [%0];\n"
+            " @P cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%6], [%7, {%8, %9}], [%0];\n"
+            " @P cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%10], [%11, {%12, %13}], [%0];\n}\n" ::"r"(smem_u32(bar)),
+            "r"(bytes), "r"(smem_u32(d0)), "l"(reinterpret_cast<uint64_t>(m0)), "r"(x0), "r"(y0),
+            "r"(smem_u32(d1)), "l"(reinterpret_cast<uint64_t>(m1)), "r"(x1), "r"(y1), "r"(smem_u32(d2)),
+            "l"(reinterpret_cast<uint64_t>(m2)), "r"(x2), "r"(y2)
+            : "memory");
+    }
+}
+
 // Named barrier over `count` threads (ids 1..15; id 0 is __syncthreads).
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

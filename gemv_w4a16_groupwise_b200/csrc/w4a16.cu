@@ -255,8 +255,9 @@ struct StreamPlan {
     bool ok = false;
     int TKC = 0, splits = 1, nbs = 0, KP = 1, RBP = kSW, rounds = 0, units = 0, grid = 0, stages = 2;
     int szw = 0, warps = kSW, sz = 0;
+    int nrb = 0, cps = 0;                      // tensor-pipe kernel: row blocks, CTAs per slice
     bool mma = false;
-    size_t smem = 0, xbytes = 0, ws = 0, partial_off = 0;
+    size_t smem = 0, xbytes = 0, ws = 0, partial_off = 0, slots_off = 0, cnt_off = 0;
 };
 
 // szw: scale / zero words per stage row (gemv_stream_sz_words of the group
@@ -350,29 +351,19 @@ StreamPlan plan_mma(int M, int N, int K, int sz, int szw, const DeviceInfo& di) 
     p.splits = (nb_total + nbs_max - 1) / nbs_max;
     p.nbs = (nb_total + p.splits - 1) / p.splits;
     p.TKC = p.nbs * kSBK;
-    const int nrb = (N + kSR - 1) / kSR;
-    double best = 1e300;
-    for (int KP = 1; KP <= p.warps && KP <= p.nbs; ++KP) {
-        if (p.warps % KP) continue;
-        const int RBP = p.warps / KP;
-        const int rounds = (nrb + RBP - 1) / RBP;
-        const int units = p.splits * rounds;
-        const int grid = std::min(units, di.sms);
-        const int per_cta = (units + grid - 1) / grid;
-        const double cost = per_cta * ((p.nbs + KP - 1) / KP + 0.5);
-        if (cost < best * 0.999) {
-            best = cost;
-            p.KP = KP;
-            p.RBP = RBP;
-            p.rounds = rounds;
-            p.units = units;
-            p.grid = grid;
-        }
-    }
+    p.nrb = (N + kSR - 1) / kSR;
+    // CTAs per slice: all the SMs, unless the slice has fewer boxes than warps
+    const long long boxes = static_cast<long long>(p.nrb) * p.nbs;
+    p.cps = static_cast<int>(std::max<long long>(
+        1, std::min<long long>(di.sms / p.splits, (boxes + p.warps - 1) / p.warps)));
+    p.grid = p.splits * p.cps;
     p.smem = gemv_mma_smem_bytes(M, p.TKC, p.warps, p.stages, sz, szw);
     p.xbytes = gemv_mma_xblock_bytes(M, p.TKC);
-    p.partial_off = (p.splits * p.xbytes + 255) / 256 * 256;
-    p.ws = p.partial_off + (p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * sizeof(float) : 0);
+    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
+    p.partial_off = up(p.splits * p.xbytes);
+    p.slots_off = p.partial_off + up(p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * sizeof(float) : 0);
+    p.cnt_off = p.slots_off + up(static_cast<size_t>(p.splits) * p.cps * p.warps * 2 * kSR * M * sizeof(float));
+    p.ws = p.cnt_off + up(static_cast<size_t>(p.splits) * p.nrb * sizeof(int));
     p.mma = true;
     p.ok = true;
     return p;
@@ -517,7 +508,7 @@ w4_status launch_gemv_stream(const StreamPlan& p, const CUtensorMap& map, const 
 // before it: its prologue and first weight loads overlap the prep kernel.
 template <int M, int GK, int SZ>
 w4_status launch_gemv_mma_k(const StreamPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
-                            const CUtensorMap& zm, const GemvStreamArgs& a, cudaStream_t st) {
+                            const CUtensorMap& zm, const GemvMmaArgs& a, cudaStream_t st) {
     auto* fn = gemv_mma_kernel<M, GK, SZ>;
     if (ensure_smem(reinterpret_cast<const void*>(fn), p.smem) != cudaSuccess) return W4_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
@@ -536,7 +527,7 @@ w4_status launch_gemv_mma_k(const StreamPlan& p, const CUtensorMap& wm, const CU
 
 template <int M, int GK>
 w4_status launch_gemv_mma_gk(const StreamPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
-                             const CUtensorMap& zm, const GemvStreamArgs& a, cudaStream_t st) {
+                             const CUtensorMap& zm, const GemvMmaArgs& a, cudaStream_t st) {
     switch (p.sz) {
         case kSzConst: return launch_gemv_mma_k<M, GK, kSzConst>(p, wm, sm, zm, a, st);
         case kSzTma2d: return launch_gemv_mma_k<M, GK, kSzTma2d>(p, wm, sm, zm, a, st);
@@ -547,14 +538,14 @@ w4_status launch_gemv_mma_gk(const StreamPlan& p, const CUtensorMap& wm, const C
 
 template <int M>
 w4_status launch_gemv_mma_m(const StreamPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
-                            const CUtensorMap& zm, const GemvStreamArgs& a, cudaStream_t st) {
+                            const CUtensorMap& zm, const GemvMmaArgs& a, cudaStream_t st) {
     if (a.G == 1) return launch_gemv_mma_gk<M, kGroupsOne>(p, wm, sm, zm, a, st);
     if (kSBK % a.g == 0) return launch_gemv_mma_gk<M, kGroupsPow2>(p, wm, sm, zm, a, st);
     return launch_gemv_mma_gk<M, kGroupsAny>(p, wm, sm, zm, a, st);
 }
 
 w4_status launch_gemv_mma(const StreamPlan& p, int M, const CUtensorMap& wm, const void* S, const void* Z,
-                          const GemvStreamArgs& a, cudaStream_t st) {
+                          const GemvMmaArgs& a, cudaStream_t st) {
     CUtensorMap sm, zm;
     std::memset(&sm, 0, sizeof sm);
     std::memset(&zm, 0, sizeof zm);
@@ -581,58 +572,86 @@ w4_status run_gemv_stream(const StreamPlan& p, int M, int N, int K, const void* 
     if (p.ws > ws_bytes || ws == nullptr) return W4_ERR_WORKSPACE;
     if (!aligned16(ws)) return W4_ERR_ALIGNMENT;
     uint8_t* xb = static_cast<uint8_t*>(ws);
+    float* partial = p.splits > 1 ? reinterpret_cast<float*>(xb + p.partial_off) : nullptr;
+    CUtensorMap map;
+    if (!make_map_2d(&map, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, kSR, kSBK / 8, 0))
+        return W4_ERR_CUDA;
+    w4_status s = W4_OK;
     if (p.mma) {
+        int* counters = reinterpret_cast<int*>(xb + p.cnt_off);
+        const int ncounters = p.splits * p.nrb;
         const long long lanes = static_cast<long long>(p.splits) * (p.TKC / 256) * M * 32;
         gemv_xfrag_kernel<<<static_cast<int>((lanes + 255) / 256), 256, 0, st>>>(
-            static_cast<const uint16_t*>(A), M, K, p.TKC, p.splits, xb);
+            static_cast<const uint16_t*>(A), M, K, p.TKC, p.splits, xb, counters, ncounters);
+        s = launch_status();
+        if (s != W4_OK) return s;
+        GemvMmaArgs a;
+        a.xblocks = xb;
+        a.S = static_cast<const __half*>(S);
+        a.Z = static_cast<const __half*>(Z);
+        a.bias = static_cast<const uint16_t*>(bias);
+        a.Y = static_cast<uint16_t*>(Y);
+        a.partial = partial;
+        a.slots = reinterpret_cast<float*>(xb + p.slots_off);
+        a.counters = counters;
+        a.N = N;
+        a.K = K;
+        a.g = meta.g;
+        a.G = meta.G;
+        a.sz_row = meta.sz_row;
+        a.TKC = p.TKC;
+        a.splits = p.splits;
+        a.nbs = p.nbs;
+        a.nrb = p.nrb;
+        a.cps = p.cps;
+        a.stages = p.stages;
+        a.szw = p.szw;
+        a.sz_total = meta.sz_row ? static_cast<long long>(N) * meta.sz_row : 1;
+        s = launch_gemv_mma(p, M, map, S, Z, a, st);
     } else {
         const long long chunks = static_cast<long long>(p.splits) * M * (p.TKC / 32);
         gemv_xprep_kernel<<<static_cast<int>((chunks + 255) / 256), 256, 0, st>>>(
             static_cast<const uint16_t*>(A), M, K, p.TKC, p.splits, xb);
-    }
-    w4_status s = launch_status();
-    if (s != W4_OK) return s;
-    CUtensorMap map;
-    if (!make_map_2d(&map, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, kSR, kSBK / 8, 0))
-        return W4_ERR_CUDA;
-    GemvStreamArgs a;
-    a.xblocks = xb;
-    a.S = static_cast<const __half*>(S);
-    a.Z = static_cast<const __half*>(Z);
-    a.bias = static_cast<const uint16_t*>(bias);
-    a.Y = static_cast<uint16_t*>(Y);
-    a.partial = p.splits > 1 ? reinterpret_cast<float*>(xb + p.partial_off) : nullptr;
-    a.N = N;
-    a.K = K;
-    a.g = meta.g;
-    a.G = meta.G;
-    a.sz_row = meta.sz_row;
-    a.TKC = p.TKC;
-    a.splits = p.splits;
-    a.nbs = p.nbs;
-    a.KP = p.KP;
-    a.RBP = p.RBP;
-    a.rounds = p.rounds;
-    a.units = p.units;
-    a.stages = p.stages;
-    a.szw = p.szw;
-    a.sz_total = meta.sz_row ? static_cast<long long>(N) * meta.sz_row : 1;
-    a.M = M;
-    if (p.mma) {
-        s = launch_gemv_mma(p, M, map, S, Z, a, st);
-    } else switch (M) {
-        case 1: s = launch_gemv_stream<1>(p, map, a, st); break;
-        case 2: s = launch_gemv_stream<2>(p, map, a, st); break;
-        case 3: s = launch_gemv_stream<3>(p, map, a, st); break;
-        case 4: s = launch_gemv_stream<4>(p, map, a, st); break;
-        default: return W4_ERR_INVALID_ARG;
+        s = launch_status();
+        if (s != W4_OK) return s;
+        GemvStreamArgs a;
+        a.xblocks = xb;
+        a.S = static_cast<const __half*>(S);
+        a.Z = static_cast<const __half*>(Z);
+        a.bias = static_cast<const uint16_t*>(bias);
+        a.Y = static_cast<uint16_t*>(Y);
+        a.partial = partial;
+        a.N = N;
+        a.K = K;
+        a.g = meta.g;
+        a.G = meta.G;
+        a.sz_row = meta.sz_row;
+        a.TKC = p.TKC;
+        a.splits = p.splits;
+        a.nbs = p.nbs;
+        a.KP = p.KP;
+        a.RBP = p.RBP;
+        a.rounds = p.rounds;
+        a.units = p.units;
+        a.stages = p.stages;
+        a.szw = p.szw;
+        a.sz_total = meta.sz_row ? static_cast<long long>(N) * meta.sz_row : 1;
+        a.M = M;
+        switch (M) {
+            case 1: s = launch_gemv_stream<1>(p, map, a, st); break;
+            case 2: s = launch_gemv_stream<2>(p, map, a, st); break;
+            case 3: s = launch_gemv_stream<3>(p, map, a, st); break;
+            case 4: s = launch_gemv_stream<4>(p, map, a, st); break;
+            default: return W4_ERR_INVALID_ARG;
+        }
     }
     if (s != W4_OK) return s;
     if (p.splits > 1) {
         const DeviceInfo di = device_info(current_device());
         const long long total = static_cast<long long>(M) * N;
         const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, di.sms * 8));
-        splits_finalize_kernel<<<blocks, 256, 0, st>>>(a.partial, p.splits, M, N, a.bias, a.Y);
+        splits_finalize_kernel<<<blocks, 256, 0, st>>>(partial, p.splits, M, N, static_cast<const uint16_t*>(bias),
+                                                        static_cast<uint16_t*>(Y));
         return launch_status();
     }
     return W4_OK;
