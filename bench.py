@@ -110,7 +110,7 @@ def source_hash():
 
 
 def committed_traffic():
-    """DRAM bytes per launch of the sweep from the committed ncu summary,
+    """DRAM bytes of one sweep step from the committed ncu summary,
     if it was taken on the current kernel sources (else None)."""
     path = os.path.join(ROOT, "profiles", "gemv_fwd_decode_sweep_traffic.json")
     try:
@@ -120,7 +120,7 @@ def committed_traffic():
         return None
     if t.get("source_hash") != source_hash():
         return None
-    return t.get("dram_bytes_per_launch")
+    return t.get("dram_bytes_per_step")
 
 
 # ------------------------------------------------------------- clock sampler
@@ -495,8 +495,8 @@ def run_ours(args):
         cpu = None
         if ws_ == 1 and not args.no_cpu:
             cpu = cpu_baseline(args.cpu_seconds, sizes)
-        per_launch_ms = ms_step / launches_per_step
-        alg_per_launch = bytes_step / launches_per_step
+        calls = len(cases)
+        alg_per_call = bytes_step / calls
         traffic = committed_traffic()
         out = {
             "metric": METRIC,
@@ -522,15 +522,21 @@ def run_ours(args):
             },
             "roofline": {
                 "bound": "hbm",
-                "achieved": round(alg_per_launch / (per_launch_ms * 1e-3) / 1e9, 2),
+                "achieved": round(alg_per_call / (ms_step / calls * 1e-3) / 1e9, 2),
                 "peak": peaks["hbm_gbs"],
                 "unit": "GB/s",
-                "frac": round(alg_per_launch / (per_launch_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-                "traffic": traffic,
+                "frac": round(alg_per_call / (ms_step / calls * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                "traffic": (round(traffic / calls) if traffic is not None else None),
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
                                else "fallback 6.65 TB/s",
-                "kernel": "gemv_fwd_tma_kernel (+ split finalize)",
-                "alg_bytes_per_launch": round(alg_per_launch),
+                "kernel": "gemv_mma_kernel, timed together with its gemv_xfrag_kernel prep "
+                          "(one GEMV call = 2 launches)",
+                "per": "GEMV call, averaged over the 40 calls of a step (CUDA events on the launching "
+                       "stream around the whole timed region)",
+                "alg_bytes_per_launch": round(alg_per_call),
+                "traffic_source": "profiles/gemv_fwd_decode_sweep_traffic.json (ncu dram__bytes_read.sum + "
+                                  "dram__bytes_write.sum of both kernels, one step; null when the kernel "
+                                  "sources changed since)",
             },
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h,

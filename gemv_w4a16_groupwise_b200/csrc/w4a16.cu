@@ -175,59 +175,7 @@ w4_status launch_status() {
     return W4_ERR_CUDA;
 }
 
-int gcd_int(int a, int b) {
-    while (b) {
-        const int t = a % b;
-        a = b;
-        b = t;
-    }
-    return a;
-}
-
 // -------------------------------------------------------- GEMV planning
-struct FwdPlan {
-    bool tma = false;
-    int F = 0, TK = 0, splits = 1, row_tiles = 0, units = 0, grid = 0;
-    size_t smem = 0, ws = 0;
-};
-
-FwdPlan plan_fwd(int M, int N, int K, const Meta& meta, int sms) {
-    FwdPlan p;
-    p.tma = (K % 32 == 0) && (meta.g % 32 == 0);
-    if (!p.tma) return p;
-    p.F = gcd_int(meta.g, kGemvBoxK);
-    p.row_tiles = (N + kGemvTileRows - 1) / kGemvTileRows;
-    const int tk_max = (M == 1) ? 16384 : (M == 2) ? 8192 : (M == 3) ? 5120 : 4096;
-    const int k_pad = (K + kGemvBoxK - 1) / kGemvBoxK * kGemvBoxK;
-    const int s_min = (k_pad + tk_max - 1) / tk_max;
-    const int s_max = std::max(s_min, k_pad / kGemvBoxK);
-    double best = -1.0;
-    for (int s = s_min; s <= std::min(s_max, s_min * 16); ++s) {
-        int tk = (k_pad + s - 1) / s;
-        tk = (tk + kGemvBoxK - 1) / kGemvBoxK * kGemvBoxK;
-        const int se = (K + tk - 1) / tk;
-        const long long units = static_cast<long long>(p.row_tiles) * se;
-        const long long waves = (units + sms - 1) / sms;
-        // per-SM serial bytes vs the ideal even share of the weights
-        const double ideal = static_cast<double>(N) * K / 2.0 / sms;
-        const double real = static_cast<double>(waves) * tk * kGemvTileRows / 2.0;
-        double eff = ideal / real;
-        const int nb = tk / kGemvBoxK;
-        if (nb < kGemvConsumerWarps) eff *= 0.5 + 0.5 * nb / kGemvConsumerWarps;  // idle warps
-        if (se > 1) eff *= 1.0 - std::min(0.5, 16.0 * se * M / K);               // partials
-        if (eff > best * 1.02) {
-            best = eff;
-            p.TK = tk;
-            p.splits = se;
-            p.units = static_cast<int>(units);
-        }
-    }
-    p.grid = std::min(p.units, sms);
-    p.smem = gemv_fwd_smem_bytes(M, p.TK, p.F);
-    p.ws = p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * sizeof(float) : 0;
-    return p;
-}
-
 struct TPlan {
     int splits = 1, rows_per_split = 0;
     size_t ws = 0;
@@ -396,95 +344,6 @@ size_t gemv_workspace(int M, int N, int K, int transposed, int sms) {
         }
     }
     return ws;
-}
-
-template <int M>
-w4_status launch_gemv_fwd(const FwdPlan& p, const CUtensorMap& map, const GemvFwdArgs& a,
-                          cudaStream_t st) {
-    const void* fn = nullptr;
-    switch (p.F) {
-        case 32: fn = reinterpret_cast<const void*>(gemv_fwd_tma_kernel<M, 32>); break;
-        case 64: fn = reinterpret_cast<const void*>(gemv_fwd_tma_kernel<M, 64>); break;
-        case 128: fn = reinterpret_cast<const void*>(gemv_fwd_tma_kernel<M, 128>); break;
-        default: return W4_ERR_UNSUPPORTED;
-    }
-    if (ensure_smem(fn, p.smem) != cudaSuccess) return W4_ERR_CUDA;
-    switch (p.F) {
-        case 32: gemv_fwd_tma_kernel<M, 32><<<p.grid, kGemvThreads, p.smem, st>>>(map, a); break;
-        case 64: gemv_fwd_tma_kernel<M, 64><<<p.grid, kGemvThreads, p.smem, st>>>(map, a); break;
-        case 128: gemv_fwd_tma_kernel<M, 128><<<p.grid, kGemvThreads, p.smem, st>>>(map, a); break;
-    }
-    return launch_status();
-}
-
-// Lanes-along-K GEMV for M <= 2 (gemv_rows_kernel): chunk = 32 k inside one
-// group, so K % 32 == 0 and g % 32 == 0.  Picks the warps per CTA and the
-// rows per round so that the persistent grid covers the SMs.
-struct RowsPlan {
-    bool ok = false;
-    int NW = 16, KB = 0, RBP = 1, rounds = 0, grid = 0;
-    size_t smem = 0;
-};
-
-RowsPlan plan_rows(int M, int N, int K, const Meta& meta, const DeviceInfo& di) {
-    RowsPlan best;
-    if (M > 2 || K % 32 != 0 || meta.g % 32 != 0) return best;
-    const int KB = (K + 1023) / 1024;
-    const int nrb = (N + kRowsRB - 1) / kRowsRB;
-    double best_score = -1.0;
-    for (int NW : {16, 8, 4}) {
-        RowsPlan p;
-        p.NW = NW;
-        p.KB = KB;
-        p.RBP = NW / gcd_int(KB, NW);
-        p.rounds = (nrb + p.RBP - 1) / p.RBP;
-        p.smem = gemv_rows_smem_bytes(M, KB, p.RBP);
-        if (p.smem > static_cast<size_t>(di.max_smem_optin)) continue;
-        const int by_smem = std::max(1, static_cast<int>((228 * 1024) / (p.smem + 1024)));
-        const int by_threads = 2048 / (NW * 32);
-        const int by_regs = 65536 / (NW * 32 * (M == 1 ? 64 : 128));
-        const int occ = std::max(1, std::min(by_smem, std::min(by_threads, by_regs)));
-        p.grid = std::min(p.rounds, di.sms * occ);
-        const long long per_cta = (p.rounds + p.grid - 1) / p.grid;
-        // warps kept busy, discounted by round imbalance and by the staging
-        // every CTA repeats (M * K activations)
-        const double busy = static_cast<double>(p.grid) * NW * p.rounds / (per_cta * p.grid);
-        const double work = static_cast<double>(per_cta) * p.RBP * kRowsRB * K;  // weights per CTA
-        const double stage = 8.0 * M * K;
-        const double score = busy * work / (work + stage);
-        if (score > best_score) {
-            best_score = score;
-            best = p;
-            best.ok = true;
-        }
-    }
-    return best;
-}
-
-w4_status run_gemv_rows(const RowsPlan& p, int M, int N, int K, const void* A, const uint32_t* packed,
-                        const void* S, const void* Z, const Meta& meta, const void* bias, void* Y,
-                        cudaStream_t st) {
-    GemvRowsArgs a;
-    a.X = static_cast<const uint16_t*>(A);
-    a.packed = packed;
-    a.S = static_cast<const __half*>(S);
-    a.Z = static_cast<const __half*>(Z);
-    a.bias = static_cast<const uint16_t*>(bias);
-    a.Y = static_cast<uint16_t*>(Y);
-    a.N = N;
-    a.K = K;
-    a.g = meta.g;
-    a.G = meta.G;
-    a.sz_row = meta.sz_row;
-    a.KB = p.KB;
-    a.RBP = p.RBP;
-    a.rounds = p.rounds;
-    const void* fn = M == 1 ? reinterpret_cast<const void*>(gemv_rows_kernel<1>)
-                            : reinterpret_cast<const void*>(gemv_rows_kernel<2>);
-    if (ensure_smem(fn, p.smem) != cudaSuccess) return W4_ERR_CUDA;
-    if (M == 1) gemv_rows_kernel<1><<<p.grid, p.NW * 32, p.smem, st>>>(a);
-    else gemv_rows_kernel<2><<<p.grid, p.NW * 32, p.smem, st>>>(a);
-    return launch_status();
 }
 
 template <int M, int GK>
@@ -667,54 +526,27 @@ w4_status run_gemv_fwd(const void* A, int M, int N, int K, const uint32_t* packe
         if (!sp.ok) sp = plan_stream(M, N, K, meta, di);
         if (sp.ok) return run_gemv_stream(sp, M, N, K, A, packed, S, Z, meta, bias, Y, ws, ws_bytes, st);
     }
-    const FwdPlan p = plan_fwd(M, N, K, meta, di.sms);
+    // K or the group length not a multiple of 32: one warp per output row
     GemvFwdArgs a;
     a.X = static_cast<const uint16_t*>(A);
     a.S = static_cast<const __half*>(S);
     a.Z = static_cast<const __half*>(Z);
     a.bias = static_cast<const uint16_t*>(bias);
     a.Y = static_cast<uint16_t*>(Y);
-    a.partial = static_cast<float*>(ws);
     a.N = N;
     a.K = K;
     a.g = meta.g;
     a.G = meta.G;
     a.sz_row = meta.sz_row;
-    a.TK = p.TK;
-    a.splits = p.splits;
-    a.row_tiles = p.row_tiles;
-    a.units = p.units;
-    if (!p.tma) {
-        const int blocks = (N * 32 + 255) / 256;
-        switch (M) {
-            case 1: gemv_fwd_simple_kernel<1><<<blocks, 256, 0, st>>>(a, packed); break;
-            case 2: gemv_fwd_simple_kernel<2><<<blocks, 256, 0, st>>>(a, packed); break;
-            case 3: gemv_fwd_simple_kernel<3><<<blocks, 256, 0, st>>>(a, packed); break;
-            case 4: gemv_fwd_simple_kernel<4><<<blocks, 256, 0, st>>>(a, packed); break;
-        }
-        return launch_status();
-    }
-    if (p.ws > ws_bytes || (p.ws > 0 && ws == nullptr)) return W4_ERR_WORKSPACE;
-    if (p.smem > static_cast<size_t>(di.max_smem_optin)) return W4_ERR_UNSUPPORTED;
-    CUtensorMap map;
-    if (!make_map_2d(&map, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, kGemvTileRows,
-                     kGemvBoxWords, 64))
-        return W4_ERR_CUDA;
-    w4_status s = W4_OK;
+    const int blocks = static_cast<int>((static_cast<long long>(N) * 32 + 255) / 256);
     switch (M) {
-        case 1: s = launch_gemv_fwd<1>(p, map, a, st); break;
-        case 2: s = launch_gemv_fwd<2>(p, map, a, st); break;
-        case 3: s = launch_gemv_fwd<3>(p, map, a, st); break;
-        case 4: s = launch_gemv_fwd<4>(p, map, a, st); break;
+        case 1: gemv_fwd_simple_kernel<1><<<blocks, 256, 0, st>>>(a, packed); break;
+        case 2: gemv_fwd_simple_kernel<2><<<blocks, 256, 0, st>>>(a, packed); break;
+        case 3: gemv_fwd_simple_kernel<3><<<blocks, 256, 0, st>>>(a, packed); break;
+        case 4: gemv_fwd_simple_kernel<4><<<blocks, 256, 0, st>>>(a, packed); break;
+        default: return W4_ERR_INVALID_ARG;
     }
-    if (s != W4_OK) return s;
-    if (p.splits > 1) {
-        const long long total = static_cast<long long>(M) * N;
-        const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, di.sms * 8));
-        splits_finalize_kernel<<<blocks, 256, 0, st>>>(a.partial, p.splits, M, N, a.bias, a.Y);
-        return launch_status();
-    }
-    return W4_OK;
+    return launch_status();
 }
 
 w4_status run_gemv_t(const void* A, int M, int N, int K, const uint32_t* packed, const void* S,
