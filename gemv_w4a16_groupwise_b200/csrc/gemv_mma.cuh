@@ -56,67 +56,105 @@ __host__ __device__ inline size_t gemv_mma_xblock_bytes(int M, int TKC) {
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// One warp per (slice, window, m); lane = 16 h + 4 t + tig converts the 8
-// activations k = 128 h + 32 tig + 8 t .. + 7 of the window (zero past K).
-// The grid also clears the GEMV's row-block counters.
+// One warp converts activation row m of window qw (256 k starting at
+// k_first) into `block`, a slice's activation block: lane = 16 h + 4 t + tig
+// converts the 8 activations k_first + 128 h + 32 tig + 8 t .. + 7 (zero past
+// K).  `block` may be global (the prep kernel) or shared memory (the GEMV
+// converting its own slice).
+// The 8 activations of the lane (zero past K).
+__device__ __forceinline__ uint4 xfrag_load(const uint16_t* __restrict__ X, int K, long long k_first, int m,
+                                            int lane) {
+    const int h = lane >> 4, t = (lane >> 2) & 3, tig = lane & 3;
+    const long long k = k_first + h * 128 + 32 * tig + 8 * t;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (k < K) v = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K + k));
+    return v;
+}
+
+// Fixed point, digits and fold constants from the lane's 8 activations v.
+// x' = round(x * 2^(140 - e)) with e the largest bf16 exponent of the lane's
+// half (128 k); the power of two is exact in fp32 unless e < 14 (values
+// below 2^-113), where the integer path below is used instead.  The digits
+// are dh = floor((x' + 128) / 256) and dl = x' - 256 dh, so dl is in
+// [-128, 127] and |dh| <= 64.
+__device__ __forceinline__ void xfrag_store(uint4 v, int M, int nqw, int qw, int m, int lane, uint8_t* block) {
+    const int h = lane >> 4, t = (lane >> 2) & 3, tig = lane & 3;
+    const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+    // largest magnitude: bf16 bit patterns order like their magnitudes
+    uint32_t mx = __vmaxu2(__vmaxu2(r[0] & 0x7FFF7FFFu, r[1] & 0x7FFF7FFFu), __vmaxu2(r[2] & 0x7FFF7FFFu, r[3] & 0x7FFF7FFFu));
+    mx = max(mx & 0xFFFFu, mx >> 16);
+    int emax = max(static_cast<int>(mx >> 7), 1);
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, o));
+    int xf[8];
+    if (emax >= 14) {
+        const float scale = __int_as_float((267 - emax) << 23);   // 2^(140 - emax), exact
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t bits = (j & 1) ? (r[j >> 1] & 0xFFFF0000u) : (r[j >> 1] << 16);
+            xf[j] = __float2int_rn(__uint_as_float(bits) * scale);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t bits = (j & 1) ? (r[j >> 1] >> 16) : (r[j >> 1] & 0xFFFFu);
+            xf[j] = bf16_fixed_bits(bits, emax, kMFrac);
+        }
+    }
+    int sum = 0;
+    uint32_t dh[8], dl[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        sum += xf[j];
+        const int hi = (xf[j] + 128) >> 8;
+        dh[j] = static_cast<uint32_t>(hi);
+        dl[j] = static_cast<uint32_t>(xf[j] - (hi << 8));
+    }
+    // bytes of elements 0,2,4,6 (even k) and 1,3,5,7 (odd k), low byte first
+    auto pack4 = [](uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+        return __byte_perm(__byte_perm(a0, a1, 0x0040), __byte_perm(a2, a3, 0x0040), 0x5410);
+    };
+    const uint32_t hi_e = pack4(dh[0], dh[2], dh[4], dh[6]), hi_o = pack4(dh[1], dh[3], dh[5], dh[7]);
+    const uint32_t lo_e = pack4(dl[0], dl[2], dl[4], dl[6]), lo_o = pack4(dl[1], dl[3], dl[5], dl[7]);
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    uint32_t* frag = reinterpret_cast<uint32_t*>(block);
+    // lane (g = 2 m + p, tig) of mma t: {even h0, even h1, odd h0, odd h1}
+    const size_t rec = (static_cast<size_t>(qw) * 4 + t) * (8 * M) + (2 * m) * 4 + tig;
+    frag[rec * 4 + h] = hi_e;
+    frag[rec * 4 + 2 + h] = hi_o;
+    frag[(rec + 4) * 4 + h] = lo_e;
+    frag[(rec + 4) * 4 + 2 + h] = lo_o;
+    if ((lane & 15) == 0) {
+        float* fs = reinterpret_cast<float*>(block + static_cast<size_t>(nqw) * M * 512);
+        // 2^(emax - 140): a normal float unless emax < 14
+        const float xs_exact = emax >= 14 ? __int_as_float((emax - 13) << 23) : ldexpf(1.0f, emax - 134 - kMFrac);
+        const size_t f0 = (static_cast<size_t>(qw) * 2 * M + 2 * m) * 4 + 2 * h;   // p = 0
+        fs[f0] = 256.0f * xs_exact;
+        fs[f0 + 1] = 0.0f;
+        fs[f0 + 4] = xs_exact;                                                     // p = 1
+        fs[f0 + 5] = xs_exact * static_cast<float>(sum);
+    }
+}
+
+__device__ __forceinline__ void xfrag_convert(const uint16_t* __restrict__ X, int M, int K, long long k_first,
+                                              int nqw, int qw, int m, int lane, uint8_t* block) {
+    xfrag_store(xfrag_load(X, K, k_first, m, lane), M, nqw, qw, m, lane, block);
+}
+
+// Prep kernel for shapes whose conversion is too much to repeat in every
+// CTA: one warp per (slice, window, m).
 __global__ void __launch_bounds__(256) gemv_xfrag_kernel(const uint16_t* __restrict__ X, int M, int K,
-                                                         int TKC, int splits, uint8_t* __restrict__ out,
-                                                         int* __restrict__ counters, int ncounters) {
+                                                         int TKC, int splits, uint8_t* __restrict__ out) {
     pdl_launch_dependents();
-    // the GEMV's per-row-block box counters start from zero on every call
-    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < ncounters;
-         i += static_cast<long long>(gridDim.x) * blockDim.x)
-        counters[i] = 0;
     const int nqw = TKC / 256;
     const long long unit = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     if (unit >= static_cast<long long>(splits) * nqw * M) return;   // whole warps
-    const int lane = threadIdx.x & 31;
     const int m = static_cast<int>(unit % M);
     const long long sq = unit / M;
     const int slice = static_cast<int>(sq / nqw), qw = static_cast<int>(sq - static_cast<long long>(slice) * nqw);
-    const int h = lane >> 4, t = (lane >> 2) & 3, tig = lane & 3;
-    const long long k = static_cast<long long>(slice) * TKC + qw * 256 + h * 128 + 32 * tig + 8 * t;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (k < K) v = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K + k));
-    const uint32_t r[4] = {v.x, v.y, v.z, v.w};
-    int emax = 1;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) emax = max(emax, max(bf16_exp1(r[q] & 0xFFFFu), bf16_exp1(r[q] >> 16)));
-#pragma unroll
-    for (int o = 1; o < 16; o <<= 1) emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, o));
-    uint32_t hi[2] = {0u, 0u}, lo[2] = {0u, 0u};   // [even / odd k] digit bytes
-    int sum = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint32_t bits = (j & 1) ? (r[j >> 1] >> 16) : (r[j >> 1] & 0xFFFFu);
-        const int xf = bf16_fixed_bits(bits, emax, kMFrac);   // |xf| <= 255 * 2^6
-        sum += xf;
-        const int dl = ((xf + 128) & 255) - 128;             // balanced low digit in [-128, 127]
-        const int dh = (xf - dl) >> 8;                        // high digit in [-64, 64]
-        hi[j & 1] |= (static_cast<uint32_t>(dh) & 0xFFu) << (8 * (j >> 1));
-        lo[j & 1] |= (static_cast<uint32_t>(dl) & 0xFFu) << (8 * (j >> 1));
-    }
-#pragma unroll
-    for (int o = 1; o < 16; o <<= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-    const size_t nqw8 = static_cast<size_t>(nqw);
-    uint8_t* block = out + static_cast<size_t>(slice) * gemv_mma_xblock_bytes(M, TKC);
-    uint32_t* frag = reinterpret_cast<uint32_t*>(block);
-    // lane (g = 2 m + p, tig) of mma t: {even h0, even h1, odd h0, odd h1}
-#pragma unroll
-    for (int p = 0; p < 2; ++p) {
-        const size_t rec = (static_cast<size_t>(qw) * 4 + t) * (8 * M) + (2 * m + p) * 4 + tig;
-        frag[rec * 4 + h] = p ? lo[0] : hi[0];
-        frag[rec * 4 + 2 + h] = p ? lo[1] : hi[1];
-    }
-    if ((lane & 15) == 0) {
-        float* fs = reinterpret_cast<float*>(block + nqw8 * M * 512);
-        const float xs = ldexpf(1.0f, emax - 134 - kMFrac);
-        const size_t f0 = (static_cast<size_t>(qw) * 2 * M + 2 * m) * 4 + 2 * h;   // p = 0
-        fs[f0] = 256.0f * xs;
-        fs[f0 + 1] = 0.0f;
-        fs[f0 + 4] = xs;                                                           // p = 1
-        fs[f0 + 5] = xs * static_cast<float>(sum);
-    }
+    xfrag_convert(X, M, K, static_cast<long long>(slice) * TKC + qw * 256, nqw, qw, m, threadIdx.x & 31,
+                  out + static_cast<size_t>(slice) * gemv_mma_xblock_bytes(M, TKC));
 }
 
 // D = A B + C and D = A B (C = 0); the fragments are plain values, so the
@@ -159,6 +197,7 @@ __host__ __device__ inline size_t gemv_mma_smem_bytes(int M, int TKC, int warps,
     size_t b = 1024;
     b += static_cast<size_t>(warps) * stages * gemv_mma_stage_bytes(sz, szw);
     b += static_cast<size_t>(warps) * kSR * 8 * 16;                 // per-box fp32 scale / zero table
+    b += static_cast<size_t>(warps) * 2 * kSR * M * 4;             // shared-row-block slots
     b += gemv_mma_xblock_bytes(M, TKC);
     b += static_cast<size_t>(warps) * stages * 8 + 8 + 16;
     return b;
@@ -166,14 +205,13 @@ __host__ __device__ inline size_t gemv_mma_smem_bytes(int M, int TKC, int warps,
 
 // Arguments of gemv_mma_kernel.
 struct GemvMmaArgs {
-    const uint8_t* xblocks;   // [splits] activation blocks from gemv_xfrag_kernel
+    const uint16_t* X;        // [M, K] bf16 (converted in the kernel when xblocks is null)
+    const uint8_t* xblocks;   // [splits] activation blocks from gemv_xfrag_kernel, or null
     const __half* S;
     const __half* Z;
     const uint16_t* bias;
     uint16_t* Y;
     float* partial;           // [splits, M, N] when splits > 1
-    float* slots;             // [splits, warps of a slice, 2, 4 rows, M] shared row blocks
-    int* counters;            // [splits, row blocks] boxes finished (zeroed by the prep kernel)
     int N, K, g, G, sz_row;
     int TKC;                  // k per slice (a whole number of boxes)
     int splits;               // slices; CTA c works on slice c / cps
@@ -185,14 +223,21 @@ struct GemvMmaArgs {
     long long sz_total;       // halves in each of S and Z (N * sz_row, or 1)
 };
 
-// Work split: the boxes of a slice, row block major (box b = row block
-// b / nbs, k box b % nbs), are cut into one contiguous range per warp of
-// the slice's CTAs, so every warp streams the same number of boxes to
-// within one and no warp waits for another.  A row block that one warp
-// covers completely is written at once; a row block shared by neighbouring
-// warps (at most the first and the last of each range) goes through
-// per-warp partial slots, and the warp that completes its box count sums
-// the slots in warp order, so the result does not depend on timing.
+// Work split: each CTA of a slice takes a contiguous range of whole row
+// blocks (balanced to within one row block), and its warps cut the CTA's
+// boxes, row block major (box b = row block b / nbs, k box b % nbs), into
+// one contiguous range each, equal to within one box; no warp waits for
+// another until the end.  A row block one warp covers completely is written
+// at once.  A row block shared by neighbouring warps goes through per-warp
+// slots in shared memory: after the CTA's single barrier, the warp holding
+// the row block's last box sums the slots in warp order, so the result does
+// not depend on timing.
+//
+// Activations: with `xblocks` null every CTA converts its K slice of X into
+// the fragment layout itself while its first weight boxes are in flight (the
+// planner picks this when the conversion is a few units per warp); else the
+// kernel is a programmatic dependent of gemv_xfrag_kernel and fetches the
+// prepared block with one bulk copy.
 template <int M, int GK, int SZ>
 __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
     gemv_mma_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
@@ -211,7 +256,8 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
     constexpr int kSzTx = SZ == kSzTma2d ? 2 * kSR * 16 * 2 : SZ == kSzTma1d ? 2 * 8 * 2 : 0;
     uint8_t* ring = base;                                                    // [warp][stage][SB]
     float4* table = reinterpret_cast<float4*>(ring + NW * NS * SB);          // [warp][8 windows][4 rows]
-    uint8_t* xblk = reinterpret_cast<uint8_t*>(table + NW * kSR * 8);
+    float* slots = reinterpret_cast<float*>(table + NW * kSR * 8);           // [warp][2][4 rows][M]
+    uint8_t* xblk = reinterpret_cast<uint8_t*>(slots + NW * 2 * kSR * M);
     const uint4* frag = reinterpret_cast<const uint4*>(xblk);                // [qw][t][8M]
     const float4* fsc = reinterpret_cast<const float4*>(xblk + static_cast<size_t>(nqw) * M * 512);  // [qw][2M]
     uint64_t* full = reinterpret_cast<uint64_t*>(xblk + xbytes);
@@ -235,21 +281,18 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
     }
     __syncthreads();
 
-    const int slice = blockIdx.x / a.cps;
-    const int W = a.cps * NW;                                   // warps of this slice
-    const int w = (blockIdx.x - slice * a.cps) * NW + warp;
-    const long long T = static_cast<long long>(a.nrb) * a.nbs;  // boxes of the slice
-    auto wstart = [&](int ww) { return static_cast<int>(static_cast<long long>(ww) * T / W); };
-    // the warp whose range holds box b
-    auto warp_of = [&](int b) {
-        return static_cast<int>((static_cast<long long>(b + 1) * W - 1) / T);
-    };
-    const int b_begin = wstart(w), b_end = wstart(w + 1);
+    const int slice = blockIdx.x / a.cps, cta = blockIdx.x - (blockIdx.x / a.cps) * a.cps;
+    const int rb_lo = static_cast<int>(static_cast<long long>(cta) * a.nrb / a.cps);
+    const int rb_hi = static_cast<int>(static_cast<long long>(cta + 1) * a.nrb / a.cps);
+    const int T = (rb_hi - rb_lo) * a.nbs;                       // boxes of this CTA
+    auto wstart = [&](int ww) { return static_cast<int>(static_cast<long long>(ww) * T / NW); };
+    auto warp_of = [&](int b) { return static_cast<int>((static_cast<long long>(b + 1) * NW - 1) / T); };
+    const int b_begin = wstart(warp), b_end = wstart(warp + 1);
     int gshift = 0;
     if (GK == kGroupsPow2) gshift = __ffs(a.g) - 1;
 
     struct Cur {
-        int b, rb, kb;
+        int b, rb, kb;   // CTA-local box, its row block (absolute) and k box
     };
     auto advance = [&](Cur& c) {
         ++c.b;
@@ -258,7 +301,7 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
             ++c.rb;
         }
     };
-    const Cur start{b_begin, b_begin / a.nbs, b_begin - (b_begin / a.nbs) * a.nbs};
+    const Cur start{b_begin, rb_lo + b_begin / a.nbs, b_begin - (b_begin / a.nbs) * a.nbs};
     auto box_k0 = [&](const Cur& c) { return slice * a.TKC + c.kb * kSBK; };
     auto box_row0 = [&](const Cur& c) { return c.rb * kSR; };
     auto first_group = [&](int k0) {
@@ -304,16 +347,39 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
             advance(ic);
         }
     };
-    // one stage of weights first; then, once the prep kernel is done, the
-    // activation block (so that it does not queue behind the whole ring);
-    // then the rest of the ring
-    issue();
-    pdl_wait();
-    if (tid == 0 && b_begin < wstart(NW * (blockIdx.x - slice * a.cps + 1))) {
-        mbar_arrive_expect_tx(xbar, xbytes);
-        bulk_load_1d(xblk, a.xblocks + static_cast<size_t>(slice) * xbytes, xbytes, xbar);
+    if (a.xblocks == nullptr) {
+        // this warp's activation units (at most 4: the planner's limit) are
+        // loaded first, the ring is filled while they are in flight, and
+        // the conversion runs while the first boxes are in flight
+        constexpr int kMaxUnits = 4;
+        const long long k_slice = static_cast<long long>(slice) * a.TKC;
+        uint4 raw[kMaxUnits];
+#pragma unroll
+        for (int i = 0; i < kMaxUnits; ++i) {
+            const int u = warp + i * NW;
+            raw[i] = make_uint4(0u, 0u, 0u, 0u);
+            if (u < nqw * M) raw[i] = xfrag_load(a.X, a.K, k_slice + (u / M) * 256, u - (u / M) * M, lane);
+        }
+        for (int b = 0; b < NS; ++b) issue();
+#pragma unroll
+        for (int i = 0; i < kMaxUnits; ++i) {
+            const int u = warp + i * NW;
+            if (u < nqw * M) xfrag_store(raw[i], M, nqw, u / M, u - (u / M) * M, lane, xblk);
+        }
+        __syncthreads();
+    } else {
+        // one stage of weights first; then, once the prep kernel is done,
+        // the activation block (so that it does not queue behind the whole
+        // ring); then the rest of the ring
+        issue();
+        pdl_wait();
+        if (tid == 0 && T > 0) {
+            mbar_arrive_expect_tx(xbar, xbytes);
+            bulk_load_1d(xblk, a.xblocks + static_cast<size_t>(slice) * xbytes, xbytes, xbar);
+        }
+        for (int b = 1; b < NS; ++b) issue();
+        if (T > 0) mbar_wait_bounded(xbar, 0, abort_flag, kErrTimeoutTmaFull);
     }
-    for (int b = 1; b < NS; ++b) issue();
 
     const int wrow = g >> 1, wchunk = (g & 1) * 4 + tig;   // the B chunk this lane loads
     const bool f_lane = g < 2 * M;
@@ -330,10 +396,9 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
     }
     float4* wtable = table + warp * kSR * 8;
     const int tq = lane & 7, ti = lane >> 3;               // table entry this lane builds
-    if (b_begin < b_end) mbar_wait_bounded(xbar, 0, abort_flag, kErrTimeoutTmaFull);
 
-    // the outputs of row block rb: lanes with even g < 2M hold (m = g / 2,
-    // row tig) after the digit shuffle
+    // outputs: after the digit shuffle, lanes with even g < 2M hold
+    // (m = g / 2, row tig) of the row block
     auto store = [&](int m, int n, float v) {
         if (a.splits == 1) {
             if (a.bias) v += bf16_bits_to_float(a.bias[n]);
@@ -345,33 +410,13 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
     const int first_rb = start.rb;
     auto finish = [&](int rb, int nb, float y) {
         const float v = y + __shfl_xor_sync(0xFFFFFFFFu, y, 4);
-        const bool out_lane = !(g & 1) && f_lane;
-        if (nb == a.nbs) {
-            const int n = rb * kSR + tig;
-            if (out_lane && n < a.N) store(g >> 1, n, v);
-            return;
-        }
-        float* sl = a.slots + ((static_cast<size_t>(slice) * W + w) * 2 + (rb == first_rb ? 0 : 1)) * (kSR * M);
-        if (out_lane) sl[tig * M + (g >> 1)] = v;
-        __threadfence();
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) last = (atomicAdd(&a.counters[slice * a.nrb + rb], nb) + nb == a.nbs);
-        last = __shfl_sync(0xFFFFFFFFu, last, 0);
-        if (!last) return;
-        __threadfence();
-        const int w0 = warp_of(rb * a.nbs), w1 = warp_of(rb * a.nbs + a.nbs - 1);
-        if (lane < kSR * M) {
-            const int r = lane / M, m = lane - (lane / M) * M;
-            float s = 0.0f;
-            for (int ww = w0; ww <= w1; ++ww) {
-                const int ws = wstart(ww);
-                if (ws == wstart(ww + 1)) continue;
-                const int sslot = (ws / a.nbs == rb) ? 0 : 1;
-                s += __ldcg(a.slots + ((static_cast<size_t>(slice) * W + ww) * 2 + sslot) * (kSR * M) + r * M + m);
+        if (!(g & 1) && f_lane) {
+            if (nb == a.nbs) {
+                const int n = rb * kSR + tig;
+                if (n < a.N) store(g >> 1, n, v);
+            } else {
+                slots[((warp * 2) + (rb == first_rb ? 0 : 1)) * (kSR * M) + tig * M + (g >> 1)] = v;
             }
-            const int n = rb * kSR + r;
-            if (n < a.N) store(m, n, s);
         }
     };
 
@@ -457,6 +502,32 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
             finish(rb, nb_rb, y);
             y = 0.0f;
             nb_rb = 0;
+        }
+    }
+
+    // row blocks shared by neighbouring warps: the warp with a shared row
+    // block's last box adds the slots of all its contributors in warp order
+    __syncthreads();
+    if (b_begin < b_end) {
+        const int last_rb = rb_lo + (b_end - 1) / a.nbs;
+        for (int side = 0; side < 2; ++side) {
+            const int rb = side ? last_rb : first_rb;
+            if (side && rb == first_rb) break;
+            const int lb0 = (rb - rb_lo) * a.nbs, lb1 = lb0 + a.nbs - 1;   // CTA-local boxes of rb
+            const bool partial = b_begin > lb0 || b_end - 1 < lb1;
+            if (!partial || warp_of(lb1) != warp) continue;
+            if (lane < kSR * M) {
+                const int r = lane / M, m = lane - (lane / M) * M;
+                float s = 0.0f;
+                for (int ww = warp_of(lb0); ww <= warp; ++ww) {
+                    const int ws = wstart(ww);
+                    if (ws == wstart(ww + 1)) continue;
+                    const int sslot = (rb_lo + ws / a.nbs == rb) ? 0 : 1;
+                    s += slots[(ww * 2 + sslot) * (kSR * M) + r * M + m];
+                }
+                const int n = rb * kSR + r;
+                if (n < a.N) store(m, n, s);
+            }
         }
     }
     if (*abort_flag) {

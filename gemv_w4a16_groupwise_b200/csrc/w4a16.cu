@@ -204,8 +204,8 @@ struct StreamPlan {
     int TKC = 0, splits = 1, nbs = 0, KP = 1, RBP = kSW, rounds = 0, units = 0, grid = 0, stages = 2;
     int szw = 0, warps = kSW, sz = 0;
     int nrb = 0, cps = 0;                      // tensor-pipe kernel: row blocks, CTAs per slice
-    bool mma = false;
-    size_t smem = 0, xbytes = 0, ws = 0, partial_off = 0, slots_off = 0, cnt_off = 0;
+    bool mma = false, in_kernel_x = false;
+    size_t smem = 0, xbytes = 0, ws = 0, partial_off = 0;
 };
 
 // szw: scale / zero words per stage row (gemv_stream_sz_words of the group
@@ -300,18 +300,17 @@ StreamPlan plan_mma(int M, int N, int K, int sz, int szw, const DeviceInfo& di) 
     p.nbs = (nb_total + p.splits - 1) / p.splits;
     p.TKC = p.nbs * kSBK;
     p.nrb = (N + kSR - 1) / kSR;
-    // CTAs per slice: all the SMs, unless the slice has fewer boxes than warps
-    const long long boxes = static_cast<long long>(p.nrb) * p.nbs;
-    p.cps = static_cast<int>(std::max<long long>(
-        1, std::min<long long>(di.sms / p.splits, (boxes + p.warps - 1) / p.warps)));
+    // CTAs per slice: all the SMs, but at least one row block each
+    p.cps = std::max(1, std::min(di.sms / p.splits, p.nrb));
     p.grid = p.splits * p.cps;
     p.smem = gemv_mma_smem_bytes(M, p.TKC, p.warps, p.stages, sz, szw);
     p.xbytes = gemv_mma_xblock_bytes(M, p.TKC);
+    // every CTA converts its own activations when that is at most a few
+    // warp-units (256 k of one row) per warp; else a prep kernel does it once
+    p.in_kernel_x = p.splits == 1 && (p.TKC / 256) * M <= 4 * p.warps;
     auto up = [](size_t v) { return (v + 255) / 256 * 256; };
-    p.partial_off = up(p.splits * p.xbytes);
-    p.slots_off = p.partial_off + up(p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * sizeof(float) : 0);
-    p.cnt_off = p.slots_off + up(static_cast<size_t>(p.splits) * p.cps * p.warps * 2 * kSR * M * sizeof(float));
-    p.ws = p.cnt_off + up(static_cast<size_t>(p.splits) * p.nrb * sizeof(int));
+    p.partial_off = p.in_kernel_x ? 0 : up(p.splits * p.xbytes);
+    p.ws = p.partial_off + (p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * sizeof(float) : 0);
     p.mma = true;
     p.ok = true;
     return p;
@@ -365,6 +364,10 @@ w4_status launch_gemv_stream(const StreamPlan& p, const CUtensorMap& map, const 
 
 // The GEMV is launched as a programmatic dependent of the prep kernel just
 // before it: its prologue and first weight loads overlap the prep kernel.
+// With a prep kernel just before it, the GEMV is launched as its
+// programmatic dependent: its prologue and first weight loads overlap the
+// prep kernel.  Without one it is an ordinary launch (it reads its inputs
+// from the start, so it must not begin before the work ahead of it ends).
 template <int M, int GK, int SZ>
 w4_status launch_gemv_mma_k(const StreamPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
                             const CUtensorMap& zm, const GemvMmaArgs& a, cudaStream_t st) {
@@ -379,7 +382,7 @@ w4_status launch_gemv_mma_k(const StreamPlan& p, const CUtensorMap& wm, const CU
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = p.in_kernel_x ? 0 : 1;
     cudaLaunchKernelEx(&cfg, fn, wm, sm, zm, a);
     return launch_status();
 }
@@ -428,8 +431,8 @@ w4_status launch_gemv_mma(const StreamPlan& p, int M, const CUtensorMap& wm, con
 w4_status run_gemv_stream(const StreamPlan& p, int M, int N, int K, const void* A, const uint32_t* packed,
                           const void* S, const void* Z, const Meta& meta, const void* bias, void* Y,
                           void* ws, size_t ws_bytes, cudaStream_t st) {
-    if (p.ws > ws_bytes || ws == nullptr) return W4_ERR_WORKSPACE;
-    if (!aligned16(ws)) return W4_ERR_ALIGNMENT;
+    if (p.ws > ws_bytes || (p.ws > 0 && ws == nullptr)) return W4_ERR_WORKSPACE;
+    if (ws && !aligned16(ws)) return W4_ERR_ALIGNMENT;
     uint8_t* xb = static_cast<uint8_t*>(ws);
     float* partial = p.splits > 1 ? reinterpret_cast<float*>(xb + p.partial_off) : nullptr;
     CUtensorMap map;
@@ -437,22 +440,21 @@ w4_status run_gemv_stream(const StreamPlan& p, int M, int N, int K, const void* 
         return W4_ERR_CUDA;
     w4_status s = W4_OK;
     if (p.mma) {
-        int* counters = reinterpret_cast<int*>(xb + p.cnt_off);
-        const int ncounters = p.splits * p.nrb;
-        const long long lanes = static_cast<long long>(p.splits) * (p.TKC / 256) * M * 32;
-        gemv_xfrag_kernel<<<static_cast<int>((lanes + 255) / 256), 256, 0, st>>>(
-            static_cast<const uint16_t*>(A), M, K, p.TKC, p.splits, xb, counters, ncounters);
-        s = launch_status();
-        if (s != W4_OK) return s;
+        if (!p.in_kernel_x) {
+            const long long lanes = static_cast<long long>(p.splits) * (p.TKC / 256) * M * 32;
+            gemv_xfrag_kernel<<<static_cast<int>((lanes + 255) / 256), 256, 0, st>>>(
+                static_cast<const uint16_t*>(A), M, K, p.TKC, p.splits, xb);
+            s = launch_status();
+            if (s != W4_OK) return s;
+        }
         GemvMmaArgs a;
-        a.xblocks = xb;
+        a.X = static_cast<const uint16_t*>(A);
+        a.xblocks = p.in_kernel_x ? nullptr : xb;
         a.S = static_cast<const __half*>(S);
         a.Z = static_cast<const __half*>(Z);
         a.bias = static_cast<const uint16_t*>(bias);
         a.Y = static_cast<uint16_t*>(Y);
         a.partial = partial;
-        a.slots = reinterpret_cast<float*>(xb + p.slots_off);
-        a.counters = counters;
         a.N = N;
         a.K = K;
         a.g = meta.g;
