@@ -11,11 +11,14 @@
 // added to the fp32 accumulator before the single bf16 rounding (vLLM
 // "Adding bias epilogue support for cutlass_scaled_mm").
 //
-// Warp roles (320 threads, one CTA per SM):
-//   warp 0      TMA producer: packed weight tile + activation tile per stage
-//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma and commits
-//   warps 2..9  dequantize packed codes into the bf16 A tile of the stage
-//               (128-byte swizzled UMMA layout), then run the epilogue
+// Warp roles (576 threads, one CTA per SM):
+//   warp 0       TMA producer: packed weight tile + activation tile per stage
+//   warp 1       TMEM allocator; lane 0 issues tcgen05.mma and commits
+//   warps 2..17  dequantize packed codes into the bf16 A tile of a stage
+//                (128-byte swizzled UMMA layout), then run the epilogue.
+//                Two groups of 8 warps take alternate stages, so two stages
+//                are being dequantized at any time and the tensor pipe is not
+//                left waiting on one stage's dequantization latency.
 // Every mbarrier wait is bounded; a wait that runs out records the reason in
 // the device error word and the CTA unwinds without hanging.
 //
@@ -31,7 +34,8 @@
 
 namespace w4 {
 
-constexpr int kTcThreads = 320;
+constexpr int kTcDeqGroups = 2;                      // dequantizing warp groups (8 warps each)
+constexpr int kTcThreads = 64 + kTcDeqGroups * 256;
 constexpr int kTcBM = 128;     // MMA M (weight rows per tile)
 constexpr int kTcBK = 64;      // reduction depth per pipeline stage
 constexpr int kTcABytes = kTcBM * kTcBK * 2;   // 16 KB dequantized tile
@@ -240,60 +244,109 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else {
         // ------------------------------------------------ dequantize
-        const int t = threadIdx.x - 64;  // 0 .. 255
+        const int grp_id = (threadIdx.x - 64) >> 8;           // this warp's group: stages kb = grp_id mod 2
+        const int t = (threadIdx.x - 64) & 255;               // 0 .. 255 within the group
         // forward: row n = r0 + t % 128, words 4h .. 4h+3 of the 8 in a k-block
         // transposed: row n = kb * 64 + t % 64, words 4q .. 4q+3 of the 16 of a k-tile
         const int prow = TR ? (t & 63) : (t & 127);
         const int pquad = TR ? (t >> 6) : (t >> 7);
         const int W8 = a.K / 8;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        // swizzled 16-byte destinations of this thread's 4 words in the A tile
+        uint32_t off[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (TR) {
+                const int kk = 32 * pquad + 8 * j;        // k within the 128-wide tile
+                const int atom = kk >> 6, c = (kk & 63) >> 3;
+                off[j] = atom * 8192 + (prow >> 3) * 1024 + (prow & 7) * 128 + ((c ^ (prow & 7)) << 4);
+            } else {
+                const int c = 4 * pquad + j;               // 16-byte chunk within the row
+                off[j] = prow * 128 + ((c ^ (prow & 7)) << 4);
+            }
+        }
+        // Scale / zero of block kb, fetched one block ahead.  With g a
+        // multiple of 32 the thread's 4 words share one group: forward, the
+        // group moves by at most 64 / g per block and is tracked by
+        // subtraction; transposed, it is fixed and only the row moves.
+        constexpr int NG = PWG ? 4 : 1;
+        const int kw_t = TR ? r0 / 8 + 4 * pquad : 4 * pquad;   // forward: + kb * 8
+        int grp_f = 0, rem_f = 0;                               // forward: (8 kw0) = grp_f * g + rem_f
+        if (!PWG && !TR) {
+            grp_f = (8 * kw_t) / a.g;
+            rem_f = 8 * kw_t - grp_f * a.g;
+        }
+        const int grp_t = (!PWG && TR) ? min((8 * kw_t) / a.g, a.G - 1) : 0;
+        auto load_sz = [&](int kb, float (&sv)[NG], float (&zv)[NG]) {
+            const int n = TR ? kb * kTcBK + prow : r0 + prow;
+            const int nc = min(n, a.N - 1);
+            const __half* sp = a.S + static_cast<size_t>(nc) * a.sz_row;
+            const __half* zp = a.Z + static_cast<size_t>(nc) * a.sz_row;
+            if (PWG) {
+                const int kw0 = TR ? kw_t : kb * (kTcBK / 8) + kw_t;
+#pragma unroll
+                for (int j = 0; j < NG; ++j) {
+                    const int grp = min((8 * (kw0 + j)) / a.g, a.G - 1);
+                    sv[j] = __half2float(__ldg(sp + grp));
+                    zv[j] = __half2float(__ldg(zp + grp));
+                }
+            } else {
+                const int grp = TR ? grp_t : min(grp_f, a.G - 1);
+                sv[0] = __half2float(__ldg(sp + grp));
+                zv[0] = __half2float(__ldg(zp + grp));
+            }
+        };
+        auto next_group = [&]() {   // forward, g a multiple of 32: advance this group's stride of k-blocks
+            if (!PWG && !TR) {
+                rem_f += kTcBK * kTcDeqGroups;
+                while (rem_f >= a.g) {
+                    rem_f -= a.g;
+                    ++grp_f;
+                }
+            }
+        };
+        if (!PWG && !TR) {   // start at this group's first block
+            rem_f += kTcBK * grp_id;
+            while (rem_f >= a.g) {
+                rem_f -= a.g;
+                ++grp_f;
+            }
+        }
+        float sv[NG], zv[NG], svn[NG], zvn[NG];
+        if (grp_id < num_kb) load_sz(grp_id, sv, zv);
+        next_group();
+        for (int kb = grp_id; kb < num_kb; kb += kTcDeqGroups) {
             const int s = kb % NS;
             const uint32_t par = static_cast<uint32_t>(kb / NS) & 1u;
-            int n, kw0;  // weight row and first packed word (global) of this thread
-            if (TR) {
-                n = kb * kTcBK + prow;
-                kw0 = r0 / 8 + 4 * pquad;
-            } else {
-                n = r0 + prow;
-                kw0 = kb * (kTcBK / 8) + 4 * pquad;
-            }
+            if (kb + kTcDeqGroups < num_kb) load_sz(kb + kTcDeqGroups, svn, zvn);
+            next_group();
+            const int n = TR ? kb * kTcBK + prow : r0 + prow;
+            const int kw0 = TR ? kw_t : kb * (kTcBK / 8) + kw_t;
             const bool row_ok = n < a.N;
-            const int nc = row_ok ? n : a.N - 1;
-            float sv[PWG ? 4 : 1], zv[PWG ? 4 : 1];
-#pragma unroll
-            for (int j = 0; j < (PWG ? 4 : 1); ++j) {
-                const int grp = min((8 * (kw0 + j)) / a.g, a.G - 1);
-                sv[j] = __half2float(__ldg(a.S + nc * a.sz_row + grp));
-                zv[j] = __half2float(__ldg(a.Z + nc * a.sz_row + grp));
-            }
             const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&tma_full[s], par, abort_flag,
                                                                       kErrTimeoutTmaFull));
-            if (!ok) continue;
-            uint8_t* st = base + s * kStageBytes;
-            const uint8_t* pk = st + kTcABytes + BN * 128;
-            const uint4 wv = TR ? *reinterpret_cast<const uint4*>(pk + prow * 64 + pquad * 16)
-                                : *reinterpret_cast<const uint4*>(pk + prow * 32 + pquad * 16);
+            if (ok) {
+                uint8_t* st = base + s * kStageBytes;
+                const uint8_t* pk = st + kTcABytes + BN * 128;
+                const uint4 wv = TR ? *reinterpret_cast<const uint4*>(pk + prow * 64 + pquad * 16)
+                                    : *reinterpret_cast<const uint4*>(pk + prow * 32 + pquad * 16);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t w = (j == 0) ? wv.x : (j == 1) ? wv.y : (j == 2) ? wv.z : wv.w;
-                const float sj = sv[PWG ? j : 0], zj = zv[PWG ? j : 0];
-                uint4 out = make_uint4(0u, 0u, 0u, 0u);
-                if (row_ok && (kw0 + j) < W8)
-                    out = dequant_word_bf16(w, sj, -(128.0f + zj) * sj, -(2048.0f + zj) * sj);
-                uint32_t off;
-                if (TR) {
-                    const int kk = 32 * pquad + 8 * j;        // k within the 128-wide tile
-                    const int atom = kk >> 6, c = (kk & 63) >> 3;
-                    off = atom * 8192 + (prow >> 3) * 1024 + (prow & 7) * 128 + ((c ^ (prow & 7)) << 4);
-                } else {
-                    const int c = 4 * pquad + j;               // 16-byte chunk within the row
-                    off = prow * 128 + ((c ^ (prow & 7)) << 4);
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t w = (j == 0) ? wv.x : (j == 1) ? wv.y : (j == 2) ? wv.z : wv.w;
+                    const float sj = sv[PWG ? j : 0], zj = zv[PWG ? j : 0];
+                    uint4 out = make_uint4(0u, 0u, 0u, 0u);
+                    if (row_ok && (kw0 + j) < W8)
+                        out = dequant_word_bf16(w, sj, -(128.0f + zj) * sj, -(2048.0f + zj) * sj);
+                    *reinterpret_cast<uint4*>(st + off[j]) = out;
                 }
-                *reinterpret_cast<uint4*>(st + off) = out;
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&deq_full[s]);
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&deq_full[s]);
+#pragma unroll
+            for (int j = 0; j < NG; ++j) {
+                sv[j] = svn[j];
+                zv[j] = zvn[j];
+            }
         }
 
         // ------------------------------------------------ epilogue
@@ -301,13 +354,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                                                   kErrTimeoutAccum));
         if (ok && !*abort_flag) {
             tc_fence_after();
+            // warp w reads TMEM lanes 32 (w % 4) .. + 31; the 16 epilogue
+            // warps split the BN columns into up to 4 parts of >= 8
             const int q = warp & 3;
-            const int half = (warp - 2) >> 2;
+            constexpr int kParts = BN / 8 < 4 ? BN / 8 : 4;
+            const int part = (warp - 2) >> 2;
             const int row = r0 + 32 * q + lane;
             const bool rv = row < L_out;
             const float bias_f = (a.bias && rv) ? bf16_bits_to_float(a.bias[row]) : 0.0f;
 #pragma unroll 1
-            for (int c0 = half * (BN / 2); c0 < (half + 1) * (BN / 2); c0 += 8) {
+            for (int c0 = part * (BN / kParts); part < kParts && c0 < (part + 1) * (BN / kParts); c0 += 8) {
                 uint32_t r[8];
                 tmem_ld_x8(tmem_d + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0), r);
 #pragma unroll

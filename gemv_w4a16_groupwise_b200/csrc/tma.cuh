@@ -43,14 +43,26 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// Test the phase; while it is incomplete the thread may be suspended in
+// hardware for up to `suspend_ns` (it resumes as soon as the phase
+// completes), so waiting threads do not take issue slots from working ones.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, uint32_t suspend_ns = 0) {
     uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
+    if (suspend_ns == 0) {
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+            " selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+            " selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+            : "memory");
+    }
     return ok != 0;
 }
 
@@ -61,15 +73,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
                                                   volatile int* abort, unsigned int err) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long start = global_timer_ns();
-    for (uint32_t spin = 1;; ++spin) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((spin & 255u) == 0) {
-            if (*abort) return false;
-            if (global_timer_ns() - start > kWaitTimeoutNs) {
-                record_error(err);
-                *abort = 1;
-                return false;
-            }
+    for (;;) {
+        // suspended for at most 20 us per test, so the abort flag and the
+        // time limit are still checked often
+        if (mbar_try_wait(bar, parity, 20000u)) return true;
+        if (*abort) return false;
+        if (global_timer_ns() - start > kWaitTimeoutNs) {
+            record_error(err);
+            *abort = 1;
+            return false;
         }
     }
 }
