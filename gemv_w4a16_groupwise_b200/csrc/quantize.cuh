@@ -19,7 +19,9 @@ namespace w4 {
 struct GroupParams {
     __half s;
     float sf;   // float(s)
+    float rs;   // 1 / sf, correctly rounded
     int z;
+    float zf;   // float(z)
 };
 
 __device__ __forceinline__ GroupParams group_params_from_range(float mn, float mx) {
@@ -29,15 +31,33 @@ __device__ __forceinline__ GroupParams group_params_from_range(float mn, float m
     if (__half2float(s) == 0.0f) s = __float2half_rn(fmaxf(fabsf(mn), 0x1p-14f));
     p.s = s;
     p.sf = __half2float(s);
+    p.rs = __frcp_rn(p.sf);
     const float zf = fminf(fmaxf(rintf(__fdiv_rn(-mn, p.sf)), 0.0f), 15.0f);
     p.z = static_cast<int>(zf);
+    p.zf = static_cast<float>(p.z);
     return p;
 }
 
+// rint(w / s) as IEEE fp32 division followed by rint gives it, without the
+// division for all but near-tie quotients.  t = w * (1/s) is within about
+// 2^-23 relative of w / s, and so is the correctly rounded quotient.  The
+// exact integer only matters while the code is not clamped, i.e. for
+// |t| <= 15 + 15 (z <= 15); there both lie within 2^-18 of w / s, so when t
+// is farther than 2^-11 from every half-integer they round to the same
+// integer.  For larger |t| the clamp gives 0 or 15 either way.  Otherwise
+// (and for NaN or infinity) the division is done exactly.
+__device__ __forceinline__ float rint_quotient(float w, const GroupParams& p) {
+    const float t = w * p.rs;
+    const float k = rintf(t);
+    if (fabsf(t - k) < 0.5f - 0x1p-11f) return k;
+    return rintf(__fdiv_rn(w, p.sf));
+}
+
 __device__ __forceinline__ uint32_t quantize_code(float w, const GroupParams& p) {
-    float t = __fadd_rn(rintf(__fdiv_rn(w, p.sf)), static_cast<float>(p.z));
+    float t = __fadd_rn(rint_quotient(w, p), p.zf);
     t = fminf(fmaxf(t, 0.0f), 15.0f);
-    return static_cast<uint32_t>(static_cast<int>(t));
+    // t is an integer in [0, 15]: adding 2^23 leaves it in the low mantissa bits
+    return __float_as_uint(__fadd_rn(t, 8388608.0f)) & 0xFu;
 }
 
 __device__ __forceinline__ void unpack8_bf16(const uint4 raw, float (&v)[8]) {
@@ -56,25 +76,29 @@ __device__ __forceinline__ uint32_t pack8(const float (&v)[8], const GroupParams
     return word;
 }
 
-// Groups of g = 8 * LPG elements, LPG a power of two <= 32: each thread owns
-// one 16-byte chunk (8 values, one packed word); the LPG lanes of a group
-// reduce min / max with shuffles inside their aligned lane segment.
-template <int LPG>
+// Groups of g = 8 * WPT * LPG elements, LPG a power of two <= 32: each
+// thread owns WPT consecutive 16-byte chunks (8 values, one packed word
+// each) of one group; the LPG lanes of a group reduce min / max with
+// shuffles inside their aligned lane segment.
+template <int LPG, int WPT>
 __global__ void __launch_bounds__(256) quantize_segmented_kernel(
     const uint16_t* __restrict__ W, long long total_words, uint32_t* __restrict__ packed,
     __half* __restrict__ scales, __half* __restrict__ zeros) {
     const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const bool active = t < total_words;
-    const long long tw = active ? t : (total_words - 1);
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(W) + tw);
-    float v[8];
-    unpack8_bf16(raw, v);
-    float mn = v[0], mx = v[0];
+    const long long w0 = t * WPT;                      // first word of the thread
+    const bool active = w0 < total_words;
+    const long long tw = active ? w0 : (total_words - WPT);
+    float v[WPT][8];
 #pragma unroll
-    for (int i = 1; i < 8; ++i) {
-        mn = fminf(mn, v[i]);
-        mx = fmaxf(mx, v[i]);
-    }
+    for (int j = 0; j < WPT; ++j) unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(W) + tw + j), v[j]);
+    float mn = v[0][0], mx = v[0][0];
+#pragma unroll
+    for (int j = 0; j < WPT; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            mn = fminf(mn, v[j][i]);
+            mx = fmaxf(mx, v[j][i]);
+        }
 #pragma unroll
     for (int off = 1; off < LPG; off <<= 1) {
         mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
@@ -82,7 +106,12 @@ __global__ void __launch_bounds__(256) quantize_segmented_kernel(
     }
     const GroupParams p = group_params_from_range(mn, mx);
     if (!active) return;
-    packed[t] = pack8(v, p);
+    if (WPT == 2) {
+        *reinterpret_cast<uint2*>(packed + w0) = make_uint2(pack8(v[0], p), pack8(v[1], p));
+    } else {
+#pragma unroll
+        for (int j = 0; j < WPT; ++j) packed[w0 + j] = pack8(v[j], p);
+    }
     if ((threadIdx.x & (LPG - 1)) == 0) {
         const long long grp = t / LPG;
         scales[grp] = p.s;

@@ -902,15 +902,19 @@ w4_status w4_quantize_pack(const void* W, int N, int K, int mode, int group_size
         global_quantize_kernel<<<qblocks, 256, 0, st>>>(w, total_words, part, blocks, packed, sc, ze);
         return launch_status();
     }
+    // words per group: two words per thread (one for g = 8), lanes of a group
+    // reduce with shuffles up to a warp; longer groups take a warp each
     const int lpg = meta.g / 8;
-    const int blocks = static_cast<int>((total_words + 255) / 256);
+    const int wpt = lpg >= 2 ? 2 : 1;
+    const int blocks = static_cast<int>((total_words / wpt + 255) / 256);
     switch (lpg) {
-        case 1: quantize_segmented_kernel<1><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
-        case 2: quantize_segmented_kernel<2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
-        case 4: quantize_segmented_kernel<4><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
-        case 8: quantize_segmented_kernel<8><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
-        case 16: quantize_segmented_kernel<16><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
-        case 32: quantize_segmented_kernel<32><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        case 1: quantize_segmented_kernel<1, 1><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        case 2: quantize_segmented_kernel<1, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        case 4: quantize_segmented_kernel<2, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        case 8: quantize_segmented_kernel<4, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        case 16: quantize_segmented_kernel<8, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        case 32: quantize_segmented_kernel<16, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        case 64: quantize_segmented_kernel<32, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
         default: {
             const long long groups = total_words / lpg;
             const int gblocks = static_cast<int>((groups + 7) / 8);
