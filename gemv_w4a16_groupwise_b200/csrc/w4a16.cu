@@ -408,8 +408,6 @@ w4_status launch_gemv_stream(const StreamPlan& p, const CUtensorMap& map, const 
     return launch_gemv_stream_gk<M, kGroupsAny>(p, map, a, st);
 }
 
-// The GEMV is launched as a programmatic dependent of the prep kernel just
-// before it: its prologue and first weight loads overlap the prep kernel.
 // With a prep kernel just before it, the GEMV is launched as its
 // programmatic dependent: its prologue and first weight loads overlap the
 // prep kernel.  Without one it is an ordinary launch (it reads its inputs
