@@ -27,6 +27,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -100,12 +101,16 @@ def case_bytes(M, N, K, groups_per_row, out_len=None):
 
 
 def source_hash():
+    """Hash of the CUDA sources with comments and blank lines removed, so a
+    comment edit does not mark committed counters as stale."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gemv_w4a16_groupwise_b200", "csrc")
     for fn in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, fn), "rb") as f:
-            h.update(fn.encode())
-            h.update(f.read())
+        with open(os.path.join(csrc, fn)) as f:
+            text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+        lines = [re.sub(r"//.*", "", l).rstrip() for l in text.splitlines()]
+        h.update(fn.encode())
+        h.update("\n".join(l for l in lines if l.strip()).encode())
     return h.hexdigest()[:16]
 
 
