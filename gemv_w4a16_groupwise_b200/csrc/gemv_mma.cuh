@@ -1,38 +1,39 @@
 // Forward GEMV for M <= 4 whose integer dot products run on the tensor
-// pipe (mma.sync m16n8k32, s8 x u8 -> s32), for group lengths that are a
+// pipe (mma.sync m16n8k32, u8 x s8 -> s32), for group lengths that are a
 // multiple of 128 (or one group per row).
 //
-// Streaming is the same as in gemv_stream_kernel: each warp walks 4
-// consecutive weight rows along K in 4 rows x 1 KB TMA boxes, with the
-// box's scales and zeros copied into the same stage by cp.async.  What
-// changes is the arithmetic, which on CUDA cores costs 4 dp4a per packed
-// word and activation row; here one mma covers 4 weight rows x 64 k for
-// every M <= 4:
+// Stream.  A producer warp walks the CTA's 16-row blocks along K and brings
+// each 16 rows x 2048 k piece (16 rows x 1 KB of packed words, one TMA box)
+// and its scales and zeros into a CTA-wide ring of stages.  Sixteen consumer
+// warps share every stage: warp w takes granule w (k = 128 w .. 128 w + 127
+// of the stage) of all 16 rows.  Row segments of 1 KB keep DRAM pages busy,
+// and the per-stage bookkeeping is paid once per 16 KB, not once per warp.
 //
-//   B (32 x 8, u8)  column n = (weight row i = n / 2, half h = n % 2): the
-//                   4-bit codes themselves, one byte each, the even and odd
-//                   nibbles of one packed word per lane;
-//   A (16 x 32, s8) row r = (half h = r / 8, activation row m, digit p):
-//                   X in 16-bit fixed point per 128-k granule, split into a
-//                   high and a low signed byte (balanced digits, so both
-//                   fit s8);
-//   D (16 x 8, s32) entries with equal halves in A and B are exact integer
-//                   dot products; the two other entries are not used.
+// Arithmetic.  One mma multiplies 16 weight rows by 32 k:
+//   A (16 x 32, u8)  the 4-bit codes, one per byte: A row r is weight row r
+//                    of the stage.  Lane (g, tig) holds four consecutive
+//                    packed words of rows g and g + 8 (words 4 tig .. 4 tig + 3
+//                    of the granule).  The even codes of a word are
+//                    w & 0x0F0F0F0F, the odd ones w & 0xF0F0F0F0 (16 q, still
+//                    a byte), so four mma cover the granule: the even and the
+//                    odd codes of words {0, 1} and of words {2, 3}.
+//   B (32 x 8, s8)   the activations in 16-bit fixed point per 128-k granule
+//                    (scaled by the granule's largest bf16 exponent), split
+//                    into a high and a low signed digit: column 2 m + p is
+//                    digit p of activation row m, so one mma serves any M <= 4.
+//   D (16 x 8, s32)  exact sums over the granule: lane (g, tig) holds rows g
+//                    and g + 8 for m = tig, digits 0 and 1, separately for the
+//                    even codes (D_e) and the odd ones (D_o, 16 times larger).
+// Per granule each lane folds
+//   16 V = 16 (256 D_e,0 + D_e,1) + 256 D_o,0 + D_o,1   (= 16 sum_k x' q)
+//   y   += s * ((xs / 16) * 16 V - z * xs * sum_k x')
+// with xs = 2^(e - 140), e the granule's largest bf16 exponent, so y
+// accumulates s * sum_k x (q - z) for its two rows.
 //
-// A quad-window is 256 k of the box: lane (g, tig) loads one 16-byte chunk
-// of weight row g / 2, chunk (g % 2) * 4 + tig, and its 4 words feed the 4
-// mma of the window, word t to mma t.  So mma t pairs slot 4 tig + e with
-// k = 128 h + 32 tig + 8 t + 2 e (even nibbles) and slot 16 + 4 tig + e
-// with the odd k after it, and half h = 0 / 1 is the first / second 128 k
-// of the window.  A small kernel (gemv_xfrag_kernel) writes the A
-// fragments in exactly this order, once per call, with the granule scales.
-//
-// Each lane then holds, per window, the exact sums sum_k q x' of weight row
-// tig against (m, p) = (g / 2, g % 2) for both halves, and folds them:
-//   y += s * (f1 * D - z * f2),  f1 = xs * 256^(1 - p),  f2 = [p == 1] xs * sum_k x'
-// with xs = 2^(e - 140), e the granule's largest bf16 exponent.  The two
-// digits meet in one shuffle when a row block is done; the work split and
-// the output are described at the kernel.
+// Output.  At the end of a row block the sixteen warps' sums meet in shared
+// memory and are added in a fixed order (so results do not depend on
+// timing), then biased and rounded once, or written as fp32 partials when K
+// is split into slices.
 #pragma once
 
 #include "gemv_stream.cuh"
@@ -40,15 +41,22 @@
 namespace w4 {
 
 constexpr int kMFrac = 6;          // fixed-point bits below the granule's leading binade
-constexpr int kMMaxWarps = 16;
+constexpr int kMR = 16;            // weight rows per stage (the mma's A rows)
+constexpr int kMK = 2048;          // k per stage
+constexpr int kMW = 16;            // consumer warps: one 128-k granule of each stage apiece
+constexpr int kMThreads = (kMW + 1) * 32;
+constexpr int kMWBytes = kMR * kMK / 2;    // 16 KB of packed weights per stage
+constexpr int kMRedStride = 68;            // floats per warp in the row-block reduction (64 + pad)
 
-// One slice's activation block: A fragments [window][mma t][8 M lanes]
-// (16 bytes each), then the fold constants [window][g = 2 m + p] as float4
-// {f1_h0, f2_h0, f1_h1, f2_h1} with f1 = xs * 256^(1 - p) and
-// f2 = [p == 1] xs * sum x'.
+// One slice's activation block: the B fragments [granule][2 halves][8 M
+// lanes][16 bytes] (lane 4 (2 m + p) + tig; half 0 holds words 0..3 of the
+// lane's 8-word record, half 1 words 4..7), then the fold constants
+// [granule][M] float2 {xs / 16, xs * sum x'}.
+__host__ __device__ inline size_t gemv_mma_xfrag_bytes(int M, int TKC) {
+    return static_cast<size_t>(TKC) / 128 * M * 256;
+}
 __host__ __device__ inline size_t gemv_mma_xblock_bytes(int M, int TKC) {
-    const size_t nqw = static_cast<size_t>(TKC) / 256;
-    return nqw * M * (4 * 8 * 16 + 2 * 16);
+    return static_cast<size_t>(TKC) / 128 * M * (256 + 8);
 }
 
 // Programmatic dependent launch: the prep kernel lets the GEMV start early,
@@ -56,12 +64,9 @@ __host__ __device__ inline size_t gemv_mma_xblock_bytes(int M, int TKC) {
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// One warp converts activation row m of window qw (256 k starting at
-// k_first) into `block`, a slice's activation block: lane = 16 h + 4 t + tig
+// A conversion unit is 256 k of one activation row: lane = 16 h + 4 t + tig
 // converts the 8 activations k_first + 128 h + 32 tig + 8 t .. + 7 (zero past
-// K).  `block` may be global (the prep kernel) or shared memory (the GEMV
-// converting its own slice).
-// The 8 activations of the lane (zero past K).
+// K), i.e. chunk t of B lane tig's 32 k in granule h of the unit.
 __device__ __forceinline__ uint4 xfrag_load(const uint16_t* __restrict__ X, int K, long long k_first, int m,
                                             int lane) {
     const int h = lane >> 4, t = (lane >> 2) & 3, tig = lane & 3;
@@ -71,13 +76,16 @@ __device__ __forceinline__ uint4 xfrag_load(const uint16_t* __restrict__ X, int 
     return v;
 }
 
-// Fixed point, digits and fold constants from the lane's 8 activations v.
-// x' = round(x * 2^(140 - e)) with e the largest bf16 exponent of the lane's
-// half (128 k); the power of two is exact in fp32 unless e < 14 (values
-// below 2^-113), where the integer path below is used instead.  The digits
-// are dh = floor((x' + 128) / 256) and dl = x' - 256 dh, so dl is in
-// [-128, 127] and |dh| <= 64.
-__device__ __forceinline__ void xfrag_store(uint4 v, int M, int nqw, int qw, int m, int lane, uint8_t* block) {
+// Fixed point, digits and fold constants from the lane's 8 activations v,
+// stored into `block` (global for the prep kernel, shared when the GEMV
+// converts its own slice) for unit qw of activation row m; ngran is the
+// slice's number of granules.
+// x' = round(x * 2^(140 - e)) with e the largest bf16 exponent of the
+// granule; the power of two is exact in fp32 unless e < 14 (values below
+// 2^-113), where the integer path is used instead.  The digits are
+// dh = floor((x' + 128) / 256) and dl = x' - 256 dh: dl is in [-128, 127]
+// and |dh| <= 64.
+__device__ __forceinline__ void xfrag_store(uint4 v, int M, int ngran, int qw, int m, int lane, uint8_t* block) {
     const int h = lane >> 4, t = (lane >> 2) & 3, tig = lane & 3;
     const uint32_t r[4] = {v.x, v.y, v.z, v.w};
     // largest magnitude: bf16 bit patterns order like their magnitudes
@@ -118,32 +126,26 @@ __device__ __forceinline__ void xfrag_store(uint4 v, int M, int nqw, int qw, int
     const uint32_t lo_e = pack4(dl[0], dl[2], dl[4], dl[6]), lo_o = pack4(dl[1], dl[3], dl[5], dl[7]);
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-    uint32_t* frag = reinterpret_cast<uint32_t*>(block);
-    // lane (g = 2 m + p, tig) of mma t: {even h0, even h1, odd h0, odd h1}
-    const size_t rec = (static_cast<size_t>(qw) * 4 + t) * (8 * M) + (2 * m) * 4 + tig;
-    frag[rec * 4 + h] = hi_e;
-    frag[rec * 4 + 2 + h] = hi_o;
-    frag[(rec + 4) * 4 + h] = lo_e;
-    frag[(rec + 4) * 4 + 2 + h] = lo_o;
+    // the 8-word record of B lane (2 m + p, tig) is {e0.b0, e0.b1, o0.b0,
+    // o0.b1, e1.b0, e1.b1, o1.b0, o1.b1}: chunk t fills word
+    // 4 (t >> 1) + (t & 1) (even k) and 4 (t >> 1) + 2 + (t & 1) (odd k)
+    const size_t gran = static_cast<size_t>(qw) * 2 + h;
+    uint32_t* half = reinterpret_cast<uint32_t*>(block + (gran * 2 + (t >> 1)) * (8 * M * 16));
+    const int l_hi = (2 * m) * 4 + tig, l_lo = l_hi + 4;
+    half[l_hi * 4 + (t & 1)] = hi_e;
+    half[l_hi * 4 + 2 + (t & 1)] = hi_o;
+    half[l_lo * 4 + (t & 1)] = lo_e;
+    half[l_lo * 4 + 2 + (t & 1)] = lo_o;
     if ((lane & 15) == 0) {
-        float* fs = reinterpret_cast<float*>(block + static_cast<size_t>(nqw) * M * 512);
+        float2* fc = reinterpret_cast<float2*>(block + static_cast<size_t>(ngran) * M * 256);
         // 2^(emax - 140): a normal float unless emax < 14
         const float xs_exact = emax >= 14 ? __int_as_float((emax - 13) << 23) : ldexpf(1.0f, emax - 134 - kMFrac);
-        const size_t f0 = (static_cast<size_t>(qw) * 2 * M + 2 * m) * 4 + 2 * h;   // p = 0
-        fs[f0] = 256.0f * xs_exact;
-        fs[f0 + 1] = 0.0f;
-        fs[f0 + 4] = xs_exact;                                                     // p = 1
-        fs[f0 + 5] = xs_exact * static_cast<float>(sum);
+        fc[gran * M + m] = make_float2(xs_exact * 0.0625f, xs_exact * static_cast<float>(sum));
     }
 }
 
-__device__ __forceinline__ void xfrag_convert(const uint16_t* __restrict__ X, int M, int K, long long k_first,
-                                              int nqw, int qw, int m, int lane, uint8_t* block) {
-    xfrag_store(xfrag_load(X, K, k_first, m, lane), M, nqw, qw, m, lane, block);
-}
-
 // Prep kernel for shapes whose conversion is too much to repeat in every
-// CTA: one warp per (slice, window, m).
+// CTA: one warp per (slice, unit of 256 k, m).
 __global__ void __launch_bounds__(256) gemv_xfrag_kernel(const uint16_t* __restrict__ X, int M, int K,
                                                          int TKC, int splits, uint8_t* __restrict__ out) {
     pdl_launch_dependents();
@@ -153,55 +155,51 @@ __global__ void __launch_bounds__(256) gemv_xfrag_kernel(const uint16_t* __restr
     const int m = static_cast<int>(unit % M);
     const long long sq = unit / M;
     const int slice = static_cast<int>(sq / nqw), qw = static_cast<int>(sq - static_cast<long long>(slice) * nqw);
-    xfrag_convert(X, M, K, static_cast<long long>(slice) * TKC + qw * 256, nqw, qw, m, threadIdx.x & 31,
-                  out + static_cast<size_t>(slice) * gemv_mma_xblock_bytes(M, TKC));
+    const int lane = threadIdx.x & 31;
+    xfrag_store(xfrag_load(X, K, static_cast<long long>(slice) * TKC + qw * 256, m, lane), M, TKC / 128, qw, m,
+                lane, out + static_cast<size_t>(slice) * gemv_mma_xblock_bytes(M, TKC));
 }
 
-// D = A B + C and D = A B (C = 0); the fragments are plain values, so the
-// compiler may schedule these freely.
-__device__ __forceinline__ void mma_s8u8_16832(int (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+// D = A B + C with A the u8 weight codes and B the s8 activation digits.
+__device__ __forceinline__ void mma_u8s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void mma_s8u8_16832_z(int (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%10,%10,%10,%10};"
-        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
-        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1), "r"(0));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // How the scales and zeros reach a stage:
 //   kSzConst  one scale and zero for the whole matrix (global mode): read
-//             once per thread, no per-box data;
-//   kSzTma2d  groupwise with G % 8 == 0: a TMA box of 4 rows x 16 groups of
-//             S and of Z, starting at the 8-aligned group at or below the
-//             box's first group;
-//   kSzTma1d  one group per row: a TMA box of the 8 rows' values around the
-//             box's 4 rows (S and Z seen as one-row 2-D tensors);
-//   kSzCopy   anything else: 4-byte cp.async copies (gemv_stream_kernel's
-//             scheme), tracked by the same barrier.
+//             once per thread, no per-stage data;
+//   kSzTma2d  groupwise with G % 8 == 0: a TMA box of the stage's rows x 16
+//             groups of S and of Z, starting at the 8-aligned group at or
+//             below the stage's first group;
+//   kSzTma1d  one group per row: a TMA box of the rows' values (S and Z seen
+//             as one-row 2-D tensors);
+//   kSzCopy   anything else: 4-byte cp.async copies by the producer warp,
+//             tracked by the same barrier.
 enum SzKind { kSzConst = 0, kSzTma2d = 1, kSzTma1d = 2, kSzCopy = 3 };
 
-// Shared-memory footprint of a stage's scales and zeros.  Tiled TMA writes
-// must start on a 128-byte boundary, so the Z box sits 128 bytes after the
-// S box in both TMA layouts.
+// Shared-memory footprint of a stage: 16 KB of weights, then S and Z
+// (tiled TMA writes start on 128-byte boundaries).
 __host__ __device__ inline int gemv_mma_sz_bytes(int sz, int szw) {
-    return sz == kSzTma2d ? 2 * 128 : sz == kSzTma1d ? 128 + 16 : sz == kSzCopy ? 2 * kSR * szw * 4 : 0;
+    return sz == kSzTma2d ? 2 * kMR * 16 * 2 : sz == kSzTma1d ? 2 * 128 : sz == kSzCopy ? 2 * kMR * szw * 4 : 0;
 }
 __host__ __device__ inline int gemv_mma_stage_bytes(int sz, int szw) {
-    return (kSBBytes + gemv_mma_sz_bytes(sz, szw) + 127) / 128 * 128;
+    return (kMWBytes + gemv_mma_sz_bytes(sz, szw) + 127) / 128 * 128;
 }
-__host__ __device__ inline size_t gemv_mma_smem_bytes(int M, int TKC, int warps, int stages, int sz, int szw) {
-    size_t b = 1024;
-    b += static_cast<size_t>(warps) * stages * gemv_mma_stage_bytes(sz, szw);
-    b += static_cast<size_t>(warps) * kSR * 8 * 16;                 // per-box fp32 scale / zero table
-    b += static_cast<size_t>(warps) * 2 * kSR * M * 4;             // shared-row-block slots
-    b += gemv_mma_xblock_bytes(M, TKC);
-    b += static_cast<size_t>(warps) * stages * 8 + 8 + 16;
+__host__ __device__ inline size_t gemv_mma_smem_bytes(int M, int TKC, int stages, int sz, int szw) {
+    size_t b = 1024;                                                   // alignment slack
+    b += static_cast<size_t>(stages) * gemv_mma_stage_bytes(sz, szw);
+    b += (gemv_mma_xblock_bytes(M, TKC) + 15) / 16 * 16;
+    b += static_cast<size_t>(2) * kMW * kMRedStride * 4;               // row-block reduction, 2 buffers
+    b += static_cast<size_t>(stages) * 16 + 8 + 16;                    // barriers, abort flag
     return b;
 }
+// Scale / zero words per row and stage on the copy path: the groups a
+// stage touches, plus one half for the 4-byte alignment, rounded up.
+__host__ __device__ inline int gemv_mma_sz_words(int g) { return ((kMK + g - 1) / g + 3) / 2; }
 
 // Arguments of gemv_mma_kernel.
 struct GemvMmaArgs {
@@ -213,66 +211,59 @@ struct GemvMmaArgs {
     uint16_t* Y;
     float* partial;           // [splits, M, N] when splits > 1
     int N, K, g, G, sz_row;
-    int TKC;                  // k per slice (a whole number of boxes)
+    int TKC;                  // k per slice (a whole number of stages)
     int splits;               // slices; CTA c works on slice c / cps
-    int nbs;                  // boxes per slice and row block
-    int nrb;                  // row blocks (4 rows each)
+    int nks;                  // stages per row block and slice
+    int nrb;                  // row blocks (16 rows each)
     int cps;                  // CTAs per slice
-    int stages;               // TMA stages per warp
+    int stages;               // ring depth
     int szw;                  // copy path: scale / zero words per row and stage
     long long sz_total;       // halves in each of S and Z (N * sz_row, or 1)
 };
 
 // Work split: each CTA of a slice takes a contiguous range of whole row
-// blocks (balanced to within one row block), and its warps cut the CTA's
-// boxes, row block major (box b = row block b / nbs, k box b % nbs), into
-// one contiguous range each, equal to within one box; no warp waits for
-// another until the end.  A row block one warp covers completely is written
-// at once.  A row block shared by neighbouring warps goes through per-warp
-// slots in shared memory: after the CTA's single barrier, the warp holding
-// the row block's last box sums the slots in warp order, so the result does
-// not depend on timing.
+// blocks (balanced to within one row block) and walks them row block by row
+// block, stage by stage along its K slice.
 //
 // Activations: with `xblocks` null every CTA converts its K slice of X into
-// the fragment layout itself while its first weight boxes are in flight (the
-// planner picks this when the conversion is a few units per warp); else the
+// the fragment layout itself while the producer fills the ring (the planner
+// picks this when the conversion is at most a few units per warp); else the
 // kernel is a programmatic dependent of gemv_xfrag_kernel and fetches the
 // prepared block with one bulk copy.
 template <int M, int GK, int SZ>
-__global__ void __launch_bounds__(kMMaxWarps * 32, 1)
+__global__ void __launch_bounds__(kMThreads, 1)
     gemv_mma_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                     const __grid_constant__ CUtensorMap zmap, const GemvMmaArgs a) {
     static_assert(M >= 1 && M <= 4, "M");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const int NW = blockDim.x >> 5;
     const int NS = a.stages;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
     const int g = lane >> 2, tig = lane & 3;
-    const int nqw = a.TKC / 256;
+    const int ngran = a.TKC / 128;
     const uint32_t xbytes = static_cast<uint32_t>(gemv_mma_xblock_bytes(M, a.TKC));
     const int SB = gemv_mma_stage_bytes(SZ, a.szw);
-    // bytes the scale / zero boxes add to a stage's transaction count
-    constexpr int kSzTx = SZ == kSzTma2d ? 2 * kSR * 16 * 2 : SZ == kSzTma1d ? 2 * 8 * 2 : 0;
-    uint8_t* ring = base;                                                    // [warp][stage][SB]
-    float4* table = reinterpret_cast<float4*>(ring + NW * NS * SB);          // [warp][8 windows][4 rows]
-    float* slots = reinterpret_cast<float*>(table + NW * kSR * 8);           // [warp][2][4 rows][M]
-    uint8_t* xblk = reinterpret_cast<uint8_t*>(slots + NW * 2 * kSR * M);
-    const uint4* frag = reinterpret_cast<const uint4*>(xblk);                // [qw][t][8M]
-    const float4* fsc = reinterpret_cast<const float4*>(xblk + static_cast<size_t>(nqw) * M * 512);  // [qw][2M]
-    uint64_t* full = reinterpret_cast<uint64_t*>(xblk + xbytes);
-    uint64_t* xbar = full + NW * NS;
+    constexpr int kSzTx = SZ == kSzTma2d ? 2 * kMR * 16 * 2 : SZ == kSzTma1d ? 2 * kMR * 2 : 0;
+    uint8_t* ring = base;                                                   // [stage][SB]
+    uint8_t* xblk = ring + NS * SB;                                         // fragments, then constants
+    float* red = reinterpret_cast<float*>(xblk + ((xbytes + 15) & ~15u));   // [2][warp][kMRedStride]
+    uint64_t* full = reinterpret_cast<uint64_t*>(red + 2 * kMW * kMRedStride);
+    uint64_t* empty = full + NS;
+    uint64_t* xbar = empty + NS;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(xbar + 1);
 
     if (tid == 0) {
-        // a stage completes on the elected lane's expect-tx arrival and its
-        // bytes; the copy path adds one cp.async arrival per lane
-        for (int i = 0; i < NW * NS; ++i) mbar_init(&full[i], SZ == kSzCopy ? 33 : 1);
+        for (int i = 0; i < NS; ++i) {
+            // a stage completes on the elected lane's expect-tx arrival and its
+            // bytes; the copy path adds one cp.async arrival per producer lane
+            mbar_init(&full[i], SZ == kSzCopy ? 33 : 1);
+            mbar_init(&empty[i], kMW);
+        }
         mbar_init(xbar, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (tid == 32) {
+    if (tid == kMW * 32) {
         tma_prefetch_desc(&wmap);
         if (SZ == kSzTma2d || SZ == kSzTma1d) {
             tma_prefetch_desc(&smap);
@@ -284,253 +275,201 @@ __global__ void __launch_bounds__(kMMaxWarps * 32, 1)
     const int slice = blockIdx.x / a.cps, cta = blockIdx.x - (blockIdx.x / a.cps) * a.cps;
     const int rb_lo = static_cast<int>(static_cast<long long>(cta) * a.nrb / a.cps);
     const int rb_hi = static_cast<int>(static_cast<long long>(cta + 1) * a.nrb / a.cps);
-    const int T = (rb_hi - rb_lo) * a.nbs;                       // boxes of this CTA
-    auto wstart = [&](int ww) { return static_cast<int>(static_cast<long long>(ww) * T / NW); };
-    auto warp_of = [&](int b) { return static_cast<int>((static_cast<long long>(b + 1) * NW - 1) / T); };
-    const int b_begin = wstart(warp), b_end = wstart(warp + 1);
+    const int items = (rb_hi - rb_lo) * a.nks;
+    const int k_slice = slice * a.TKC;
     int gshift = 0;
     if (GK == kGroupsPow2) gshift = __ffs(a.g) - 1;
-
-    struct Cur {
-        int b, rb, kb;   // CTA-local box, its row block (absolute) and k box
-    };
-    auto advance = [&](Cur& c) {
-        ++c.b;
-        if (++c.kb == a.nbs) {
-            c.kb = 0;
-            ++c.rb;
-        }
-    };
-    const Cur start{b_begin, rb_lo + b_begin / a.nbs, b_begin - (b_begin / a.nbs) * a.nbs};
-    auto box_k0 = [&](const Cur& c) { return slice * a.TKC + c.kb * kSBK; };
-    auto box_row0 = [&](const Cur& c) { return c.rb * kSR; };
-    auto first_group = [&](int k0) {
+    auto group_of = [&](int k) {
         if (GK == kGroupsOne) return 0;
-        if (GK == kGroupsPow2) return k0 >> gshift;
-        return k0 / a.g;
+        if (GK == kGroupsPow2) return k >> gshift;
+        return k / a.g;
     };
 
-    const int sz_arr = (lane >> 2) & 1, sz_row_i = lane & 3;   // copy path: lane's array and row
-    int islot = 0;
-    Cur ic = start;
-    auto issue = [&]() {
-        if (ic.b < b_end) {
-            const int k0 = box_k0(ic), row0 = box_row0(ic);
-            const int st = warp * NS + islot;
-            uint8_t* sd = ring + st * SB;
+    if (warp == kMW) {
+        // ------------------------------------------------------ producer
+        int rb = rb_lo, ks = 0;
+        for (int it = 0; it < items; ++it) {
+            const int s = it % NS;
+            if (it >= NS) {
+                const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&empty[s], ((it / NS) - 1) & 1u,
+                                                                          abort_flag, kErrTimeoutEmpty));
+                if (!ok) break;
+            }
+            uint8_t* sd = ring + s * SB;
+            const int k0 = k_slice + ks * kMK, row0 = rb * kMR;
             if (SZ == kSzCopy) {
-                const long long h0 =
-                    (static_cast<long long>(row0 + sz_row_i) * a.sz_row + first_group(k0)) & ~1ll;
-                uint32_t* szd = reinterpret_cast<uint32_t*>(sd + kSBBytes) + (sz_arr * kSR + sz_row_i) * a.szw;
-                const __half* src = sz_arr ? a.Z : a.S;
-                for (int q = lane >> 3; q < a.szw; q += 4) {
+                // lane -> (array, row): the row's szw words around the stage's
+                // groups, zero-filled past the end of S / Z
+                const int arr = lane >> 4, r = lane & 15;
+                const long long h0 = (static_cast<long long>(row0 + r) * a.sz_row + group_of(k0)) & ~1ll;
+                uint32_t* dst = reinterpret_cast<uint32_t*>(sd + kMWBytes) + (arr * kMR + r) * a.szw;
+                const __half* src = arr ? a.Z : a.S;
+                for (int q = 0; q < a.szw; ++q) {
                     const long long hh = h0 + 2 * q;
                     const long long avail = a.sz_total - hh;
                     const uint32_t bytes = avail >= 2 ? 4u : (avail == 1 ? 2u : 0u);
-                    cp_async_4(szd + q, src + (bytes ? hh : 0), bytes);
+                    cp_async_4(dst + q, src + (bytes ? hh : 0), bytes);
                 }
-                cp_async_arrive_noinc(&full[st]);
+                cp_async_arrive_noinc(&full[s]);
             }
-            // (after a timed-out wait the loads keep coming; the kernel lets
-            // them land before it exits)
             if (SZ == kSzTma2d) {
-                const int x = first_group(k0) & ~7;
-                tma_issue_elected<3>(&full[st], kSBBytes + kSzTx, sd, &wmap, k0 / 8, row0, sd + kSBBytes, &smap, x,
-                                     row0, sd + kSBBytes + 128, &zmap, x, row0);
+                const int x = group_of(k0) & ~7;
+                tma_issue_elected<3>(&full[s], kMWBytes + kSzTx, sd, &wmap, k0 / 8, row0, sd + kMWBytes, &smap, x,
+                                     row0, sd + kMWBytes + kMR * 32, &zmap, x, row0);
             } else if (SZ == kSzTma1d) {
-                tma_issue_elected<3>(&full[st], kSBBytes + kSzTx, sd, &wmap, k0 / 8, row0, sd + kSBBytes, &smap,
-                                     row0 & ~7, 0, sd + kSBBytes + 128, &zmap, row0 & ~7, 0);
+                tma_issue_elected<3>(&full[s], kMWBytes + kSzTx, sd, &wmap, k0 / 8, row0, sd + kMWBytes, &smap, row0,
+                                     0, sd + kMWBytes + 128, &zmap, row0, 0);
             } else {
-                tma_issue_elected<1>(&full[st], kSBBytes, sd, &wmap, k0 / 8, row0);
+                tma_issue_elected<1>(&full[s], kMWBytes, sd, &wmap, k0 / 8, row0);
             }
-            if (++islot == NS) islot = 0;
-            advance(ic);
+            if (it == 0 && a.xblocks != nullptr) {
+                // the prepared activation block right after the first stage,
+                // so that it does not queue behind the whole ring
+                pdl_wait();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(xbar, xbytes);
+                    bulk_load_1d(xblk, a.xblocks + static_cast<size_t>(slice) * xbytes, xbytes, xbar);
+                }
+                __syncwarp();
+            }
+            if (++ks == a.nks) {
+                ks = 0;
+                ++rb;
+            }
         }
-    };
-    if (a.xblocks == nullptr) {
-        // this warp's activation units (at most 4: the planner's limit) are
-        // loaded first, the ring is filled while they are in flight, and
-        // the conversion runs while the first boxes are in flight
-        constexpr int kMaxUnits = 4;
-        const long long k_slice = static_cast<long long>(slice) * a.TKC;
-        uint4 raw[kMaxUnits];
-#pragma unroll
-        for (int i = 0; i < kMaxUnits; ++i) {
-            const int u = warp + i * NW;
-            raw[i] = make_uint4(0u, 0u, 0u, 0u);
-            if (u < nqw * M) raw[i] = xfrag_load(a.X, a.K, k_slice + (u / M) * 256, u - (u / M) * M, lane);
-        }
-        for (int b = 0; b < NS; ++b) issue();
-#pragma unroll
-        for (int i = 0; i < kMaxUnits; ++i) {
-            const int u = warp + i * NW;
-            if (u < nqw * M) xfrag_store(raw[i], M, nqw, u / M, u - (u / M) * M, lane, xblk);
-        }
-        __syncthreads();
     } else {
-        // one stage of weights first; then, once the prep kernel is done,
-        // the activation block (so that it does not queue behind the whole
-        // ring); then the rest of the ring
-        issue();
-        pdl_wait();
-        if (tid == 0 && T > 0) {
-            mbar_arrive_expect_tx(xbar, xbytes);
-            bulk_load_1d(xblk, a.xblocks + static_cast<size_t>(slice) * xbytes, xbytes, xbar);
-        }
-        for (int b = 1; b < NS; ++b) issue();
-        if (T > 0) mbar_wait_bounded(xbar, 0, abort_flag, kErrTimeoutTmaFull);
-    }
-
-    const int wrow = g >> 1, wchunk = (g & 1) * 4 + tig;   // the B chunk this lane loads
-    const bool f_lane = g < 2 * M;
-    // lanes without activation rows (g >= 2M) never load: their fragments
-    // and fold constants stay zero for the whole kernel
-    uint4 af[4];
+        // ------------------------------------------------------ consumers
+        if (a.xblocks == nullptr) {
+            // this warp's activation units (at most 4: the planner's limit)
+            // are loaded, converted and stored while the ring fills
+            constexpr int kMaxUnits = 4;
+            const int nunits = (a.TKC / 256) * M;
+            uint4 raw[kMaxUnits];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) af[t] = make_uint4(0u, 0u, 0u, 0u);
-    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-    float s_const = 0.f, z_const = 0.f;
-    if (SZ == kSzConst) {
-        s_const = __half2float(a.S[0]);
-        z_const = __half2float(a.Z[0]);
-    }
-    float4* wtable = table + warp * kSR * 8;
-    const int tq = lane & 7, ti = lane >> 3;               // table entry this lane builds
-
-    // outputs: after the digit shuffle, lanes with even g < 2M hold
-    // (m = g / 2, row tig) of the row block
-    auto store = [&](int m, int n, float v) {
-        if (a.splits == 1) {
-            if (a.bias) v += bf16_bits_to_float(a.bias[n]);
-            a.Y[static_cast<size_t>(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-        } else {
-            a.partial[(static_cast<size_t>(slice) * M + m) * a.N + n] = v;
-        }
-    };
-    const int first_rb = start.rb;
-    auto finish = [&](int rb, int nb, float y) {
-        const float v = y + __shfl_xor_sync(0xFFFFFFFFu, y, 4);
-        if (!(g & 1) && f_lane) {
-            if (nb == a.nbs) {
-                const int n = rb * kSR + tig;
-                if (n < a.N) store(g >> 1, n, v);
-            } else {
-                slots[((warp * 2) + (rb == first_rb ? 0 : 1)) * (kSR * M) + tig * M + (g >> 1)] = v;
+            for (int i = 0; i < kMaxUnits; ++i) {
+                const int u = warp + i * kMW;
+                raw[i] = make_uint4(0u, 0u, 0u, 0u);
+                if (u < nunits) raw[i] = xfrag_load(a.X, a.K, k_slice + (u / M) * 256, u - (u / M) * M, lane);
             }
-        }
-    };
-
-    int cslot = 0;
-    uint32_t cpar = 0;
-    Cur cc = start;
-    float y = 0.0f;
-    int nb_rb = 0;
-    for (int b = b_begin; b < b_end; ++b) {
-        const int k0 = box_k0(cc), row0 = box_row0(cc);
-        const int st = warp * NS + cslot;
-        __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[st], cpar, abort_flag, kErrTimeoutTmaFull));
-        if (++cslot == NS) {
-            cslot = 0;
-            cpar ^= 1u;
-        }
-        const uint8_t* sb = ring + st * SB;
-        if (SZ != kSzConst) {
-            // fp32 table of (s, z) for window tq, row ti, both halves (the 4
-            // rows of a window are adjacent: the readers hit 4 distinct banks)
-            const int grp_lo = first_group(k0);
-            int o0, o1;
-            if (GK == kGroupsOne) {
-                o0 = 0;
-                o1 = 0;
-            } else if (GK == kGroupsPow2) {
-                o0 = (tq * 256) >> gshift;
-                o1 = (tq * 256 + 128) >> gshift;
-            } else {
-                const int r0 = k0 - grp_lo * a.g;
-                o0 = (r0 + tq * 256) / a.g;
-                o1 = (r0 + tq * 256 + 128) / a.g;
-            }
-            const __half* sh = reinterpret_cast<const __half*>(sb + kSBBytes);
-            const __half *ps, *pz;
-            if (SZ == kSzTma2d) {
-                ps = sh + ti * 16 + (grp_lo & 7);
-                pz = ps + 64;                    // Z box 128 bytes after the S box
-            } else if (SZ == kSzTma1d) {
-                ps = sh + (row0 & 7) + ti;
-                pz = ps + 64;
-            } else {
-                ps = sh + ti * 2 * a.szw + ((((row0 + ti) & a.sz_row) ^ grp_lo) & 1);
-                pz = ps + kSR * 2 * a.szw;
-            }
-            wtable[tq * kSR + ti] = make_float4(__half2float(ps[o0]), __half2float(pz[o0]), __half2float(ps[o1]),
-                                                __half2float(pz[o1]));
-            __syncwarp();
-        }
-        // per-box bases: every window below is an immediate offset from them
-        const uint8_t* wsrc = sb + wrow * 1024 + wchunk * 16;
-        const int qw0 = cc.kb * (kSBK / 256);
-        const uint4* fb = frag + qw0 * (32 * M) + lane;
-        const float4* cb = fsc + qw0 * (2 * M) + g;
 #pragma unroll
-        for (int qwl = 0; qwl < kSBK / 256; ++qwl) {
-            const uint4 wv = *reinterpret_cast<const uint4*>(wsrc + qwl * 128);
-            if (lane < 8 * M) {
-#pragma unroll
-                for (int t = 0; t < 4; ++t) af[t] = fb[(qwl * 4 + t) * (8 * M)];
+            for (int i = 0; i < kMaxUnits; ++i) {
+                const int u = warp + i * kMW;
+                if (u < nunits) xfrag_store(raw[i], M, ngran, u / M, u - (u / M) * M, lane, xblk);
             }
-            if (f_lane) f = cb[qwl * 2 * M];
-            int acc[2][4];
-            mma_s8u8_16832_z(acc[0], af[0], wv.x & 0x0F0F0F0Fu, (wv.x >> 4) & 0x0F0F0F0Fu);
-            mma_s8u8_16832_z(acc[1], af[1], wv.y & 0x0F0F0F0Fu, (wv.y >> 4) & 0x0F0F0F0Fu);
-            mma_s8u8_16832(acc[0], af[2], wv.z & 0x0F0F0F0Fu, (wv.z >> 4) & 0x0F0F0F0Fu);
-            mma_s8u8_16832(acc[1], af[3], wv.w & 0x0F0F0F0Fu, (wv.w >> 4) & 0x0F0F0F0Fu);
-            const int d0 = acc[0][0] + acc[1][0];   // half 0: A row g, B column (tig, 0)
-            const int d1 = acc[0][3] + acc[1][3];   // half 1: A row g + 8, B column (tig, 1)
-            float4 sz;
-            if (SZ == kSzConst) sz = make_float4(s_const, z_const, s_const, z_const);
-            else sz = wtable[qwl * kSR + tig];
-            y = fmaf(sz.x, fmaf(f.x, static_cast<float>(d0), -sz.y * f.y), y);
-            y = fmaf(sz.z, fmaf(f.z, static_cast<float>(d1), -sz.w * f.w), y);
+            named_barrier_sync(1, kMW * 32);
+        } else if (items > 0) {
+            // the producer fetches the prepared block once the prep kernel is done
+            mbar_wait_bounded(xbar, 0, abort_flag, kErrTimeoutTmaFull);
         }
-        __syncwarp();
-        issue();
-        ++nb_rb;
-        const int rb = cc.rb;
-        const bool rb_done = (cc.kb == a.nbs - 1) || (b == b_end - 1);
-        advance(cc);
-        if (rb_done) {
-            finish(rb, nb_rb, y);
-            y = 0.0f;
-            nb_rb = 0;
-        }
-    }
 
-    // row blocks shared by neighbouring warps: the warp with a shared row
-    // block's last box adds the slots of all its contributors in warp order
-    __syncthreads();
-    if (b_begin < b_end) {
-        const int last_rb = rb_lo + (b_end - 1) / a.nbs;
-        for (int side = 0; side < 2; ++side) {
-            const int rb = side ? last_rb : first_rb;
-            if (side && rb == first_rb) break;
-            const int lb0 = (rb - rb_lo) * a.nbs, lb1 = lb0 + a.nbs - 1;   // CTA-local boxes of rb
-            const bool partial = b_begin > lb0 || b_end - 1 < lb1;
-            if (!partial || warp_of(lb1) != warp) continue;
-            if (lane < kSR * M) {
-                const int r = lane / M, m = lane - (lane / M) * M;
-                float s = 0.0f;
-                for (int ww = warp_of(lb0); ww <= warp; ++ww) {
-                    const int ws = wstart(ww);
-                    if (ws == wstart(ww + 1)) continue;
-                    const int sslot = (rb_lo + ws / a.nbs == rb) ? 0 : 1;
-                    s += slots[(ww * 2 + sslot) * (kSR * M) + r * M + m];
+        const bool b_lane = lane < 8 * M;        // lanes whose B columns hold activations
+        const int mf = min(tig, M - 1);          // fold constants of activation row m = tig
+        float s_const = 0.f, z_const = 0.f;
+        if (SZ == kSzConst) {
+            s_const = __half2float(a.S[0]);
+            z_const = __half2float(a.Z[0]);
+        }
+        const uint4* xb4 = reinterpret_cast<const uint4*>(xblk);
+        const float2* fcs = reinterpret_cast<const float2*>(xblk + static_cast<size_t>(ngran) * M * 256);
+        float y0 = 0.f, y1 = 0.f;                // rows g and g + 8 of the row block, m = tig
+        int rb = rb_lo, ks = 0, rbi = 0;
+        for (int it = 0; it < items; ++it) {
+            const int s = it % NS;
+            __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[s], (it / NS) & 1u, abort_flag, kErrTimeoutTmaFull));
+            const uint8_t* sb = ring + s * SB;
+            const int gl = ks * (kMK / 128) + warp;               // granule within the slice
+            const int kg = k_slice + gl * 128;                    // its first k
+            if (kg < a.K) {
+                const uint8_t* wrow = sb + g * 1024 + warp * 64 + tig * 16;
+                const uint4 wa = *reinterpret_cast<const uint4*>(wrow);
+                const uint4 wb = *reinterpret_cast<const uint4*>(wrow + 8 * 1024);
+                uint4 b0 = make_uint4(0u, 0u, 0u, 0u), b1 = b0;
+                if (b_lane) {
+                    const uint4* xg = xb4 + static_cast<size_t>(gl) * (16 * M);
+                    b0 = xg[lane];
+                    b1 = xg[8 * M + lane];
                 }
-                const int n = rb * kSR + r;
-                if (n < a.N) store(m, n, s);
+                const float2 fc = fcs[gl * M + mf];
+                int de[4] = {0, 0, 0, 0}, dd[4] = {0, 0, 0, 0};
+                constexpr uint32_t kLo = 0x0F0F0F0Fu, kHi = 0xF0F0F0F0u;
+                mma_u8s8_16832(de, wa.x & kLo, wb.x & kLo, wa.y & kLo, wb.y & kLo, b0.x, b0.y);
+                mma_u8s8_16832(dd, wa.x & kHi, wb.x & kHi, wa.y & kHi, wb.y & kHi, b0.z, b0.w);
+                mma_u8s8_16832(de, wa.z & kLo, wb.z & kLo, wa.w & kLo, wb.w & kLo, b1.x, b1.y);
+                mma_u8s8_16832(dd, wa.z & kHi, wb.z & kHi, wa.w & kHi, wb.w & kHi, b1.z, b1.w);
+                // scales and zeros of rows g and g + 8 for this granule's group
+                float s0, z0, s1, z1;
+                if (SZ == kSzConst) {
+                    s0 = s1 = s_const;
+                    z0 = z1 = z_const;
+                } else {
+                    const __half* sh = reinterpret_cast<const __half*>(sb + kMWBytes);
+                    const int grp = group_of(kg);
+                    if (SZ == kSzTma2d) {
+                        const int gi = grp - (group_of(k_slice + ks * kMK) & ~7);
+                        s0 = __half2float(sh[g * 16 + gi]);
+                        s1 = __half2float(sh[(g + 8) * 16 + gi]);
+                        z0 = __half2float(sh[kMR * 16 + g * 16 + gi]);
+                        z1 = __half2float(sh[kMR * 16 + (g + 8) * 16 + gi]);
+                    } else if (SZ == kSzTma1d) {
+                        s0 = __half2float(sh[g]);
+                        s1 = __half2float(sh[g + 8]);
+                        z0 = __half2float(sh[64 + g]);
+                        z1 = __half2float(sh[64 + g + 8]);
+                    } else {
+                        // row r's words start at half (row r, first group)
+                        // rounded down to even
+                        const int fg = group_of(k_slice + ks * kMK);
+                        const int row0 = rb * kMR;
+                        const int o0 = grp - fg + ((((row0 + g) & a.sz_row) ^ fg) & 1);
+                        const int o1 = grp - fg + ((((row0 + g + 8) & a.sz_row) ^ fg) & 1);
+                        const int w2 = 2 * a.szw;
+                        s0 = __half2float(sh[g * w2 + o0]);
+                        s1 = __half2float(sh[(g + 8) * w2 + o1]);
+                        z0 = __half2float(sh[(kMR + g) * w2 + o0]);
+                        z1 = __half2float(sh[(kMR + g + 8) * w2 + o1]);
+                    }
+                }
+                const int v0 = (de[0] * 256 + de[1]) * 16 + dd[0] * 256 + dd[1];
+                const int v1 = (de[2] * 256 + de[3]) * 16 + dd[2] * 256 + dd[3];
+                y0 = fmaf(s0, fmaf(fc.x, static_cast<float>(v0), -z0 * fc.y), y0);
+                y1 = fmaf(s1, fmaf(fc.x, static_cast<float>(v1), -z1 * fc.y), y1);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            if (++ks == a.nks) {
+                // row block done: the 16 warps' sums meet in shared memory and
+                // are added in a fixed order (warp pairs, then a shuffle tree)
+                float* rbuf = red + (rbi & 1) * (kMW * kMRedStride);
+                reinterpret_cast<float2*>(rbuf + warp * kMRedStride)[lane] = make_float2(y0, y1);
+                named_barrier_sync(1, kMW * 32);
+                const int t = warp * 32 + lane;
+                const int v = t >> 3, j = t & 7;        // output (row r, m) and its pair of warps
+                const int r = v >> 2, m = v & 3;
+                const int src = ((r & 7) * 4 + m) * 2 + (r >> 3);
+                float sum = rbuf[(2 * j) * kMRedStride + src] + rbuf[(2 * j + 1) * kMRedStride + src];
+                sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+                sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+                sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
+                const int n = rb * kMR + r;
+                if (j == 0 && m < M && n < a.N) {
+                    if (a.splits == 1) {
+                        float o = sum;
+                        if (a.bias) o += bf16_bits_to_float(a.bias[n]);
+                        a.Y[static_cast<size_t>(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+                    } else {
+                        a.partial[(static_cast<size_t>(slice) * M + m) * a.N + n] = sum;
+                    }
+                }
+                y0 = 0.f;
+                y1 = 0.f;
+                ks = 0;
+                ++rb;
+                ++rbi;
             }
         }
     }
     if (*abort_flag) {
+        // let copies still in flight land before the CTA's memory is released
         const unsigned long long t0 = global_timer_ns();
         while (global_timer_ns() - t0 < 1000000ull) {
         }

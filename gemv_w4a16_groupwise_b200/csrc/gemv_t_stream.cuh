@@ -7,7 +7,7 @@
 // apart (rows are contiguous along K), so each CTA owns a strip of 2048 k
 // (one box width) and walks a range of rows:
 //   * a producer warp streams 4-row x 1 KB boxes of the strip (and the
-//     rows' scale / zero boxes, as in gemv_mma_kernel) through a CTA-wide
+//     rows' scale / zero boxes) through a CTA-wide
 //     ring; a stage is refilled once all 8 consumer warps released it;
 //   * consumer warp w owns k = 256 w .. 256 w + 255 of the strip, lane l
 //     one packed word (8 k, inside one group) of it;
@@ -44,9 +44,16 @@ struct GemvTStreamArgs {
     int stages;
 };
 
+// A stage: one 4-row x 1 KB box of packed words, then the S and Z boxes
+// (4 rows x 16 groups each, or the 8 rows' values around the box with one
+// group per row), each starting on a 128-byte boundary.
+__host__ __device__ inline int gemv_t_stage_bytes(int sz) {
+    return (kSBBytes + (sz == kSzTma2d ? 2 * 128 : sz == kSzTma1d ? 128 + 16 : 0) + 127) / 128 * 128;
+}
+
 // Ring, barriers, and dY of the CTA's rows as one float4 per row.
 __host__ __device__ inline size_t gemv_t_stream_smem_bytes(int stages, int sz, int rows_per_split) {
-    return 1024 + static_cast<size_t>(stages) * gemv_mma_stage_bytes(sz, 0) + static_cast<size_t>(stages) * 16 + 16 +
+    return 1024 + static_cast<size_t>(stages) * gemv_t_stage_bytes(sz) + static_cast<size_t>(stages) * 16 + 16 +
            static_cast<size_t>(rows_per_split) * 16;
 }
 
@@ -59,7 +66,7 @@ __global__ void __launch_bounds__(kTSThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int NS = a.stages;
-    const int SB = gemv_mma_stage_bytes(SZ, 0);
+    const int SB = gemv_t_stage_bytes(SZ);
     constexpr int kSzTx = SZ == kSzTma2d ? 2 * kSR * 16 * 2 : SZ == kSzTma1d ? 2 * 8 * 2 : 0;
     uint8_t* ring = base;                                                    // [stage][SB]
     uint64_t* full = reinterpret_cast<uint64_t*>(ring + NS * SB);

@@ -244,7 +244,7 @@ struct StreamPlan {
     bool ok = false;
     int TKC = 0, splits = 1, nbs = 0, KP = 1, RBP = kSW, rounds = 0, units = 0, grid = 0, stages = 2;
     int szw = 0, warps = kSW, sz = 0;
-    int nrb = 0, cps = 0;                      // tensor-pipe kernel: row blocks, CTAs per slice
+    int nrb = 0, cps = 0, nks = 0;             // tensor-pipe kernel: row blocks, CTAs per slice, stages per row block
     bool mma = false, in_kernel_x = false;
     size_t smem = 0, xbytes = 0, ws = 0, partial_off = 0;
 };
@@ -310,45 +310,46 @@ StreamPlan plan_stream(int M, int N, int K, const Meta& meta, const DeviceInfo& 
 }
 
 // Tensor-pipe GEMV (gemv_mma_kernel): group length a multiple of 128, or
-// one group per row.  Same slicing as the CUDA-core kernel, but the ring
-// may hold 8, 12 or 16 warps: the deepest ring (warps x stages) whose
-// activation block for all of K fits wins; if none fits, 8 warps x 2
-// stages and K split into slices.
+// one group per row.  A CTA-wide ring of 16-row x 2048-k stages beside the
+// slice's activation block; K is split into slices only when the block of
+// all of K leaves no room for a ring of 4 stages (then 3).
 StreamPlan plan_mma(int M, int N, int K, int sz, int szw, const DeviceInfo& di) {
     StreamPlan p;
     p.szw = szw;
     p.sz = sz;
-    const int nb_total = (K + kSBK - 1) / kSBK;
-    auto nbs_fit = [&](int warps, int stages) {
-        int best = 0;
-        for (int nb = 1; nb <= nb_total; ++nb) {
-            if (gemv_mma_smem_bytes(M, nb * kSBK, warps, stages, sz, szw) > static_cast<size_t>(di.max_smem_optin))
-                break;
-            best = nb;
+    p.warps = kMThreads / 32;
+    const int nk_total = (K + kMK - 1) / kMK;
+    const size_t cap = static_cast<size_t>(di.max_smem_optin);
+    // the fewest K slices whose activation block leaves room for a ring of
+    // at least 4 stages (deeper rings first, up to 8), else 3
+    for (int min_st : {4, 3}) {
+        for (int splits = 1; splits <= nk_total; ++splits) {
+            const int nks = (nk_total + splits - 1) / splits;
+            int st = 0;
+            for (int c = 8; c >= min_st; --c)
+                if (gemv_mma_smem_bytes(M, nks * kMK, c, sz, szw) <= cap) {
+                    st = c;
+                    break;
+                }
+            if (st == 0) continue;
+            p.splits = (nk_total + nks - 1) / nks;
+            p.nks = nks;
+            p.stages = st;
+            break;
         }
-        return best;
-    };
-    static const int kRings[][2] = {{16, 3}, {12, 4}, {16, 2}, {12, 3}, {8, 4}, {12, 2}, {8, 3}, {8, 2}};
-    int nbs_max = 0;
-    for (const auto& r : kRings) {
-        p.warps = r[0];
-        p.stages = r[1];
-        nbs_max = nbs_fit(p.warps, p.stages);
-        if (nbs_max >= nb_total) break;
+        if (p.stages) break;
     }
-    if (nbs_max == 0) return p;
-    p.splits = (nb_total + nbs_max - 1) / nbs_max;
-    p.nbs = (nb_total + p.splits - 1) / p.splits;
-    p.TKC = p.nbs * kSBK;
-    p.nrb = (N + kSR - 1) / kSR;
+    if (p.stages == 0) return p;
+    p.TKC = p.nks * kMK;
+    p.nrb = (N + kMR - 1) / kMR;
     // CTAs per slice: all the SMs, but at least one row block each
     p.cps = std::max(1, std::min(di.sms / p.splits, p.nrb));
     p.grid = p.splits * p.cps;
-    p.smem = gemv_mma_smem_bytes(M, p.TKC, p.warps, p.stages, sz, szw);
+    p.smem = gemv_mma_smem_bytes(M, p.TKC, p.stages, sz, szw);
     p.xbytes = gemv_mma_xblock_bytes(M, p.TKC);
-    // every CTA converts its own activations when that is at most a few
-    // warp-units (256 k of one row) per warp; else a prep kernel does it once
-    p.in_kernel_x = p.splits == 1 && (p.TKC / 256) * M <= 4 * p.warps;
+    // every CTA converts its own activations when that is at most 4 units
+    // (256 k of one row) per consumer warp; else a prep kernel does it once
+    p.in_kernel_x = p.splits == 1 && (p.TKC / 256) * M <= 4 * kMW;
     auto up = [](size_t v) { return (v + 255) / 256 * 256; };
     p.partial_off = p.in_kernel_x ? 0 : up(p.splits * p.xbytes);
     p.ws = p.partial_off + (p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * sizeof(float) : 0);
@@ -383,10 +384,14 @@ size_t gemv_workspace(int M, int N, int K, int transposed, int sms) {
     for (int szw = gemv_stream_sz_words(K); szw <= gemv_stream_sz_words(32); ++szw) {
         const StreamPlan p = plan_stream_szw(M, N, K, szw, di);
         if (p.ok) ws = std::max(ws, p.ws);
-        for (int sz : {kSzConst, kSzTma2d, kSzTma1d, kSzCopy}) {
-            const StreamPlan q = plan_mma(M, N, K, sz, szw, di);
-            if (q.ok) ws = std::max(ws, q.ws);
-        }
+    }
+    for (int sz : {kSzConst, kSzTma2d, kSzTma1d}) {
+        const StreamPlan q = plan_mma(M, N, K, sz, 0, di);
+        if (q.ok) ws = std::max(ws, q.ws);
+    }
+    for (int szw = gemv_mma_sz_words(K); szw <= gemv_mma_sz_words(128); ++szw) {
+        const StreamPlan q = plan_mma(M, N, K, kSzCopy, szw, di);
+        if (q.ok) ws = std::max(ws, q.ws);
     }
     return ws;
 }
@@ -419,7 +424,7 @@ w4_status launch_gemv_mma_k(const StreamPlan& p, const CUtensorMap& wm, const CU
     if (ensure_smem(reinterpret_cast<const void*>(fn), p.smem) != cudaSuccess) return W4_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid);
-    cfg.blockDim = dim3(p.warps * 32);
+    cfg.blockDim = dim3(kMThreads);
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -457,11 +462,11 @@ w4_status launch_gemv_mma(const StreamPlan& p, int M, const CUtensorMap& wm, con
     std::memset(&zm, 0, sizeof zm);
     bool ok = true;
     if (p.sz == kSzTma2d) {
-        ok = make_map_2d(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.G, kSR, 16, 0) &&
-             make_map_2d(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.G, kSR, 16, 0);
+        ok = make_map_2d(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.G, kMR, 16, 0) &&
+             make_map_2d(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.G, kMR, 16, 0);
     } else if (p.sz == kSzTma1d) {
-        ok = make_map_row(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, 8) &&
-             make_map_row(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, 8);
+        ok = make_map_row(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, kMR) &&
+             make_map_row(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, kMR);
     }
     if (!ok) return W4_ERR_CUDA;
     switch (M) {
@@ -480,7 +485,7 @@ w4_status run_gemv_stream(const StreamPlan& p, int M, int N, int K, const void* 
     uint8_t* xb = static_cast<uint8_t*>(ws);
     float* partial = p.splits > 1 ? reinterpret_cast<float*>(xb + p.partial_off) : nullptr;
     CUtensorMap map;
-    if (!make_map_2d(&map, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, kSR, kSBK / 8, 0))
+    if (!make_map_2d(&map, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, p.mma ? kMR : kSR, kSBK / 8, 0))
         return W4_ERR_CUDA;
     w4_status s = W4_OK;
     if (p.mma) {
@@ -506,7 +511,7 @@ w4_status run_gemv_stream(const StreamPlan& p, int M, int N, int K, const void* 
         a.sz_row = meta.sz_row;
         a.TKC = p.TKC;
         a.splits = p.splits;
-        a.nbs = p.nbs;
+        a.nks = p.nks;
         a.nrb = p.nrb;
         a.cps = p.cps;
         a.stages = p.stages;
@@ -568,7 +573,10 @@ w4_status run_gemv_fwd(const void* A, int M, int N, int K, const uint32_t* packe
     const DeviceInfo di = device_info(current_device());
     {
         StreamPlan sp;
-        if (mma_eligible(K, meta)) sp = plan_mma(M, N, K, mma_sz_kind(meta), gemv_stream_sz_words(meta.g), di);
+        if (mma_eligible(K, meta)) {
+            const int sz = mma_sz_kind(meta);
+            sp = plan_mma(M, N, K, sz, sz == kSzCopy ? gemv_mma_sz_words(meta.g) : 0, di);
+        }
         if (!sp.ok) sp = plan_stream(M, N, K, meta, di);
         if (sp.ok) return run_gemv_stream(sp, M, N, K, A, packed, S, Z, meta, bias, Y, ws, ws_bytes, st);
     }

@@ -75,7 +75,10 @@ GEMV_SHAPES = [
     (200, 3072, "global", 0),
     (300, 1056, "groupwise", 32),       # K not a multiple of the 256-k box
     (130, 520, "groupwise", 8),         # K % 32 != 0: plain kernel
-    (64, 9216, "groupwise", 256),       # split K for M = 4
+    (64, 9216, "groupwise", 256),       # activation prep kernel for M >= 2
+    (48, 20480, "groupwise", 128),      # K split into slices for M = 4
+    (40, 11008, "groupwise", 128),      # G % 8 != 0: scales and zeros by cp.async
+    (24, 6144, "groupwise", 384),       # group length not a power of two
 ]
 
 
