@@ -288,11 +288,12 @@ __global__ void __launch_bounds__(kMThreads, 1)
     if (warp == kMW) {
         // ------------------------------------------------------ producer
         int rb = rb_lo, ks = 0;
+        int s = 0;
+        uint32_t round = 0;                      // completed passes over the ring
         for (int it = 0; it < items; ++it) {
-            const int s = it % NS;
-            if (it >= NS) {
-                const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&empty[s], ((it / NS) - 1) & 1u,
-                                                                          abort_flag, kErrTimeoutEmpty));
+            if (round > 0) {
+                const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&empty[s], (round - 1) & 1u, abort_flag,
+                                                                          kErrTimeoutEmpty));
                 if (!ok) break;
             }
             uint8_t* sd = ring + s * SB;
@@ -336,6 +337,10 @@ __global__ void __launch_bounds__(kMThreads, 1)
                 ks = 0;
                 ++rb;
             }
+            if (++s == NS) {
+                s = 0;
+                ++round;
+            }
         }
     } else {
         // ------------------------------------------------------ consumers
@@ -373,9 +378,10 @@ __global__ void __launch_bounds__(kMThreads, 1)
         const float2* fcs = reinterpret_cast<const float2*>(xblk + static_cast<size_t>(ngran) * M * 256);
         float y0 = 0.f, y1 = 0.f;                // rows g and g + 8 of the row block, m = tig
         int rb = rb_lo, ks = 0, rbi = 0;
+        int s = 0;
+        uint32_t phase = 0;
         for (int it = 0; it < items; ++it) {
-            const int s = it % NS;
-            __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[s], (it / NS) & 1u, abort_flag, kErrTimeoutTmaFull));
+            __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[s], phase, abort_flag, kErrTimeoutTmaFull));
             const uint8_t* sb = ring + s * SB;
             const int gl = ks * (kMK / 128) + warp;               // granule within the slice
             const int kg = k_slice + gl * 128;                    // its first k
@@ -436,6 +442,10 @@ __global__ void __launch_bounds__(kMThreads, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
+            if (++s == NS) {
+                s = 0;
+                phase ^= 1u;
+            }
             if (++ks == a.nks) {
                 // row block done: the 16 warps' sums meet in shared memory and
                 // are added in a fixed order (warp pairs, then a shuffle tree)
