@@ -30,10 +30,10 @@
 // with xs = 2^(e - 140), e the granule's largest bf16 exponent, so y
 // accumulates s * sum_k x (q - z) for its two rows.
 //
-// Output.  At the end of a row block the sixteen warps' sums meet in shared
-// memory and are added in a fixed order (so results do not depend on
-// timing), then biased and rounded once, or written as fp32 partials when K
-// is split into slices.
+// Output.  At the end of a row block each consumer warp leaves its sums in
+// shared memory and moves on; a reducer warp adds the sixteen in a fixed
+// order (so results do not depend on timing), then biases and rounds once,
+// or writes fp32 partials when K is split into slices.
 #pragma once
 
 #include "gemv_stream.cuh"
@@ -44,7 +44,7 @@ constexpr int kMFrac = 6;          // fixed-point bits below the granule's leadi
 constexpr int kMR = 16;            // weight rows per stage (the mma's A rows)
 constexpr int kMK = 2048;          // k per stage
 constexpr int kMW = 16;            // consumer warps: one 128-k granule of each stage apiece
-constexpr int kMThreads = (kMW + 1) * 32;
+constexpr int kMThreads = (kMW + 2) * 32;  // + the producer warp and the reducer warp
 constexpr int kMWBytes = kMR * kMK / 2;    // 16 KB of packed weights per stage
 constexpr int kMRedStride = 68;            // floats per warp in the row-block reduction (64 + pad)
 
@@ -194,7 +194,7 @@ __host__ __device__ inline size_t gemv_mma_smem_bytes(int M, int TKC, int stages
     b += static_cast<size_t>(stages) * gemv_mma_stage_bytes(sz, szw);
     b += (gemv_mma_xblock_bytes(M, TKC) + 15) / 16 * 16;
     b += static_cast<size_t>(2) * kMW * kMRedStride * 4;               // row-block reduction, 2 buffers
-    b += static_cast<size_t>(stages) * 16 + 8 + 16;                    // barriers, abort flag
+    b += static_cast<size_t>(stages) * 16 + 32 + 8 + 16;               // barriers, abort flag
     return b;
 }
 // Scale / zero words per row and stage on the copy path: the groups a
@@ -249,7 +249,9 @@ __global__ void __launch_bounds__(kMThreads, 1)
     float* red = reinterpret_cast<float*>(xblk + ((xbytes + 15) & ~15u));   // [2][warp][kMRedStride]
     uint64_t* full = reinterpret_cast<uint64_t*>(red + 2 * kMW * kMRedStride);
     uint64_t* empty = full + NS;
-    uint64_t* xbar = empty + NS;
+    uint64_t* rfull = empty + NS;              // [2] a row block's 16 warp sums are in
+    uint64_t* rempty = rfull + 2;              // [2] the reducer is done with a buffer
+    uint64_t* xbar = rempty + 2;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(xbar + 1);
 
     if (tid == 0) {
@@ -258,6 +260,10 @@ __global__ void __launch_bounds__(kMThreads, 1)
             // bytes; the copy path adds one cp.async arrival per producer lane
             mbar_init(&full[i], SZ == kSzCopy ? 33 : 1);
             mbar_init(&empty[i], kMW);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&rfull[i], kMW);
+            mbar_init(&rempty[i], 1);
         }
         mbar_init(xbar, 1);
         *abort_flag = 0;
@@ -341,6 +347,39 @@ __global__ void __launch_bounds__(kMThreads, 1)
                 s = 0;
                 ++round;
             }
+        }
+    } else if (warp == kMW + 1) {
+        // ------------------------------------------------------ reducer
+        // adds the 16 consumer warps' sums of each row block in warp order
+        // (so results do not depend on timing), then biases and rounds once,
+        // or writes fp32 partials when K is split into slices
+        const int nrows = rb_hi - rb_lo;
+        for (int i = 0; i < nrows; ++i) {
+            const int b = i & 1;
+            if (!mbar_wait_bounded(&rfull[b], (i >> 1) & 1u, abort_flag, kErrTimeoutTmaFull)) break;
+            const float* rbuf = red + b * (kMW * kMRedStride);
+            const int rb = rb_lo + i;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int v = lane + 32 * h;            // output (row r, m)
+                const int r = v >> 2, m = v & 3;
+                const int src = ((r & 7) * 4 + m) * 2 + (r >> 3);
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < kMW; ++w) sum += rbuf[w * kMRedStride + src];
+                const int n = rb * kMR + r;
+                if (m < M && n < a.N) {
+                    if (a.splits == 1) {
+                        float o = sum;
+                        if (a.bias) o += bf16_bits_to_float(a.bias[n]);
+                        a.Y[static_cast<size_t>(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+                    } else {
+                        a.partial[(static_cast<size_t>(slice) * M + m) * a.N + n] = sum;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&rempty[b]);
         }
     } else {
         // ------------------------------------------------------ consumers
@@ -447,29 +486,17 @@ __global__ void __launch_bounds__(kMThreads, 1)
                 phase ^= 1u;
             }
             if (++ks == a.nks) {
-                // row block done: the 16 warps' sums meet in shared memory and
-                // are added in a fixed order (warp pairs, then a shuffle tree)
-                float* rbuf = red + (rbi & 1) * (kMW * kMRedStride);
+                // row block done: hand this warp's sums to the reducer (its
+                // buffer is free once the reducer finished the row block two
+                // before)
+                const int b = rbi & 1;
+                if (rbi >= 2)
+                    __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&rempty[b], ((rbi >> 1) - 1) & 1u, abort_flag,
+                                                              kErrTimeoutTmaFull));
+                float* rbuf = red + b * (kMW * kMRedStride);
                 reinterpret_cast<float2*>(rbuf + warp * kMRedStride)[lane] = make_float2(y0, y1);
-                named_barrier_sync(1, kMW * 32);
-                const int t = warp * 32 + lane;
-                const int v = t >> 3, j = t & 7;        // output (row r, m) and its pair of warps
-                const int r = v >> 2, m = v & 3;
-                const int src = ((r & 7) * 4 + m) * 2 + (r >> 3);
-                float sum = rbuf[(2 * j) * kMRedStride + src] + rbuf[(2 * j + 1) * kMRedStride + src];
-                sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
-                sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-                sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
-                const int n = rb * kMR + r;
-                if (j == 0 && m < M && n < a.N) {
-                    if (a.splits == 1) {
-                        float o = sum;
-                        if (a.bias) o += bf16_bits_to_float(a.bias[n]);
-                        a.Y[static_cast<size_t>(m) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
-                    } else {
-                        a.partial[(static_cast<size_t>(slice) * M + m) * a.N + n] = sum;
-                    }
-                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&rfull[b]);
                 y0 = 0.f;
                 y1 = 0.f;
                 ks = 0;
