@@ -59,8 +59,8 @@ __host__ __device__ inline size_t gemv_mma_xblock_bytes(int M, int TKC) {
     return static_cast<size_t>(TKC) / 128 * M * (256 + 8);
 }
 
-// Programmatic dependent launch: the prep kernel lets the GEMV start early,
-// and the GEMV waits for the prep kernel's results only where it needs them.
+// Programmatic dependent launch: a kernel lets its dependents start early;
+// a dependent waits for the kernels before it where it needs their results.
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
@@ -277,6 +277,14 @@ __global__ void __launch_bounds__(kMThreads, 1)
         }
     }
     __syncthreads();
+    // Programmatic dependent launch: the next kernel in the stream may start
+    // its own prologue as SMs free up.  This kernel itself was launched as a
+    // dependent of the work before it, so it touches no global memory until
+    // that work is complete -- except, after a prep kernel (which started
+    // only once everything before it was done), the weights, which no kernel
+    // in between writes.
+    pdl_launch_dependents();
+    if (a.xblocks == nullptr) pdl_wait();
 
     const int slice = blockIdx.x / a.cps, cta = blockIdx.x - (blockIdx.x / a.cps) * a.cps;
     const int rb_lo = static_cast<int>(static_cast<long long>(cta) * a.nrb / a.cps);

@@ -413,10 +413,11 @@ w4_status launch_gemv_stream(const StreamPlan& p, const CUtensorMap& map, const 
     return launch_gemv_stream_gk<M, kGroupsAny>(p, map, a, st);
 }
 
-// With a prep kernel just before it, the GEMV is launched as its
-// programmatic dependent: its prologue and first weight loads overlap the
-// prep kernel.  Without one it is an ordinary launch (it reads its inputs
-// from the start, so it must not begin before the work ahead of it ends).
+// The GEMV is always launched as a programmatic dependent of the work just
+// before it.  After its own prep kernel, its prologue and first weight
+// loads overlap the prep kernel; otherwise only its prologue overlaps the
+// previous kernel's tail, and it waits for that kernel before reading any
+// input.
 template <int M, int GK, int SZ>
 w4_status launch_gemv_mma_k(const StreamPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
                             const CUtensorMap& zm, const GemvMmaArgs& a, cudaStream_t st) {
@@ -431,7 +432,7 @@ w4_status launch_gemv_mma_k(const StreamPlan& p, const CUtensorMap& wm, const CU
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = p.in_kernel_x ? 0 : 1;
+    cfg.numAttrs = 1;
     cudaLaunchKernelEx(&cfg, fn, wm, sm, zm, a);
     return launch_status();
 }
