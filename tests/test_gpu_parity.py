@@ -79,6 +79,7 @@ GEMV_SHAPES = [
     (48, 20480, "groupwise", 128),      # K split into slices for M = 4
     (40, 11008, "groupwise", 128),      # G % 8 != 0: scales and zeros by cp.async
     (24, 6144, "groupwise", 384),       # group length not a power of two
+    (2600, 2048, "groupwise", 128),     # CTAs with 2 and 3 eight-row units: full and half blocks
 ]
 
 
