@@ -342,8 +342,15 @@ __global__ void __launch_bounds__(kMThreads, 1)
                 // so that it does not queue behind the whole ring
                 pdl_wait();
                 if (lane == 0) {
+                    // every CTA of the slice copies the same block: in 8
+                    // pieces, each CTA starting at a different one
                     mbar_arrive_expect_tx(xbar, xbytes);
-                    bulk_load_1d(xblk, a.xblocks + static_cast<size_t>(slice) * xbytes, xbytes, xbar);
+                    const uint8_t* src = a.xblocks + static_cast<size_t>(slice) * xbytes;
+                    const uint32_t piece = (xbytes / 8 + 15) & ~15u;
+                    for (int q = 0; q < 8; ++q) {
+                        const uint32_t o = ((q + blockIdx.x) & 7) * piece;
+                        if (o < xbytes) bulk_load_1d(xblk + o, src + o, min(piece, xbytes - o), xbar);
+                    }
                 }
                 __syncwarp();
             }
@@ -393,20 +400,29 @@ __global__ void __launch_bounds__(kMThreads, 1)
         // ------------------------------------------------------ consumers
         if (a.xblocks == nullptr) {
             // this warp's activation units (at most 4: the planner's limit)
-            // are loaded, converted and stored while the ring fills
+            // are loaded, converted and stored while the ring fills.  Every
+            // CTA reads all of X; each starts at a different unit, so that
+            // the CTAs do not all queue on the same L2 lines at once.
             constexpr int kMaxUnits = 4;
             const int nunits = (a.TKC / 256) * M;
+            const int rot = static_cast<int>((static_cast<unsigned>(blockIdx.x) * 7u) % static_cast<unsigned>(nunits));
             uint4 raw[kMaxUnits];
 #pragma unroll
             for (int i = 0; i < kMaxUnits; ++i) {
-                const int u = warp + i * kMW;
+                int u = warp + i * kMW;
                 raw[i] = make_uint4(0u, 0u, 0u, 0u);
-                if (u < nunits) raw[i] = xfrag_load(a.X, a.K, k_slice + (u / M) * 256, u - (u / M) * M, lane);
+                if (u < nunits) {
+                    u = u + rot < nunits ? u + rot : u + rot - nunits;
+                    raw[i] = xfrag_load(a.X, a.K, k_slice + (u / M) * 256, u - (u / M) * M, lane);
+                }
             }
 #pragma unroll
             for (int i = 0; i < kMaxUnits; ++i) {
-                const int u = warp + i * kMW;
-                if (u < nunits) xfrag_store(raw[i], M, ngran, u / M, u - (u / M) * M, lane, xblk);
+                int u = warp + i * kMW;
+                if (u < nunits) {
+                    u = u + rot < nunits ? u + rot : u + rot - nunits;
+                    xfrag_store(raw[i], M, ngran, u / M, u - (u / M) * M, lane, xblk);
+                }
             }
             named_barrier_sync(1, kMW * 32);
         } else if (items > 0) {
