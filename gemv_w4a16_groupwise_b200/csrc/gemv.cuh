@@ -52,20 +52,36 @@ __device__ __forceinline__ float half_to_float_ldg(const __half* p) {
 }
 
 
-// Finalize a split reduction: out[m, l] = bf16(sum_s partial[s, m, l] + bias[l]),
-// slices added in ascending order.
+// Finalize a split reduction: out[m, l] = bf16(sum_s partial[s, m, l] + bias[l]).
+// A block takes 64 consecutive outputs; thread (q, o) adds slices q, q + 4,
+// q + 8, ... of output o in ascending order (independent loads, so many are
+// in flight), and the four partial sums are then added in the order
+// q = 0, 1, 2, 3: a fixed order, so the result does not depend on timing.
+constexpr int kFinOut = 64;
 __global__ void __launch_bounds__(256) splits_finalize_kernel(const float* __restrict__ partial,
                                                               int splits, int M, int L,
                                                               const uint16_t* __restrict__ bias,
                                                               uint16_t* __restrict__ out) {
+    __shared__ float red[4][kFinOut];
     const long long total = static_cast<long long>(M) * L;
-    for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-         idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int o = threadIdx.x % kFinOut, q = threadIdx.x / kFinOut;
+    for (long long b0 = static_cast<long long>(blockIdx.x) * kFinOut; b0 < total;
+         b0 += static_cast<long long>(gridDim.x) * kFinOut) {
+        const long long idx = b0 + o;
         float s = 0.0f;
-        for (int sp = 0; sp < splits; ++sp) s += partial[static_cast<long long>(sp) * total + idx];
-        const int l = static_cast<int>(idx % L);
-        if (bias) s += bf16_bits_to_float(bias[l]);
-        out[idx] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+        if (idx < total) {
+#pragma unroll 4
+            for (int sp = q; sp < splits; sp += 4) s += __ldg(partial + static_cast<long long>(sp) * total + idx);
+        }
+        red[q][o] = s;
+        __syncthreads();
+        if (q == 0 && idx < total) {
+            float v = ((red[0][o] + red[1][o]) + red[2][o]) + red[3][o];
+            const int l = static_cast<int>(idx % L);
+            if (bias) v += bf16_bits_to_float(bias[l]);
+            out[idx] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        }
+        __syncthreads();
     }
 }
 

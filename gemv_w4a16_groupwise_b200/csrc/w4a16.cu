@@ -560,7 +560,7 @@ w4_status run_gemv_stream(const StreamPlan& p, int M, int N, int K, const void* 
     if (p.splits > 1) {
         const DeviceInfo di = device_info(current_device());
         const long long total = static_cast<long long>(M) * N;
-        const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, di.sms * 8));
+        const int blocks = static_cast<int>(std::min<long long>((total + kFinOut - 1) / kFinOut, di.sms * 16));
         splits_finalize_kernel<<<blocks, 256, 0, st>>>(partial, p.splits, M, N, static_cast<const uint16_t*>(bias),
                                                         static_cast<uint16_t*>(Y));
         return launch_status();
@@ -669,7 +669,7 @@ w4_status run_gemv_t_stream(const TStreamPlan& p, int M, int N, int K, const voi
     if (p.splits > 1) {
         const DeviceInfo di = device_info(current_device());
         const long long total = static_cast<long long>(M) * K;
-        const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, di.sms * 8));
+        const int blocks = static_cast<int>(std::min<long long>((total + kFinOut - 1) / kFinOut, di.sms * 16));
         splits_finalize_kernel<<<blocks, 256, 0, st>>>(a.partial, p.splits, M, K, a.bias, a.dX);
         return launch_status();
     }
@@ -713,7 +713,7 @@ w4_status run_gemv_t(const void* A, int M, int N, int K, const uint32_t* packed,
     if (s != W4_OK) return s;
     if (p.splits > 1) {
         const long long total = static_cast<long long>(M) * K;
-        const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, di.sms * 8));
+        const int blocks = static_cast<int>(std::min<long long>((total + kFinOut - 1) / kFinOut, di.sms * 16));
         splits_finalize_kernel<<<blocks, 256, 0, st>>>(a.partial, p.splits, M, K, a.bias, a.dX);
         return launch_status();
     }
