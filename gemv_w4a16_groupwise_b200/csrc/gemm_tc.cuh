@@ -11,14 +11,19 @@
 // added to the fp32 accumulator before the single bf16 rounding (vLLM
 // "Adding bias epilogue support for cutlass_scaled_mm").
 //
-// Warp roles (576 threads, one CTA per SM):
+// Persistent: one CTA per SM walks tiles blockIdx.x, + gridDim.x, ...; the
+// stage ring runs on across tile boundaries and the fp32 accumulator is
+// double-buffered in TMEM, so one tile's epilogue overlaps the next tile's
+// main loop.  Warp roles (704 threads):
 //   warp 0       TMA producer: packed weight tile + activation tile per stage
 //   warp 1       TMEM allocator; lane 0 issues tcgen05.mma and commits
 //   warps 2..17  dequantize packed codes into the bf16 A tile of a stage
-//                (128-byte swizzled UMMA layout), then run the epilogue.
-//                Two groups of 8 warps take alternate stages, so two stages
-//                are being dequantized at any time and the tensor pipe is not
-//                left waiting on one stage's dequantization latency.
+//                (128-byte swizzled UMMA layout).  Two groups of 8 warps take
+//                alternate stages, so two stages are being dequantized at any
+//                time and the tensor pipe is not left waiting on one stage's
+//                dequantization latency.
+//   warps 18..21 epilogue: TMEM -> registers, fp32 bias, one bf16 rounding,
+//                store (warp w reads the TMEM lanes 32 (w % 4) .. + 31).
 // Every mbarrier wait is bounded; a wait that runs out records the reason in
 // the device error word and the CTA unwinds without hanging.
 //
@@ -35,7 +40,8 @@
 namespace w4 {
 
 constexpr int kTcDeqGroups = 2;                      // dequantizing warp groups (8 warps each)
-constexpr int kTcThreads = 64 + kTcDeqGroups * 256;
+constexpr int kTcEpiWarps = 4;
+constexpr int kTcThreads = 64 + kTcDeqGroups * 256 + kTcEpiWarps * 32;
 constexpr int kTcBM = 128;     // MMA M (weight rows per tile)
 constexpr int kTcBK = 64;      // reduction depth per pipeline stage
 constexpr int kTcABytes = kTcBM * kTcBK * 2;   // 16 KB dequantized tile
@@ -156,7 +162,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                    const TcArgs a) {
     static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 256, "BN");
     constexpr int kStageBytes = tc_stage_bytes(BN);
-    constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+    constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;          // one accumulator buffer
+    constexpr uint32_t kTmemCols = 2 * kAccCols;              // two, a power of two >= 64
     constexpr uint32_t kTxBytes = kTcPBytes + BN * 128;
     constexpr uint32_t kIdesc = umma_idesc_bf16(BN, TR);
 
@@ -166,16 +173,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t* tma_full = reinterpret_cast<uint64_t*>(base + NS * kStageBytes);
     uint64_t* deq_full = tma_full + NS;
     uint64_t* empty = deq_full + NS;
-    uint64_t* acc_full = empty + NS;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+    uint64_t* acc_full = empty + NS;          // [2] an accumulator buffer holds a finished tile
+    uint64_t* acc_empty = acc_full + 2;       // [2] the epilogue has drained a buffer
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * BN;          // first token of the tile
-    const int r0 = blockIdx.y * kTcBM;       // first output row (n, or k when transposed)
     const int L_out = TR ? a.K : a.N;        // output row length
     const int red_len = TR ? a.N : a.K;      // reduction length
     const int num_kb = (red_len + kTcBK - 1) / kTcBK;
+    const int tiles_m = (a.M + BN - 1) / BN;
+    const int tiles = tiles_m * ((L_out + kTcBM - 1) / kTcBM);
+    // this CTA's tiles: blockIdx.x, + gridDim.x, ...; tile t covers tokens
+    // (t % tiles_m) * BN .. and output rows (t / tiles_m) * 128 ..
+    const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    auto tile_of = [&](int i) { return blockIdx.x + i * gridDim.x; };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -183,7 +195,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(&deq_full[s], 8);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_full, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], kTcEpiWarps);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -204,47 +219,72 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
             tma_prefetch_desc(&pmap);
             tma_prefetch_desc(&bmap);
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const int s = kb % NS;
-                const uint32_t use = static_cast<uint32_t>(kb / NS);
-                if (use > 0 && !mbar_wait_bounded(&empty[s], (use - 1) & 1u, abort_flag, kErrTimeoutEmpty))
-                    break;
-                uint8_t* st = base + s * kStageBytes;
-                mbar_arrive_expect_tx(&tma_full[s], kTxBytes);
-                if (TR)
-                    tma_load_2d(st + kTcABytes + BN * 128, &pmap, r0 / 8, kb * kTcBK, &tma_full[s]);
-                else
-                    tma_load_2d(st + kTcABytes + BN * 128, &pmap, kb * (kTcBK / 8), r0, &tma_full[s]);
-                tma_load_2d(st + kTcABytes, &bmap, kb * kTcBK, m0, &tma_full[s]);
+            int s = 0;
+            uint32_t round = 0;
+            bool ok = true;
+            for (int i = 0; i < my_tiles && ok; ++i) {
+                const int t = tile_of(i);
+                const int m0 = (t % tiles_m) * BN, r0 = (t / tiles_m) * kTcBM;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (round > 0 && !mbar_wait_bounded(&empty[s], (round - 1) & 1u, abort_flag, kErrTimeoutEmpty)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = base + s * kStageBytes;
+                    mbar_arrive_expect_tx(&tma_full[s], kTxBytes);
+                    if (TR)
+                        tma_load_2d(st + kTcABytes + BN * 128, &pmap, r0 / 8, kb * kTcBK, &tma_full[s]);
+                    else
+                        tma_load_2d(st + kTcABytes + BN * 128, &pmap, kb * (kTcBK / 8), r0, &tma_full[s]);
+                    tma_load_2d(st + kTcABytes, &bmap, kb * kTcBK, m0, &tma_full[s]);
+                    if (++s == NS) {
+                        s = 0;
+                        ++round;
+                    }
+                }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             bool ok = true;
-            for (int kb = 0; kb < num_kb && ok; ++kb) {
-                const int s = kb % NS;
-                const uint32_t par = static_cast<uint32_t>(kb / NS) & 1u;
-                ok = mbar_wait_bounded(&tma_full[s], par, abort_flag, kErrTimeoutTmaFull) &&
-                     mbar_wait_bounded(&deq_full[s], par, abort_flag, kErrTimeoutDequant);
+            int s = 0;
+            uint32_t phase = 0;
+            for (int i = 0; i < my_tiles && ok; ++i) {
+                const int buf = i & 1;
+                // the epilogue has drained this buffer (tile i - 2)
+                if (i >= 2) ok = mbar_wait_bounded(&acc_empty[buf], ((i >> 1) - 1) & 1u, abort_flag, kErrTimeoutAccum);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t a_addr = smem_u32(base + s * kStageBytes);
-                const uint32_t b_addr = a_addr + kTcABytes;
+                const uint32_t acc = tmem_d + static_cast<uint32_t>(buf) * kAccCols;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    ok = mbar_wait_bounded(&tma_full[s], phase, abort_flag, kErrTimeoutTmaFull) &&
+                         mbar_wait_bounded(&deq_full[s], phase, abort_flag, kErrTimeoutDequant);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(base + s * kStageBytes);
+                    const uint32_t b_addr = a_addr + kTcABytes;
 #pragma unroll
-                for (int i = 0; i < kTcBK / 16; ++i) {
-                    const uint64_t adesc = TR ? umma_desc_sw128(a_addr + i * 2048, 8192, 1024)
-                                              : umma_desc_sw128(a_addr + i * 32, 16, 1024);
-                    const uint64_t bdesc = umma_desc_sw128(b_addr + i * 32, 16, 1024);
-                    umma_bf16(tmem_d, adesc, bdesc, kIdesc, (kb | i) != 0 ? 1u : 0u);
+                    for (int j = 0; j < kTcBK / 16; ++j) {
+                        const uint64_t adesc = TR ? umma_desc_sw128(a_addr + j * 2048, 8192, 1024)
+                                                  : umma_desc_sw128(a_addr + j * 32, 16, 1024);
+                        const uint64_t bdesc = umma_desc_sw128(b_addr + j * 32, 16, 1024);
+                        umma_bf16(acc, adesc, bdesc, kIdesc, (kb | j) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(&empty[s]);
+                    if (++s == NS) {
+                        s = 0;
+                        phase ^= 1u;
+                    }
                 }
-                umma_commit(&empty[s]);
+                umma_commit(&acc_full[buf]);   // also tracks any MMA issued before an abort
             }
-            umma_commit(acc_full);  // also tracks any MMA issued before an abort
         }
-    } else {
+    } else if (warp < 2 + 8 * kTcDeqGroups) {
         // ------------------------------------------------ dequantize
-        const int grp_id = (threadIdx.x - 64) >> 8;           // this warp's group: stages kb = grp_id mod 2
+        // Stages are numbered across the CTA's tiles (c = i * num_kb + kb);
+        // group grp_id takes c = grp_id, grp_id + 2, ...
+        const int grp_id = (threadIdx.x - 64) >> 8;
         const int t = (threadIdx.x - 64) & 255;               // 0 .. 255 within the group
         // forward: row n = r0 + t % 128, words 4h .. 4h+3 of the 8 in a k-block
         // transposed: row n = kb * 64 + t % 64, words 4q .. 4q+3 of the 16 of a k-tile
@@ -264,65 +304,50 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 off[j] = prow * 128 + ((c ^ (prow & 7)) << 4);
             }
         }
-        // Scale / zero of block kb, fetched one block ahead.  With g a
-        // multiple of 32 the thread's 4 words share one group: forward, the
-        // group moves by at most 64 / g per block and is tracked by
-        // subtraction; transposed, it is fixed and only the row moves.
+        int gshift = -1;                                  // log2(g) when g is a power of two
+        if ((a.g & (a.g - 1)) == 0) gshift = __ffs(a.g) - 1;
+        auto group_of = [&](int k) { return min(gshift >= 0 ? (k >> gshift) : k / a.g, a.G - 1); };
+        // Scale / zero of one stage (tile i, block kb); with g a multiple of
+        // 32 the thread's 4 words share one group.
         constexpr int NG = PWG ? 4 : 1;
-        const int kw_t = TR ? r0 / 8 + 4 * pquad : 4 * pquad;   // forward: + kb * 8
-        int grp_f = 0, rem_f = 0;                               // forward: (8 kw0) = grp_f * g + rem_f
-        if (!PWG && !TR) {
-            grp_f = (8 * kw_t) / a.g;
-            rem_f = 8 * kw_t - grp_f * a.g;
-        }
-        const int grp_t = (!PWG && TR) ? min((8 * kw_t) / a.g, a.G - 1) : 0;
-        auto load_sz = [&](int kb, float (&sv)[NG], float (&zv)[NG]) {
+        auto load_sz = [&](int i, int kb, float (&sv)[NG], float (&zv)[NG]) {
+            const int r0 = (tile_of(i) / tiles_m) * kTcBM;
             const int n = TR ? kb * kTcBK + prow : r0 + prow;
             const int nc = min(n, a.N - 1);
             const __half* sp = a.S + static_cast<size_t>(nc) * a.sz_row;
             const __half* zp = a.Z + static_cast<size_t>(nc) * a.sz_row;
-            if (PWG) {
-                const int kw0 = TR ? kw_t : kb * (kTcBK / 8) + kw_t;
+            const int kw0 = TR ? r0 / 8 + 4 * pquad : kb * (kTcBK / 8) + 4 * pquad;
 #pragma unroll
-                for (int j = 0; j < NG; ++j) {
-                    const int grp = min((8 * (kw0 + j)) / a.g, a.G - 1);
-                    sv[j] = __half2float(__ldg(sp + grp));
-                    zv[j] = __half2float(__ldg(zp + grp));
-                }
-            } else {
-                const int grp = TR ? grp_t : min(grp_f, a.G - 1);
-                sv[0] = __half2float(__ldg(sp + grp));
-                zv[0] = __half2float(__ldg(zp + grp));
+            for (int j = 0; j < NG; ++j) {
+                const int grp = group_of(8 * (kw0 + j));
+                sv[j] = __half2float(__ldg(sp + grp));
+                zv[j] = __half2float(__ldg(zp + grp));
             }
         };
-        auto next_group = [&]() {   // forward, g a multiple of 32: advance this group's stride of k-blocks
-            if (!PWG && !TR) {
-                rem_f += kTcBK * kTcDeqGroups;
-                while (rem_f >= a.g) {
-                    rem_f -= a.g;
-                    ++grp_f;
-                }
-            }
-        };
-        if (!PWG && !TR) {   // start at this group's first block
-            rem_f += kTcBK * grp_id;
-            while (rem_f >= a.g) {
-                rem_f -= a.g;
-                ++grp_f;
-            }
+        const int total = my_tiles * num_kb;
+        // this group's first stage, and its ring slot and phase
+        int ci = 0, ckb = grp_id;
+        while (ckb >= num_kb && ci < my_tiles) {
+            ckb -= num_kb;
+            ++ci;
         }
+        int s = grp_id % NS;
+        uint32_t phase = static_cast<uint32_t>(grp_id / NS) & 1u;
         float sv[NG], zv[NG], svn[NG], zvn[NG];
-        if (grp_id < num_kb) load_sz(grp_id, sv, zv);
-        next_group();
-        for (int kb = grp_id; kb < num_kb; kb += kTcDeqGroups) {
-            const int s = kb % NS;
-            const uint32_t par = static_cast<uint32_t>(kb / NS) & 1u;
-            if (kb + kTcDeqGroups < num_kb) load_sz(kb + kTcDeqGroups, svn, zvn);
-            next_group();
-            const int n = TR ? kb * kTcBK + prow : r0 + prow;
-            const int kw0 = TR ? kw_t : kb * (kTcBK / 8) + kw_t;
+        if (grp_id < total) load_sz(ci, ckb, sv, zv);
+        for (int c = grp_id; c < total; c += kTcDeqGroups) {
+            // the next stage of this group, whose scales are fetched now
+            int ni = ci, nkb = ckb + kTcDeqGroups;
+            while (nkb >= num_kb) {
+                nkb -= num_kb;
+                ++ni;
+            }
+            if (c + kTcDeqGroups < total) load_sz(ni, nkb, svn, zvn);
+            const int r0 = (tile_of(ci) / tiles_m) * kTcBM;
+            const int n = TR ? ckb * kTcBK + prow : r0 + prow;
+            const int kw0 = TR ? r0 / 8 + 4 * pquad : ckb * (kTcBK / 8) + 4 * pquad;
             const bool row_ok = n < a.N;
-            const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&tma_full[s], par, abort_flag,
+            const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&tma_full[s], phase, abort_flag,
                                                                       kErrTimeoutTmaFull));
             if (ok) {
                 uint8_t* st = base + s * kStageBytes;
@@ -347,25 +372,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 sv[j] = svn[j];
                 zv[j] = zvn[j];
             }
+            ci = ni;
+            ckb = nkb;
+            s += kTcDeqGroups;
+            while (s >= NS) {
+                s -= NS;
+                phase ^= 1u;
+            }
         }
-
+    } else {
         // ------------------------------------------------ epilogue
-        const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(acc_full, 0u, abort_flag,
-                                                                  kErrTimeoutAccum));
-        if (ok && !*abort_flag) {
+        const int q = warp & 3;                 // TMEM lanes 32 q .. 32 q + 31
+        for (int i = 0; i < my_tiles; ++i) {
+            const int buf = i & 1;
+            const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1u, abort_flag,
+                                                                      kErrTimeoutAccum));
+            if (!ok || *abort_flag) break;
             tc_fence_after();
-            // warp w reads TMEM lanes 32 (w % 4) .. + 31; the 16 epilogue
-            // warps split the BN columns into up to 4 parts of >= 8
-            const int q = warp & 3;
-            constexpr int kParts = BN / 8 < 4 ? BN / 8 : 4;
-            const int part = (warp - 2) >> 2;
+            const int t = tile_of(i);
+            const int m0 = (t % tiles_m) * BN, r0 = (t / tiles_m) * kTcBM;
             const int row = r0 + 32 * q + lane;
             const bool rv = row < L_out;
             const float bias_f = (a.bias && rv) ? bf16_bits_to_float(a.bias[row]) : 0.0f;
+            const uint32_t acc = tmem_d + static_cast<uint32_t>(buf) * kAccCols + (static_cast<uint32_t>(32 * q) << 16);
 #pragma unroll 1
-            for (int c0 = part * (BN / kParts); part < kParts && c0 < (part + 1) * (BN / kParts); c0 += 8) {
+            for (int c0 = 0; c0 < BN; c0 += 8) {
                 uint32_t r[8];
-                tmem_ld_x8(tmem_d + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0), r);
+                tmem_ld_x8(acc + static_cast<uint32_t>(c0), r);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int m = m0 + c0 + e;
@@ -374,6 +407,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[e]) + bias_f));
                 }
             }
+            // this warp's reads of the buffer are complete
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
     }
 
@@ -389,4 +426,3 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 }  // namespace w4
-

@@ -792,7 +792,7 @@ w4_status run_gemm_tc(const TcProblem& p, cudaStream_t st) {
     int stages = static_cast<int>((static_cast<size_t>(di.max_smem_optin) - fixed - 64) / (stage + 24));
     stages = std::min(stages, 8);
     if (stages < 2) return W4_ERR_UNSUPPORTED;
-    const size_t smem = fixed + static_cast<size_t>(stages) * stage + static_cast<size_t>(3 * stages + 1) * 8 + 16;
+    const size_t smem = fixed + static_cast<size_t>(stages) * stage + static_cast<size_t>(3 * stages + 4) * 8 + 16;
     const bool tr = p.transposed != 0;
     CUtensorMap pm, bm;
     // packed weights [N, K/8] uint32: box 8 words x 128 rows (forward) or
@@ -815,8 +815,10 @@ w4_status run_gemm_tc(const TcProblem& p, cudaStream_t st) {
     a.sz_row = p.sz_row;
     a.stages = stages;
     const int L_out = tr ? p.K : p.N;
-    const dim3 grid((p.M + BN - 1) / BN, (L_out + kTcBM - 1) / kTcBM);
-    if (grid.y > 65535) return W4_ERR_UNSUPPORTED;
+    // persistent: one CTA per SM (or per tile, when there are fewer tiles)
+    const long long tiles = static_cast<long long>((p.M + BN - 1) / BN) * ((L_out + kTcBM - 1) / kTcBM);
+    if (tiles > (1ll << 30)) return W4_ERR_UNSUPPORTED;
+    const dim3 grid(static_cast<unsigned>(std::min<long long>(tiles, di.sms)));
     const bool pwg = (p.g % 32) != 0;
     if (tr) return pwg ? launch_tc_bn<true, true>(BN, pm, bm, a, grid, smem, st)
                        : launch_tc_bn<true, false>(BN, pm, bm, a, grid, smem, st);
