@@ -310,8 +310,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // Scale / zero of one stage (tile i, block kb); with g a multiple of
         // 32 the thread's 4 words share one group.
         constexpr int NG = PWG ? 4 : 1;
-        auto load_sz = [&](int i, int kb, float (&sv)[NG], float (&zv)[NG]) {
-            const int r0 = (tile_of(i) / tiles_m) * kTcBM;
+        auto tile_r0 = [&](int i) { return (tile_of(i) / tiles_m) * kTcBM; };
+        auto load_sz = [&](int r0, int kb, float (&sv)[NG], float (&zv)[NG]) {
             const int n = TR ? kb * kTcBK + prow : r0 + prow;
             const int nc = min(n, a.N - 1);
             const __half* sp = a.S + static_cast<size_t>(nc) * a.sz_row;
@@ -334,7 +334,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int s = grp_id % NS;
         uint32_t phase = static_cast<uint32_t>(grp_id / NS) & 1u;
         float sv[NG], zv[NG], svn[NG], zvn[NG];
-        if (grp_id < total) load_sz(ci, ckb, sv, zv);
+        int cr0 = grp_id < total ? tile_r0(ci) : 0;          // output row offset of the current tile
+        if (grp_id < total) load_sz(cr0, ckb, sv, zv);
         for (int c = grp_id; c < total; c += kTcDeqGroups) {
             // the next stage of this group, whose scales are fetched now
             int ni = ci, nkb = ckb + kTcDeqGroups;
@@ -342,8 +343,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 nkb -= num_kb;
                 ++ni;
             }
-            if (c + kTcDeqGroups < total) load_sz(ni, nkb, svn, zvn);
-            const int r0 = (tile_of(ci) / tiles_m) * kTcBM;
+            const int nr0 = (ni != ci && c + kTcDeqGroups < total) ? tile_r0(ni) : cr0;
+            if (c + kTcDeqGroups < total) load_sz(nr0, nkb, svn, zvn);
+            const int r0 = cr0;
             const int n = TR ? ckb * kTcBK + prow : r0 + prow;
             const int kw0 = TR ? r0 / 8 + 4 * pquad : ckb * (kTcBK / 8) + 4 * pquad;
             const bool row_ok = n < a.N;
@@ -374,6 +376,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             ci = ni;
             ckb = nkb;
+            cr0 = nr0;
             s += kTcDeqGroups;
             while (s >= NS) {
                 s -= NS;
@@ -395,17 +398,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const bool rv = row < L_out;
             const float bias_f = (a.bias && rv) ? bf16_bits_to_float(a.bias[row]) : 0.0f;
             const uint32_t acc = tmem_d + static_cast<uint32_t>(buf) * kAccCols + (static_cast<uint32_t>(32 * q) << 16);
+            // lanes pair up: for token column c0 + e the even lane of a pair
+            // stores rows (row, row + 1) when e is even and the odd lane when
+            // e is odd, as one 4-byte bf16x2; with L_out odd such a pair
+            // would be misaligned, so every lane stores its own row instead
+            const bool odd = (lane & 1) != 0;
+            const int prow = row - (odd ? 1 : 0);            // first row of the pair
+            const bool pv = prow < L_out;
+            if (L_out & 1) {
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 8) {
+                    uint32_t r[8];
+                    tmem_ld_x8(acc + static_cast<uint32_t>(c0), r);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int m = m0 + c0 + e;
+                        if (rv && m < a.M)
+                            a.Y[static_cast<size_t>(m) * L_out + row] =
+                                __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[e]) + bias_f));
+                    }
+                }
+            } else {
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 8) {
                 uint32_t r[8];
                 tmem_ld_x8(acc + static_cast<uint32_t>(c0), r);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
+                    const float v = __uint_as_float(r[e]) + bias_f;
+                    const float o = __shfl_xor_sync(0xFFFFFFFFu, v, 1);
                     const int m = m0 + c0 + e;
-                    if (rv && m < a.M)
-                        a.Y[static_cast<size_t>(m) * L_out + row] =
-                            __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[e]) + bias_f));
+                    if (((e & 1) != 0) == odd && pv && m < a.M) {
+                        const float lo = odd ? o : v, hi = odd ? v : o;
+                        *reinterpret_cast<uint32_t*>(a.Y + static_cast<size_t>(m) * L_out + prow) =
+                            bf162_bits(__floats2bfloat162_rn(lo, hi));
+                    }
                 }
+            }
             }
             // this warp's reads of the buffer are complete
             tc_fence_before();

@@ -122,6 +122,15 @@ def test_gemm_parity(cuda_device, M, N, K, mode, g, transposed):
     assert_close(y, ref, f"gemm M={M} N={N} K={K} {mode} g={g} t={transposed}")
 
 
+@pytest.mark.parametrize("M", [5, 40, 300])
+def test_gemm_odd_output_length(cuda_device, M):
+    """An odd number of output rows: the epilogue stores single bf16 values."""
+    N, K, mode, g = 257, 512, "groupwise", 64
+    y, ref = run_matmul("w4a16_gemm", M, N, K, mode, g, False, bias=True,
+                        seed=synth.config_seed("gemm_odd", M, N, K), dev=cuda_device)
+    assert_close(y, ref, f"gemm odd N M={M}")
+
+
 @pytest.mark.parametrize("M", [4, 64, 512])
 @pytest.mark.parametrize("transposed", [False, True])
 def test_gemm_bias(cuda_device, M, transposed):
