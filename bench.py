@@ -275,6 +275,9 @@ def measure_rows(torch, w4, dev, peaks, stream):
         ts = []
         for _ in range(reps):
             flush_l2(torch, flush)
+            # keep the GPU busy (no memory traffic) while the host enqueues
+            # the call, so the events bracket device time only
+            torch.cuda._sleep(1_000_000)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)

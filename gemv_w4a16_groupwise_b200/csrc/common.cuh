@@ -28,6 +28,12 @@ __device__ __forceinline__ void record_error(unsigned int code) {
     atomicCAS(&g_error_word, 0u, code);
 }
 
+// Programmatic dependent launch: a kernel lets its dependents start early;
+// a dependent waits for the kernels before it where it needs their results.
+// Both are no-ops in a kernel launched without the programmatic attribute.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
     return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }

@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(256) splits_finalize_kernel(const float* __res
                                                               int splits, int M, int L,
                                                               const uint16_t* __restrict__ bias,
                                                               uint16_t* __restrict__ out) {
+    pdl_wait();   // when launched as a programmatic dependent of the split kernel
     __shared__ float red[4][kFinOut];
     const long long total = static_cast<long long>(M) * L;
     const int o = threadIdx.x % kFinOut, q = threadIdx.x / kFinOut;
@@ -80,6 +81,68 @@ __global__ void __launch_bounds__(256) splits_finalize_kernel(const float* __res
             const int l = static_cast<int>(idx % L);
             if (bias) v += bf16_bits_to_float(bias[l]);
             out[idx] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        }
+        __syncthreads();
+    }
+}
+
+// The same sum for L a multiple of 4, four outputs per thread: a block
+// takes 64 consecutive outputs (16 float4 columns); thread (q, c) adds
+// slices q, q + 16, q + 32, ... of column c in ascending order.  Its loads
+// go out together, eight at a time (indices past the last slice are clamped
+// to it, so every load is unconditional, and those values are dropped); the
+// sixteen partial sums are then added in the order q = 0 .. 15.
+constexpr int kFin4Cols = 16;
+constexpr int kFin4Q = 16;
+__global__ void __launch_bounds__(256) splits_finalize_vec4_kernel(const float* __restrict__ partial,
+                                                                   int splits, int M, int L,
+                                                                   const uint16_t* __restrict__ bias,
+                                                                   uint16_t* __restrict__ out) {
+    pdl_wait();   // when launched as a programmatic dependent of the split kernel
+    __shared__ float4 red[kFin4Q][kFin4Cols];
+    const long long total4 = static_cast<long long>(M) * L / 4;
+    const int c = threadIdx.x % kFin4Cols, q = threadIdx.x / kFin4Cols;
+    const float4* p4 = reinterpret_cast<const float4*>(partial);
+    for (long long b0 = static_cast<long long>(blockIdx.x) * kFin4Cols; b0 < total4;
+         b0 += static_cast<long long>(gridDim.x) * kFin4Cols) {
+        const long long idx = min(b0 + c, total4 - 1);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp0 = q; sp0 < splits; sp0 += kFin4Q * 8) {
+            float4 v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                v[j] = __ldg(p4 + static_cast<long long>(min(sp0 + kFin4Q * j, splits - 1)) * total4 + idx);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (sp0 + kFin4Q * j < splits) {
+                    acc.x += v[j].x;
+                    acc.y += v[j].y;
+                    acc.z += v[j].z;
+                    acc.w += v[j].w;
+                }
+        }
+        red[q][c] = acc;
+        __syncthreads();
+        if (q == 0 && b0 + c < total4) {
+            float r[4] = {red[0][c].x, red[0][c].y, red[0][c].z, red[0][c].w};
+#pragma unroll
+            for (int i = 1; i < kFin4Q; ++i) {
+                r[0] += red[i][c].x;
+                r[1] += red[i][c].y;
+                r[2] += red[i][c].z;
+                r[3] += red[i][c].w;
+            }
+            const int l = static_cast<int>((idx * 4) % L);
+            if (bias) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) r[e] += bf16_bits_to_float(bias[l + e]);
+            }
+            uint2 o;
+            o.x = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(r[0]))) |
+                  (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(r[1]))) << 16);
+            o.y = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(r[2]))) |
+                  (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(r[3]))) << 16);
+            *reinterpret_cast<uint2*>(out + idx * 4) = o;
         }
         __syncthreads();
     }

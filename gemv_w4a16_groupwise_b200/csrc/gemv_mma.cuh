@@ -59,11 +59,6 @@ __host__ __device__ inline size_t gemv_mma_xblock_bytes(int M, int TKC) {
     return static_cast<size_t>(TKC) / 128 * M * (256 + 8);
 }
 
-// Programmatic dependent launch: a kernel lets its dependents start early;
-// a dependent waits for the kernels before it where it needs their results.
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 // A conversion unit is 256 k of one activation row: lane = 16 h + 4 t + tig
 // converts the 8 activations k_first + 128 h + 32 tig + 8 t .. + 7 (zero past
 // K), i.e. chunk t of B lane tig's 32 k in granule h of the unit.

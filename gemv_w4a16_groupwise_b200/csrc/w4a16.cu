@@ -15,6 +15,7 @@
 #include "gemv_stream.cuh"
 #include "gemv_mma.cuh"
 #include "gemv_t_stream.cuh"
+#include "gemv_t_mma.cuh"
 #include "quantize.cuh"
 #include "w4a16.h"
 
@@ -81,6 +82,24 @@ cudaError_t ensure_smem(const void* fn, size_t bytes) {
     }
     if (count < 512) table[count++] = Entry{dev, fn, bytes};
     return cudaSuccess;
+}
+
+// Launch `fn` as a programmatic dependent of the work before it on `st`:
+// it may start once that work has let it (griddepcontrol.launch_dependents)
+// and must wait (griddepcontrol.wait) before reading that work's results.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*fn)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, fn, static_cast<KArgs>(args)...);
 }
 
 // ------------------------------------------------------------ tensor maps
@@ -229,6 +248,39 @@ TStreamPlan plan_t_stream(int M, int N, int K, int sz, int sms) {
     return p;
 }
 
+// Tensor-pipe transposed GEMV (gemv_t_mma_kernel): the same shapes as the
+// streaming kernel.  Row ranges are whole 32-row stages; the grid is a whole
+// number of splits per strip, at most one CTA per SM, with the fp32
+// partials held under about a tenth of the weights.
+struct TMmaPlan {
+    bool ok = false;
+    int strips = 0, splits = 1, rows_per_split = 0, stages = 0, grid = 0;
+    size_t smem = 0, ws = 0;
+};
+
+TMmaPlan plan_t_mma(int M, int N, int K, int sms, int max_smem) {
+    TMmaPlan p;
+    p.strips = (K + kTMStrip - 1) / kTMStrip;
+    int splits = std::max(1, sms / p.strips);
+    splits = std::min(splits, std::max(1, N / (80 * M)));
+    splits = std::min(splits, std::max(1, N / (kTMRows * 4)));   // at least 4 stages of rows per split
+    auto set_rows = [&](int sp) {
+        p.rows_per_split = ((N + sp - 1) / sp + kTMRows - 1) / kTMRows * kTMRows;
+        p.splits = (N + p.rows_per_split - 1) / p.rows_per_split;
+    };
+    set_rows(splits);
+    // the split's dY rows live in shared memory: keep them under 32 KB
+    while (static_cast<size_t>(p.rows_per_split) * 16 > 32 * 1024) set_rows(++splits);
+    p.grid = p.strips * p.splits;
+    const size_t fixed = gemv_t_mma_smem_bytes(0, p.rows_per_split);
+    const size_t avail = max_smem > 0 ? static_cast<size_t>(max_smem) : 232448;
+    p.stages = avail > fixed ? static_cast<int>(std::min<size_t>(8, (avail - fixed) / (kTMStageBytes + 16))) : 0;
+    p.smem = gemv_t_mma_smem_bytes(p.stages, p.rows_per_split);
+    p.ws = p.splits > 1 ? static_cast<size_t>(p.splits) * M * K * sizeof(float) : 0;
+    p.ok = p.stages >= 2;
+    return p;
+}
+
 bool t_stream_eligible(int K, const Meta& meta) {
     if (K % 32 != 0) return false;
     if (meta.sz_row == 0 || meta.G == 1) return true;
@@ -371,8 +423,10 @@ int mma_sz_kind(const Meta& meta) {
 size_t gemv_workspace(int M, int N, int K, int transposed, int sms) {
     if (transposed) {
         size_t ws = plan_t(M, N, K, sms).ws;
-        if (K % 32 == 0)
+        if (K % 32 == 0) {
             for (int sz : {kSzConst, kSzTma2d, kSzTma1d}) ws = std::max(ws, plan_t_stream(M, N, K, sz, sms).ws);
+            ws = std::max(ws, plan_t_mma(M, N, K, sms, device_info(current_device()).max_smem_optin).ws);
+        }
         return ws;
     }
     if (K % 32 != 0) return 0;
@@ -676,12 +730,88 @@ w4_status run_gemv_t_stream(const TStreamPlan& p, int M, int N, int K, const voi
     return W4_OK;
 }
 
+template <int M, int SZ>
+w4_status launch_t_mma_k(const TMmaPlan& p, const CUtensorMap& wm, const CUtensorMap& sm, const CUtensorMap& zm,
+                         const GemvTMmaArgs& a, cudaStream_t st) {
+    auto* fn = gemv_t_mma_kernel<M, SZ>;
+    if (ensure_smem(reinterpret_cast<const void*>(fn), p.smem) != cudaSuccess) return W4_ERR_CUDA;
+    launch_pdl(fn, dim3(p.grid), dim3(kTMThreads), p.smem, st, wm, sm, zm, a);
+    return launch_status();
+}
+
+template <int M>
+w4_status launch_t_mma_m(const TMmaPlan& p, int sz, const CUtensorMap& wm, const CUtensorMap& sm,
+                         const CUtensorMap& zm, const GemvTMmaArgs& a, cudaStream_t st) {
+    switch (sz) {
+        case kSzConst: return launch_t_mma_k<M, kSzConst>(p, wm, sm, zm, a, st);
+        case kSzTma1d: return launch_t_mma_k<M, kSzTma1d>(p, wm, sm, zm, a, st);
+        default: return launch_t_mma_k<M, kSzTma2d>(p, wm, sm, zm, a, st);
+    }
+}
+
+w4_status run_gemv_t_mma(const TMmaPlan& p, int sz, int M, int N, int K, const void* A, const uint32_t* packed,
+                         const void* S, const void* Z, const Meta& meta, const void* bias, void* Y, void* ws,
+                         size_t ws_bytes, cudaStream_t st) {
+    if (p.ws > ws_bytes || (p.ws > 0 && ws == nullptr)) return W4_ERR_WORKSPACE;
+    CUtensorMap wm, sm, zm;
+    std::memset(&sm, 0, sizeof sm);
+    std::memset(&zm, 0, sizeof zm);
+    // packed rows as K / 16 8-byte elements: boxes of 32 rows x 1040 bytes
+    bool ok = make_map_2d(&wm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, N, K / 16, kTMRows, kTMBoxX, 0);
+    if (sz == kSzTma2d)
+        ok = ok && make_map_2d(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, meta.G, kTMRows, 16, 0) &&
+             make_map_2d(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, meta.G, kTMRows, 16, 0);
+    else if (sz == kSzTma1d)
+        ok = ok && make_map_row(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, kTMRows) &&
+             make_map_row(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, kTMRows);
+    if (!ok) return W4_ERR_CUDA;
+    GemvTMmaArgs a;
+    a.dY = static_cast<const uint16_t*>(A);
+    a.packed = packed;
+    a.S = static_cast<const __half*>(S);
+    a.Z = static_cast<const __half*>(Z);
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.dX = static_cast<uint16_t*>(Y);
+    a.partial = static_cast<float*>(ws);
+    a.N = N;
+    a.K = K;
+    a.g = meta.g;
+    a.G = meta.G;
+    a.sz_row = meta.sz_row;
+    a.strips = p.strips;
+    a.splits = p.splits;
+    a.rows_per_split = p.rows_per_split;
+    a.stages = p.stages;
+    w4_status s = W4_OK;
+    switch (M) {
+        case 1: s = launch_t_mma_m<1>(p, sz, wm, sm, zm, a, st); break;
+        case 2: s = launch_t_mma_m<2>(p, sz, wm, sm, zm, a, st); break;
+        case 3: s = launch_t_mma_m<3>(p, sz, wm, sm, zm, a, st); break;
+        case 4: s = launch_t_mma_m<4>(p, sz, wm, sm, zm, a, st); break;
+        default: return W4_ERR_INVALID_ARG;
+    }
+    if (s != W4_OK) return s;
+    if (p.splits > 1) {
+        // a programmatic dependent: its launch overlaps the split kernel,
+        // whose partials it waits for
+        const DeviceInfo di = device_info(current_device());
+        const long long total4 = static_cast<long long>(M) * K / 4;     // K % 32 == 0
+        const int blocks = static_cast<int>(std::min<long long>((total4 + kFin4Cols - 1) / kFin4Cols, di.sms * 8));
+        launch_pdl(splits_finalize_vec4_kernel, dim3(blocks), dim3(256), 0, st,
+                   static_cast<const float*>(a.partial), p.splits, M, K, a.bias, a.dX);
+        return launch_status();
+    }
+    return W4_OK;
+}
+
 w4_status run_gemv_t(const void* A, int M, int N, int K, const uint32_t* packed, const void* S,
                      const void* Z, const Meta& meta, const void* bias, void* Y, void* ws,
                      size_t ws_bytes, cudaStream_t st) {
     const DeviceInfo di = device_info(current_device());
     if (t_stream_eligible(K, meta)) {
         const int sz = meta.sz_row == 0 ? kSzConst : (meta.G == 1 ? kSzTma1d : kSzTma2d);
+        const TMmaPlan mp = plan_t_mma(M, N, K, di.sms, di.max_smem_optin);
+        if (mp.ok) return run_gemv_t_mma(mp, sz, M, N, K, A, packed, S, Z, meta, bias, Y, ws, ws_bytes, st);
         const TStreamPlan tp = plan_t_stream(M, N, K, sz, di.sms);
         return run_gemv_t_stream(tp, M, N, K, A, packed, S, Z, meta, bias, Y, ws, ws_bytes, st);
     }

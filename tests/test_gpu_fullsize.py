@@ -117,3 +117,26 @@ def test_llama3_8b_serving_bias(cuda_device, M):
     ref, _ = oracle.linear(X, p_ref, s_ref, z_ref, "groupwise", 128, N, K, bias=b, cols=cols)
     assert_close(from_dev_bits(y)[:, cols], ref, f"l38 M={M}")
     assert w4.w4_device_error() == 0
+
+
+@pytest.mark.parametrize("mode,g", [("groupwise", 128), ("rowwise", 0), ("global", 0)])
+def test_llama3_8b_transposed_gemv(cuda_device, mode, g):
+    """Transposed GEMV (M = 1..4) at the gate_up shape N = 28672, K = 4096:
+    every row split of the grid, sampled output columns, run to run equal."""
+    import torch
+    import gemv_w4a16_groupwise_b200 as w4
+    dev = cuda_device
+    N, K = 28672, 4096
+    seed = synth.config_seed("l38t", N, K)
+    W = synth.weights(N, K, seed)
+    (p, s, z), (p_ref, s_ref, z_ref) = quantize_both(W, mode, g, dev)
+    kc = sample_cols(K, 96, seed)
+    for M in (1, 2, 3, 4):
+        dY = synth.grads(M, N, seed + M)
+        dYd = to_dev_bf16(dY, dev)
+        x1 = w4.w4a16_gemv(dYd, p, s, z, mode, g, N=N, K=K, transposed=True)
+        x2 = w4.w4a16_gemv(dYd, p, s, z, mode, g, N=N, K=K, transposed=True)
+        assert torch.equal(x1, x2), "transposed GEMV is not deterministic"
+        ref, _ = oracle.linear_t(dY, p_ref, s_ref, z_ref, mode, g, N, K, cols=kc)
+        assert_close(from_dev_bits(x1)[:, kc], ref, f"l38^T M={M} {mode}")
+    assert w4.w4_device_error() == 0
