@@ -193,8 +193,15 @@ __global__ void __launch_bounds__(kTMThreads, 1)
         // in acc are in units of xs = 2^(E - 140).  When a stage raises E[m],
         // the lanes of m first move acc into the fp32 sums fac (in units of
         // the old xs) and clear it, and every lane rescales its sum of c' z.
-        int E[4] = {14, 14, 14, 14};
-        auto xs_of = [](int e) { return __int_as_float((e - 13) << 23); };    // 2^(e - 140)
+        // The precision of c' is never below that of one exponent for all
+        // of the CTA's rows.
+        // thr[m] = 2^(E[m] - 126): |c| >= thr[m] means an exponent above E[m];
+        // from its bits, 2^(140 - E) = bits 0x86000000 - thr and
+        // 2^(E - 140) = bits thr - 0x07000000
+        float thr[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) thr[m] = __int_as_float((14 + 1) << 23);
+        auto xs_of = [](float th) { return __int_as_float(__float_as_int(th) - 0x07000000); };
         // this lane's stage row r = 8 i + 2 t + h and its table bytes
         const int ti = lane >> 3, tt = (lane >> 1) & 3, th = lane & 1;
         uint8_t* tab = tabs + warp * kTMTabBytes;
@@ -239,6 +246,15 @@ __global__ void __launch_bounds__(kTMThreads, 1)
                                                                       kErrTimeoutTmaFull));
             if (!ok) break;
             const uint8_t* sb = ring + s * kTMStageBytes;
+            // ---- this lane's code words first, so that their latency overlaps
+            // the digits: words 2 gid (S = 0) and 2 gid + 1 (S = 1) of the
+            // warp's 16, rows 8 i + 2 tig + h
+            uint2 w[2][4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    w[h][i] = *reinterpret_cast<const uint2*>(sb + col0 + (8 * i + h) * kTMPitch);
             // ---- digits of c for stage row `lane` and the warp's group
             {
                 float sv, zv;
@@ -256,23 +272,25 @@ __global__ void __launch_bounds__(kTMThreads, 1)
                 }
                 const float4 d4 = dys[b * kTMRows + lane];
                 const float c[4] = {d4.x * sv, d4.y * sv, d4.z * sv, d4.w * sv};
-                int es[4];
-                bool raise = false;
+                const bool up = fabsf(c[0]) >= thr[0] || fabsf(c[1]) >= thr[1] || fabsf(c[2]) >= thr[2] ||
+                                fabsf(c[3]) >= thr[3];
+                if (__any_sync(0xFFFFFFFFu, up)) {              // rare: an exponent rises
+                    float tn[4];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    es[m] = min(static_cast<int>(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(c[m]) & 0x7FFFFFFFu) >> 23),
-                                254);
-                    raise |= es[m] > E[m];
-                }
-                if (raise) {                                  // warp-uniform
-                    if (pick(es) > pick(E)) fold(xs_of(pick(E)));
+                    for (int m = 0; m < 4; ++m) {
+                        const int e = min(static_cast<int>(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(c[m]) & 0x7FFFFFFFu) >> 23),
+                                          254);
+                        tn[m] = fmaxf(thr[m], __int_as_float((e + 1) << 23));
+                    }
+                    if (pick(tn) > pick(thr)) fold(xs_of(pick(thr)));
 #pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        if (es[m] > E[m]) {
-                            const int f = 127 + E[m] - es[m];               // 2^(E_old - E_new), or 0 below 2^-126
-                            zt[m] *= f > 0 ? __int_as_float(f << 23) : 0.0f;
-                            E[m] = es[m];
-                        }
+                    for (int m = 0; m < 4; ++m) {
+                        // 2^(E_old - E_new) from the exponent fields (thr may
+                        // be +inf, the bits of E = 254), or 0 below 2^-126
+                        const int f = 127 + ((__float_as_int(thr[m]) - __float_as_int(tn[m])) >> 23);
+                        zt[m] *= f > 0 ? __int_as_float(f << 23) : 0.0f;
+                        thr[m] = tn[m];
+                    }
                 }
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
@@ -280,7 +298,7 @@ __global__ void __launch_bounds__(kTMThreads, 1)
                     // in one rounding; the bit pattern of t is 0x4B400000 + c', so
                     // its low byte is the low digit lo = c' - 256 hi (as a signed
                     // byte) and byte 1 of bits + 128 is hi = (c' + 128) >> 8
-                    const float t = fmaf(c[m], __int_as_float((267 - E[m]) << 23), 12582912.0f);   // 2^(140 - E)
+                    const float t = fmaf(c[m], __int_as_float(0x86000000 - __float_as_int(thr[m])), 12582912.0f);
                     const uint32_t tb = __float_as_uint(t);
                     tab[m * 32 + tbyte] = static_cast<uint8_t>((tb + 128u) >> 8);
                     tab[(4 + m) * 32 + tbyte] = static_cast<uint8_t>(tb);
@@ -289,14 +307,7 @@ __global__ void __launch_bounds__(kTMThreads, 1)
             }
             __syncwarp();
             const uint32_t b0 = tabw[bsel], b1 = tabw[bsel + 4];
-            // ---- codes: words 2 gid (S = 0) and 2 gid + 1 (S = 1) of the
-            // warp's 16, four nibble pairs each
-            uint2 w[2][4];
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    w[h][i] = *reinterpret_cast<const uint2*>(sb + col0 + (8 * i + h) * kTMPitch);
+            // ---- codes: four nibble pairs of each word
 #pragma unroll
             for (int S = 0; S < 2; ++S) {
                 uint32_t x0[4], x1[4];
@@ -323,7 +334,7 @@ __global__ void __launch_bounds__(kTMThreads, 1)
         for (int m = 0; m < 4; ++m)
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) zt[m] += __shfl_xor_sync(0xFFFFFFFFu, zt[m], o);
-        const float xsm = xs_of(pick(E));
+        const float xsm = xs_of(pick(thr));
         fold(xsm);
         const float zterm = pick(zt) * xsm;
         const int k = kw + 16 * gid;                     // words 2 gid, 2 gid + 1
