@@ -11,10 +11,14 @@
 // added to the fp32 accumulator before the single bf16 rounding (vLLM
 // "Adding bias epilogue support for cutlass_scaled_mm").
 //
-// Persistent: one CTA per SM walks tiles blockIdx.x, + gridDim.x, ...; the
-// stage ring runs on across tile boundaries and the fp32 accumulator is
-// double-buffered in TMEM, so one tile's epilogue overlaps the next tile's
-// main loop.  Warp roles (704 threads):
+// Persistent: one CTA per SM walks work units blockIdx.x, + gridDim.x, ...;
+// the stage ring runs on across unit boundaries and the fp32 accumulator is
+// double-buffered in TMEM, so one unit's epilogue overlaps the next unit's
+// main loop.  A unit is a whole tile, or, for the tiles of a last partial
+// wave (from tile F on), one of S slices of the tile's k-blocks: those
+// units write fp32 partial tiles, which gemm_tail_finalize_kernel adds in
+// slice order (with the bias) and rounds, so the last wave takes about
+// 1 / S of a tile's time instead of a whole one.  Warp roles (704 threads):
 //   warp 0       TMA producer: packed weight tile + activation tile per stage
 //   warp 1       TMEM allocator; lane 0 issues tcgen05.mma and commits
 //   warps 2..17  dequantize packed codes into the bf16 A tile of a stage
@@ -52,9 +56,12 @@ struct TcArgs {
     const __half* Z;
     const uint16_t* bias;
     uint16_t* Y;
+    float* part;          // [(tiles - F) * nslice][BN][128] fp32 partial tiles of the split tail
     int M, N, K;
     int g, G, sz_row;
     int stages;
+    int F;                // tiles 0 .. F - 1 are whole work units
+    int nslice;           // k slices of each tile from F on (1: no split)
 };
 
 struct TcProblem {
@@ -184,10 +191,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int num_kb = (red_len + kTcBK - 1) / kTcBK;
     const int tiles_m = (a.M + BN - 1) / BN;
     const int tiles = tiles_m * ((L_out + kTcBM - 1) / kTcBM);
-    // this CTA's tiles: blockIdx.x, + gridDim.x, ...; tile t covers tokens
+    const int units = a.F + (tiles - a.F) * a.nslice;
+    // this CTA's units: blockIdx.x, + gridDim.x, ...; tile t covers tokens
     // (t % tiles_m) * BN .. and output rows (t / tiles_m) * 128 ..
-    const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    auto tile_of = [&](int i) { return blockIdx.x + i * gridDim.x; };
+    const int my_units = blockIdx.x < units ? (units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    struct Unit {
+        int t, kb0, kb1;
+        int part;        // index of the partial tile, or -1 for a whole tile
+    };
+    auto unit_of = [&](int i) {
+        const int u = blockIdx.x + i * gridDim.x;
+        Unit w;
+        if (u < a.F) {
+            w.t = u;
+            w.kb0 = 0;
+            w.kb1 = num_kb;
+            w.part = -1;
+        } else {
+            const int v = u - a.F, sl = v % a.nslice;
+            w.t = a.F + v / a.nslice;
+            w.kb0 = sl * num_kb / a.nslice;
+            w.kb1 = (sl + 1) * num_kb / a.nslice;
+            w.part = v;
+        }
+        return w;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -222,10 +250,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int s = 0;
             uint32_t round = 0;
             bool ok = true;
-            for (int i = 0; i < my_tiles && ok; ++i) {
-                const int t = tile_of(i);
-                const int m0 = (t % tiles_m) * BN, r0 = (t / tiles_m) * kTcBM;
-                for (int kb = 0; kb < num_kb; ++kb) {
+            for (int i = 0; i < my_units && ok; ++i) {
+                const Unit w = unit_of(i);
+                const int m0 = (w.t % tiles_m) * BN, r0 = (w.t / tiles_m) * kTcBM;
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (round > 0 && !mbar_wait_bounded(&empty[s], (round - 1) & 1u, abort_flag, kErrTimeoutEmpty)) {
                         ok = false;
                         break;
@@ -250,14 +278,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             bool ok = true;
             int s = 0;
             uint32_t phase = 0;
-            for (int i = 0; i < my_tiles && ok; ++i) {
+            for (int i = 0; i < my_units && ok; ++i) {
+                const Unit w = unit_of(i);
                 const int buf = i & 1;
                 // the epilogue has drained this buffer (tile i - 2)
                 if (i >= 2) ok = mbar_wait_bounded(&acc_empty[buf], ((i >> 1) - 1) & 1u, abort_flag, kErrTimeoutAccum);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t acc = tmem_d + static_cast<uint32_t>(buf) * kAccCols;
-                for (int kb = 0; kb < num_kb; ++kb) {
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     ok = mbar_wait_bounded(&tma_full[s], phase, abort_flag, kErrTimeoutTmaFull) &&
                          mbar_wait_bounded(&deq_full[s], phase, abort_flag, kErrTimeoutDequant);
                     if (!ok) break;
@@ -269,7 +298,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         const uint64_t adesc = TR ? umma_desc_sw128(a_addr + j * 2048, 8192, 1024)
                                                   : umma_desc_sw128(a_addr + j * 32, 16, 1024);
                         const uint64_t bdesc = umma_desc_sw128(b_addr + j * 32, 16, 1024);
-                        umma_bf16(acc, adesc, bdesc, kIdesc, (kb | j) != 0 ? 1u : 0u);
+                        umma_bf16(acc, adesc, bdesc, kIdesc, (kb != w.kb0 || j != 0) ? 1u : 0u);
                     }
                     umma_commit(&empty[s]);
                     if (++s == NS) {
@@ -282,8 +311,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp < 2 + 8 * kTcDeqGroups) {
         // ------------------------------------------------ dequantize
-        // Stages are numbered across the CTA's tiles (c = i * num_kb + kb);
-        // group grp_id takes c = grp_id, grp_id + 2, ...
+        // Stages are numbered across the CTA's units, in order; group grp_id
+        // takes stages grp_id, grp_id + 2, ...
         const int grp_id = (threadIdx.x - 64) >> 8;
         const int t = (threadIdx.x - 64) & 255;               // 0 .. 255 within the group
         // forward: row n = r0 + t % 128, words 4h .. 4h+3 of the 8 in a k-block
@@ -310,7 +339,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // Scale / zero of one stage (tile i, block kb); with g a multiple of
         // 32 the thread's 4 words share one group.
         constexpr int NG = PWG ? 4 : 1;
-        auto tile_r0 = [&](int i) { return (tile_of(i) / tiles_m) * kTcBM; };
+        auto tile_r0 = [&](int i) { return (unit_of(i).t / tiles_m) * kTcBM; };
         auto load_sz = [&](int r0, int kb, float (&sv)[NG], float (&zv)[NG]) {
             const int n = TR ? kb * kTcBK + prow : r0 + prow;
             const int nc = min(n, a.N - 1);
@@ -324,27 +353,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 zv[j] = __half2float(__ldg(zp + grp));
             }
         };
-        const int total = my_tiles * num_kb;
-        // this group's first stage, and its ring slot and phase
-        int ci = 0, ckb = grp_id;
-        while (ckb >= num_kb && ci < my_tiles) {
-            ckb -= num_kb;
-            ++ci;
+        // (ci, ckb): unit and k-block of this group's current stage; cb1 is
+        // the end of the unit's k-blocks.  Advancing by `step` stages walks
+        // into the following units.
+        auto advance = [&](int& i, int& kb, int& kb1, int step) {
+            kb += step;
+            while (i < my_units && kb >= kb1) {
+                const int over = kb - kb1;
+                if (++i >= my_units) break;
+                const Unit w = unit_of(i);
+                kb = w.kb0 + over;
+                kb1 = w.kb1;
+            }
+        };
+        int ci = 0, ckb = 0, cb1 = 0;
+        if (my_units > 0) {
+            const Unit w0 = unit_of(0);
+            ckb = w0.kb0;
+            cb1 = w0.kb1;
+            advance(ci, ckb, cb1, grp_id);
         }
         int s = grp_id % NS;
         uint32_t phase = static_cast<uint32_t>(grp_id / NS) & 1u;
         float sv[NG], zv[NG], svn[NG], zvn[NG];
-        int cr0 = grp_id < total ? tile_r0(ci) : 0;          // output row offset of the current tile
-        if (grp_id < total) load_sz(cr0, ckb, sv, zv);
-        for (int c = grp_id; c < total; c += kTcDeqGroups) {
+        int cr0 = ci < my_units ? tile_r0(ci) : 0;           // output row offset of the current tile
+        if (ci < my_units) load_sz(cr0, ckb, sv, zv);
+        while (ci < my_units) {
             // the next stage of this group, whose scales are fetched now
-            int ni = ci, nkb = ckb + kTcDeqGroups;
-            while (nkb >= num_kb) {
-                nkb -= num_kb;
-                ++ni;
-            }
-            const int nr0 = (ni != ci && c + kTcDeqGroups < total) ? tile_r0(ni) : cr0;
-            if (c + kTcDeqGroups < total) load_sz(nr0, nkb, svn, zvn);
+            int ni = ci, nkb = ckb, nb1 = cb1;
+            advance(ni, nkb, nb1, kTcDeqGroups);
+            const bool more = ni < my_units;
+            const int nr0 = (more && ni != ci) ? tile_r0(ni) : cr0;
+            if (more) load_sz(nr0, nkb, svn, zvn);
             const int r0 = cr0;
             const int n = TR ? ckb * kTcBK + prow : r0 + prow;
             const int kw0 = TR ? r0 / 8 + 4 * pquad : ckb * (kTcBK / 8) + 4 * pquad;
@@ -376,6 +416,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             ci = ni;
             ckb = nkb;
+            cb1 = nb1;
             cr0 = nr0;
             s += kTcDeqGroups;
             while (s >= NS) {
@@ -386,13 +427,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else {
         // ------------------------------------------------ epilogue
         const int q = warp & 3;                 // TMEM lanes 32 q .. 32 q + 31
-        for (int i = 0; i < my_tiles; ++i) {
+        for (int i = 0; i < my_units; ++i) {
             const int buf = i & 1;
             const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1u, abort_flag,
                                                                       kErrTimeoutAccum));
             if (!ok || *abort_flag) break;
             tc_fence_after();
-            const int t = tile_of(i);
+            const Unit w = unit_of(i);
+            const int t = w.t;
             const int m0 = (t % tiles_m) * BN, r0 = (t / tiles_m) * kTcBM;
             const int row = r0 + 32 * q + lane;
             const bool rv = row < L_out;
@@ -405,7 +447,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const bool odd = (lane & 1) != 0;
             const int prow = row - (odd ? 1 : 0);            // first row of the pair
             const bool pv = prow < L_out;
-            if (L_out & 1) {
+            if (w.part >= 0) {
+                // a k slice of a tail tile: fp32 partial [token][row] of the tile
+                float* pt = a.part + static_cast<size_t>(w.part) * (BN * kTcBM) + 32 * q + lane;
+#pragma unroll 1
+                for (int c0 = 0; c0 < BN; c0 += 8) {
+                    uint32_t r[8];
+                    tmem_ld_x8(acc + static_cast<uint32_t>(c0), r);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) pt[(c0 + e) * kTcBM] = __uint_as_float(r[e]);
+                }
+            } else if (L_out & 1) {
 #pragma unroll 1
                 for (int c0 = 0; c0 < BN; c0 += 8) {
                     uint32_t r[8];
@@ -452,6 +504,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      "r"(kTmemCols)
                      : "memory");
     }
+}
+
+// The tail tiles of a split GEMM: out[m, row] = bf16(sum over the S slices
+// of the tile's fp32 partials, in slice order, + bias[row]).  One thread
+// per (token, row) of a tile, rows fastest (coalesced reads and stores).
+__global__ void __launch_bounds__(256) gemm_tail_finalize_kernel(const float* __restrict__ part, int F, int S,
+                                                                 int ntail, int tiles_m, int BN, int M, int L_out,
+                                                                 const uint16_t* __restrict__ bias,
+                                                                 uint16_t* __restrict__ Y) {
+    pdl_wait();   // launched as a programmatic dependent of the GEMM
+    const long long per_tile = static_cast<long long>(BN) * kTcBM;
+    const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= per_tile * ntail) return;
+    const int tt = static_cast<int>(idx / per_tile);            // tail tile
+    const int e = static_cast<int>(idx - tt * per_tile);
+    const int ml = e / kTcBM, rl = e % kTcBM;
+    const int t = F + tt;
+    const int m = (t % tiles_m) * BN + ml, row = (t / tiles_m) * kTcBM + rl;
+    if (m >= M || row >= L_out) return;
+    const float* p = part + static_cast<size_t>(tt) * S * per_tile + e;
+    float v = 0.0f;
+    for (int sl = 0; sl < S; ++sl) v += __ldg(p + static_cast<size_t>(sl) * per_tile);
+    if (bias) v += bf16_bits_to_float(bias[row]);
+    Y[static_cast<size_t>(m) * L_out + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
 }  // namespace w4

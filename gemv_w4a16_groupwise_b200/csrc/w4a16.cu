@@ -874,21 +874,66 @@ w4_status run_gemv(const void* A, int M, int N, int K, const uint32_t* packed, c
 
 
 // ---------------------------------------------------------- tensor-core GEMM
-size_t gemm_tc_workspace_bytes(int M, int N, int K, int transposed, int sms) {
-    (void)M;
-    (void)N;
-    (void)K;
-    (void)transposed;
-    (void)sms;
-    return 0;
-}
-
 int tc_pick_bn(int M) {
     if (M <= 16) return 16;
     if (M <= 32) return 32;
     if (M <= 64) return 64;
     if (M <= 128) return 128;
     return 256;
+}
+
+// Work split of the persistent GEMM.  With T tiles on P SMs, T / P whole
+// waves run as whole tiles; the R = T mod P tiles of a last partial wave
+// (all tiles, when T < P) are cut into S slices of their k-blocks when that
+// pays: the tail then takes ceil(R S / P) / S of a tile's time instead of a
+// whole one, against the cost of writing and re-reading R S fp32 partial
+// tiles plus a finalize launch; S maximizes the difference.  Slices keep at
+// least 4 k-blocks.
+struct TcPlan {
+    int BN = 0, tiles_m = 0, tiles = 0, F = 0, S = 1, grid = 0;
+    size_t ws = 0;
+};
+
+TcPlan plan_tc(int M, int N, int K, int transposed, int sms) {
+    TcPlan p;
+    p.BN = tc_pick_bn(M);
+    const int L_out = transposed ? K : N;
+    const int red = transposed ? N : K;
+    const int num_kb = (red + kTcBK - 1) / kTcBK;
+    p.tiles_m = (M + p.BN - 1) / p.BN;
+    const long long tiles = static_cast<long long>(p.tiles_m) * ((L_out + kTcBM - 1) / kTcBM);
+    p.tiles = static_cast<int>(std::min<long long>(tiles, 1ll << 30));
+    const int P = std::max(1, sms);
+    const int R = p.tiles % P;
+    p.F = p.tiles;
+    if (R > 0) {
+        // a tile's time in microseconds, roughly: a 64-k block of 128 x BN
+        // takes ~0.5 us per 256 tokens at the rates this kernel reaches
+        const double tile_us = num_kb * (p.BN / 256.0) * 0.5;
+        double best = 0.0;
+        int bestS = 1;
+        for (int S = 2; S <= std::min(16, num_kb / 4); ++S) {
+            const double tail = static_cast<double>((static_cast<long long>(R) * S + P - 1) / P) / S;
+            const double cost = 3.0 + 2.0 * R * S * p.BN * kTcBM * 4 / 4.0e6;   // us
+            const double gain = (1.0 - tail) * tile_us - cost;
+            if (gain > best + 1e-9) {
+                best = gain;
+                bestS = S;
+            }
+        }
+        if (bestS > 1) {
+            p.S = bestS;
+            p.F = p.tiles - R;
+        }
+    }
+    const long long units = p.F + static_cast<long long>(p.tiles - p.F) * p.S;
+    p.grid = static_cast<int>(std::min<long long>(units, P));
+    p.ws = static_cast<size_t>(p.tiles - p.F) * p.S * p.BN * kTcBM * sizeof(float);
+    return p;
+}
+
+size_t gemm_tc_workspace_bytes(int M, int N, int K, int transposed, int sms) {
+    return plan_tc(M, N, K, transposed, sms).ws;
 }
 
 template <bool TR, int BN, bool PWG>
@@ -912,11 +957,13 @@ w4_status launch_tc_bn(int BN, const CUtensorMap& pm, const CUtensorMap& bm, con
     }
 }
 
-w4_status run_gemm_tc(const TcProblem& p, cudaStream_t st) {
+w4_status run_gemm_tc(const TcProblem& p, void* ws, size_t ws_bytes, cudaStream_t st) {
     if (p.K % 32 != 0) return W4_ERR_UNSUPPORTED;      // packed rows must be 16-byte strided
     if (p.transposed && p.N % 8 != 0) return W4_ERR_UNSUPPORTED;  // dY rows 16-byte strided
     const DeviceInfo di = device_info(current_device());
-    const int BN = tc_pick_bn(p.M);
+    const TcPlan plan = plan_tc(p.M, p.N, p.K, p.transposed, di.sms);
+    if (plan.ws > ws_bytes || (plan.ws > 0 && ws == nullptr)) return W4_ERR_WORKSPACE;
+    const int BN = plan.BN;
     const int stage = tc_stage_bytes(BN);
     const size_t fixed = 1024 + 64;
     int stages = static_cast<int>((static_cast<size_t>(di.max_smem_optin) - fixed - 64) / (stage + 24));
@@ -944,16 +991,25 @@ w4_status run_gemm_tc(const TcProblem& p, cudaStream_t st) {
     a.G = p.G;
     a.sz_row = p.sz_row;
     a.stages = stages;
+    a.part = static_cast<float*>(ws);
+    a.F = plan.F;
+    a.nslice = plan.S;
     const int L_out = tr ? p.K : p.N;
-    // persistent: one CTA per SM (or per tile, when there are fewer tiles)
-    const long long tiles = static_cast<long long>((p.M + BN - 1) / BN) * ((L_out + kTcBM - 1) / kTcBM);
-    if (tiles > (1ll << 30)) return W4_ERR_UNSUPPORTED;
-    const dim3 grid(static_cast<unsigned>(std::min<long long>(tiles, di.sms)));
+    if (static_cast<long long>(p.M + BN - 1) / BN * ((L_out + kTcBM - 1) / kTcBM) > (1ll << 30))
+        return W4_ERR_UNSUPPORTED;
+    // persistent: one CTA per SM (or per work unit, when there are fewer)
+    const dim3 grid(static_cast<unsigned>(plan.grid));
     const bool pwg = (p.g % 32) != 0;
-    if (tr) return pwg ? launch_tc_bn<true, true>(BN, pm, bm, a, grid, smem, st)
-                       : launch_tc_bn<true, false>(BN, pm, bm, a, grid, smem, st);
-    return pwg ? launch_tc_bn<false, true>(BN, pm, bm, a, grid, smem, st)
-               : launch_tc_bn<false, false>(BN, pm, bm, a, grid, smem, st);
+    w4_status s = tr ? (pwg ? launch_tc_bn<true, true>(BN, pm, bm, a, grid, smem, st)
+                            : launch_tc_bn<true, false>(BN, pm, bm, a, grid, smem, st))
+                     : (pwg ? launch_tc_bn<false, true>(BN, pm, bm, a, grid, smem, st)
+                            : launch_tc_bn<false, false>(BN, pm, bm, a, grid, smem, st));
+    if (s != W4_OK || plan.F == plan.tiles) return s;
+    const long long elems = static_cast<long long>(plan.tiles - plan.F) * BN * kTcBM;
+    launch_pdl(gemm_tail_finalize_kernel, dim3(static_cast<unsigned>((elems + 255) / 256)), dim3(256), 0, st,
+               static_cast<const float*>(a.part), plan.F, plan.S, plan.tiles - plan.F, plan.tiles_m, BN, p.M, L_out,
+               a.bias, a.Y);
+    return launch_status();
 }
 
 
@@ -1113,7 +1169,7 @@ w4_status w4a16_gemm(const void* A, int M, int N, int K, const uint32_t* packed,
     pr.transposed = transposed;
     pr.Y = Y;
     pr.sms = sms;
-    return run_gemm_tc(pr, st);
+    return run_gemm_tc(pr, workspace, workspace_bytes, st);
 }
 
 // Forward GEMV (M <= 4) that allocates nothing: its workspace goes to

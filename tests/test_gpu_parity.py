@@ -122,6 +122,21 @@ def test_gemm_parity(cuda_device, M, N, K, mode, g, transposed):
     assert_close(y, ref, f"gemm M={M} N={N} K={K} {mode} g={g} t={transposed}")
 
 
+@pytest.mark.parametrize("M,N,K,mode,g,transposed,bias", [
+    (64, 4096, 4096, "groupwise", 64, False, True),     # 32 tiles < SMs: every tile in k slices
+    (64, 4096, 4096, "groupwise", 128, True, False),
+    (512, 512, 2048, "rowwise", 0, False, False),
+])
+def test_gemm_split_tail(cuda_device, M, N, K, mode, g, transposed, bias):
+    """Tiles of a last partial wave (here, all tiles) split into k slices whose
+    fp32 partials are added by the tail finalize."""
+    import gemv_w4a16_groupwise_b200 as w4
+    y, ref = run_matmul("w4a16_gemm", M, N, K, mode, g, transposed, bias=bias,
+                        seed=synth.config_seed("split", M, N, K, mode, g), dev=cuda_device)
+    assert w4.w4_workspace_bytes(M, N, K, transposed) > 0      # the split path runs
+    assert_close(y, ref, f"gemm split M={M} N={N} K={K} t={transposed}")
+
+
 @pytest.mark.parametrize("M", [5, 40, 300])
 def test_gemm_odd_output_length(cuda_device, M):
     """An odd number of output rows: the epilogue stores single bf16 values."""
