@@ -908,13 +908,14 @@ TcPlan plan_tc(int M, int N, int K, int transposed, int sms) {
     p.F = p.tiles;
     if (R > 0) {
         // a tile's time in microseconds, roughly: a 64-k block of 128 x BN
-        // takes ~0.5 us per 256 tokens at the rates this kernel reaches
-        const double tile_us = num_kb * (p.BN / 256.0) * 0.5;
+        // takes ~0.75 us per 256 tokens at the rates this kernel reaches
+        const double tile_us = num_kb * (p.BN / 256.0) * 0.75;
         double best = 0.0;
         int bestS = 1;
         for (int S = 2; S <= std::min(16, num_kb / 4); ++S) {
             const double tail = static_cast<double>((static_cast<long long>(R) * S + P - 1) / P) / S;
-            const double cost = 3.0 + 2.0 * R * S * p.BN * kTcBM * 4 / 4.0e6;   // us
+            // the partials are written and read back through L2 (~8 TB/s)
+            const double cost = 3.0 + 2.0 * R * S * p.BN * kTcBM * 4 / 8.0e6;   // us
             const double gain = (1.0 - tail) * tile_us - cost;
             if (gain > best + 1e-9) {
                 best = gain;
