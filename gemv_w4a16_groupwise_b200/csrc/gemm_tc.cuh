@@ -507,27 +507,56 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // The tail tiles of a split GEMM: out[m, row] = bf16(sum over the S slices
-// of the tile's fp32 partials, in slice order, + bias[row]).  One thread
-// per (token, row) of a tile, rows fastest (coalesced reads and stores).
+// of the tile's fp32 partials, in slice order, + bias[row]).  One thread per
+// four consecutive rows of one token of a tile: its slice loads (float4,
+// up to 8 at a time, indices past the last slice clamped to it and the
+// values dropped) go out together; rows fastest, so reads and stores are
+// coalesced.
 __global__ void __launch_bounds__(256) gemm_tail_finalize_kernel(const float* __restrict__ part, int F, int S,
                                                                  int ntail, int tiles_m, int BN, int M, int L_out,
                                                                  const uint16_t* __restrict__ bias,
                                                                  uint16_t* __restrict__ Y) {
     pdl_wait();   // launched as a programmatic dependent of the GEMM
-    const long long per_tile = static_cast<long long>(BN) * kTcBM;
+    const long long per_tile4 = static_cast<long long>(BN) * (kTcBM / 4);
     const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (idx >= per_tile * ntail) return;
-    const int tt = static_cast<int>(idx / per_tile);            // tail tile
-    const int e = static_cast<int>(idx - tt * per_tile);
-    const int ml = e / kTcBM, rl = e % kTcBM;
+    if (idx >= per_tile4 * ntail) return;
+    const int tt = static_cast<int>(idx / per_tile4);           // tail tile
+    const int e4 = static_cast<int>(idx - tt * per_tile4);
+    const int ml = e4 / (kTcBM / 4), rl = (e4 % (kTcBM / 4)) * 4;
     const int t = F + tt;
     const int m = (t % tiles_m) * BN + ml, row = (t / tiles_m) * kTcBM + rl;
     if (m >= M || row >= L_out) return;
-    const float* p = part + static_cast<size_t>(tt) * S * per_tile + e;
-    float v = 0.0f;
-    for (int sl = 0; sl < S; ++sl) v += __ldg(p + static_cast<size_t>(sl) * per_tile);
-    if (bias) v += bf16_bits_to_float(bias[row]);
-    Y[static_cast<size_t>(m) * L_out + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    const float4* p = reinterpret_cast<const float4*>(part) + static_cast<size_t>(tt) * S * per_tile4 + e4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < S; s0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = __ldg(p + static_cast<size_t>(min(s0 + j, S - 1)) * per_tile4);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (s0 + j < S) {
+                acc.x += v[j].x;
+                acc.y += v[j].y;
+                acc.z += v[j].z;
+                acc.w += v[j].w;
+            }
+    }
+    float r[4] = {acc.x, acc.y, acc.z, acc.w};
+    uint16_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        if (bias && row + q < L_out) r[q] += bf16_bits_to_float(bias[row + q]);
+        o[q] = __bfloat16_as_ushort(__float2bfloat16_rn(r[q]));
+    }
+    uint16_t* y = Y + static_cast<size_t>(m) * L_out + row;
+    if ((L_out & 3) == 0) {              // row + 3 < L_out, and y is 8-byte aligned
+        *reinterpret_cast<uint2*>(y) = make_uint2(o[0] | (static_cast<uint32_t>(o[1]) << 16),
+                                                  o[2] | (static_cast<uint32_t>(o[3]) << 16));
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            if (row + q < L_out) y[q] = o[q];
+    }
 }
 
 }  // namespace w4

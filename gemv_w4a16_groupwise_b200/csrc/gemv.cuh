@@ -7,12 +7,13 @@
 //  * gemv_fwd_simple_kernel: the forward product for shapes the streaming
 //    kernels do not take (K or the group length not a multiple of 32): one
 //    warp per output row, lanes along K, plain fp32 arithmetic;
-//  * splits_finalize_kernel: adds the fp32 partials of a split reduction
-//    (and the bias) in a fixed order;
-//  * gemv_t_kernel: the transposed product dX = dY . dequant(W) for M <= 4.
+//  * splits_finalize_kernel, splits_finalize_vec4_kernel: add the fp32
+//    partials of a split reduction (and the bias) in a fixed order;
+//  * gemv_t_kernel: the transposed product dX = dY . dequant(W) for M <= 4
+//    on shapes the tensor-pipe kernel does not take.
 //
 // The forward GEMV proper is in gemv_stream.cuh (CUDA cores) and
-// gemv_mma.cuh (tensor pipe).
+// gemv_mma.cuh (tensor pipe); the transposed one in gemv_t_mma.cuh.
 #pragma once
 
 #include "tma.cuh"

@@ -14,7 +14,6 @@
 #include "gemv.cuh"
 #include "gemv_stream.cuh"
 #include "gemv_mma.cuh"
-#include "gemv_t_stream.cuh"
 #include "gemv_t_mma.cuh"
 #include "quantize.cuh"
 #include "w4a16.h"
@@ -214,42 +213,9 @@ TPlan plan_t(int M, int N, int K, int sms) {
     return p;
 }
 
-// Streaming transposed GEMV (gemv_t_stream_kernel): K % 32 == 0 and the
+// Tensor-pipe transposed GEMV (gemv_t_mma_kernel): K % 32 == 0 and the
 // tensor-pipe GEMV's scale/zero layouts (g a multiple of 128 with G % 8 == 0,
-// one group per row, or one global pair).  Row splits fill the SMs with one
-// CTA each while the fp32 partials stay under about a tenth of the weights.
-struct TStreamPlan {
-    bool ok = false;
-    int strips = 0, splits = 1, rows_per_split = 0, stages = 24, grid = 0, sz = 0;
-    size_t smem = 0, ws = 0;
-};
-
-TStreamPlan plan_t_stream(int M, int N, int K, int sz, int sms) {
-    TStreamPlan p;
-    p.sz = sz;
-    p.strips = (K + kTSStrip - 1) / kTSStrip;
-    // one CTA per SM: the grid is a whole number of splits per strip, at
-    // most one wave, so no SM carries twice the rows of another
-    int splits = std::max(1, sms / p.strips);
-    splits = std::min(splits, std::max(1, N / (80 * M)));
-    splits = std::min(splits, std::max(1, N / (4 * 8)));   // at least 8 boxes per split
-    p.rows_per_split = ((N + splits - 1) / splits + kSR - 1) / kSR * kSR;
-    p.splits = (N + p.rows_per_split - 1) / p.rows_per_split;
-    // the split's dY rows live in shared memory: keep them under 48 KB
-    while (static_cast<size_t>(p.rows_per_split) * 16 > 48 * 1024) {
-        ++splits;
-        p.rows_per_split = ((N + splits - 1) / splits + kSR - 1) / kSR * kSR;
-        p.splits = (N + p.rows_per_split - 1) / p.rows_per_split;
-    }
-    p.grid = p.strips * p.splits;
-    p.smem = gemv_t_stream_smem_bytes(p.stages, sz, p.rows_per_split);
-    p.ws = p.splits > 1 ? static_cast<size_t>(p.splits) * M * K * sizeof(float) : 0;
-    p.ok = true;
-    return p;
-}
-
-// Tensor-pipe transposed GEMV (gemv_t_mma_kernel): the same shapes as the
-// streaming kernel.  Row ranges are whole 32-row stages; the grid is a whole
+// one group per row, or one global pair).  Row ranges are whole 32-row stages; the grid is a whole
 // number of splits per strip, at most one CTA per SM, with the fp32
 // partials held under about a tenth of the weights.
 struct TMmaPlan {
@@ -281,7 +247,7 @@ TMmaPlan plan_t_mma(int M, int N, int K, int sms, int max_smem) {
     return p;
 }
 
-bool t_stream_eligible(int K, const Meta& meta) {
+bool t_mma_eligible(int K, const Meta& meta) {
     if (K % 32 != 0) return false;
     if (meta.sz_row == 0 || meta.G == 1) return true;
     return meta.g % 128 == 0 && meta.G % 8 == 0;
@@ -423,10 +389,8 @@ int mma_sz_kind(const Meta& meta) {
 size_t gemv_workspace(int M, int N, int K, int transposed, int sms) {
     if (transposed) {
         size_t ws = plan_t(M, N, K, sms).ws;
-        if (K % 32 == 0) {
-            for (int sz : {kSzConst, kSzTma2d, kSzTma1d}) ws = std::max(ws, plan_t_stream(M, N, K, sz, sms).ws);
+        if (K % 32 == 0)
             ws = std::max(ws, plan_t_mma(M, N, K, sms, device_info(current_device()).max_smem_optin).ws);
-        }
         return ws;
     }
     if (K % 32 != 0) return 0;
@@ -658,78 +622,6 @@ w4_status run_gemv_fwd(const void* A, int M, int N, int K, const uint32_t* packe
     return launch_status();
 }
 
-template <int M, int GK, int SZ>
-w4_status launch_t_stream_k(const TStreamPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
-                            const CUtensorMap& zm, const GemvTStreamArgs& a, cudaStream_t st) {
-    auto* fn = gemv_t_stream_kernel<M, GK, SZ>;
-    if (ensure_smem(reinterpret_cast<const void*>(fn), p.smem) != cudaSuccess) return W4_ERR_CUDA;
-    fn<<<p.grid, kTSThreads, p.smem, st>>>(wm, sm, zm, a);
-    return launch_status();
-}
-
-template <int M>
-w4_status launch_t_stream_m(const TStreamPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
-                            const CUtensorMap& zm, const GemvTStreamArgs& a, cudaStream_t st) {
-    if (a.G == 1) {
-        switch (p.sz) {
-            case kSzConst: return launch_t_stream_k<M, kGroupsOne, kSzConst>(p, wm, sm, zm, a, st);
-            default: return launch_t_stream_k<M, kGroupsOne, kSzTma1d>(p, wm, sm, zm, a, st);
-        }
-    }
-    if (kSBK % a.g == 0) return launch_t_stream_k<M, kGroupsPow2, kSzTma2d>(p, wm, sm, zm, a, st);
-    return launch_t_stream_k<M, kGroupsAny, kSzTma2d>(p, wm, sm, zm, a, st);
-}
-
-w4_status run_gemv_t_stream(const TStreamPlan& p, int M, int N, int K, const void* A, const uint32_t* packed,
-                            const void* S, const void* Z, const Meta& meta, const void* bias, void* Y, void* ws,
-                            size_t ws_bytes, cudaStream_t st) {
-    if (p.ws > ws_bytes || (p.ws > 0 && ws == nullptr)) return W4_ERR_WORKSPACE;
-    CUtensorMap wm, sm, zm;
-    std::memset(&sm, 0, sizeof sm);
-    std::memset(&zm, 0, sizeof zm);
-    bool ok = make_map_2d(&wm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, kSR, kSBK / 8, 0);
-    if (p.sz == kSzTma2d)
-        ok = ok && make_map_2d(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, meta.G, kSR, 16, 0) &&
-             make_map_2d(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, meta.G, kSR, 16, 0);
-    else if (p.sz == kSzTma1d)
-        ok = ok && make_map_row(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, 8) &&
-             make_map_row(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, 8);
-    if (!ok) return W4_ERR_CUDA;
-    GemvTStreamArgs a;
-    a.dY = static_cast<const uint16_t*>(A);
-    a.S = static_cast<const __half*>(S);
-    a.Z = static_cast<const __half*>(Z);
-    a.bias = static_cast<const uint16_t*>(bias);
-    a.dX = static_cast<uint16_t*>(Y);
-    a.partial = static_cast<float*>(ws);
-    a.N = N;
-    a.K = K;
-    a.g = meta.g;
-    a.G = meta.G;
-    a.sz_row = meta.sz_row;
-    a.strips = p.strips;
-    a.splits = p.splits;
-    a.rows_per_split = p.rows_per_split;
-    a.stages = p.stages;
-    w4_status s = W4_OK;
-    switch (M) {
-        case 1: s = launch_t_stream_m<1>(p, wm, sm, zm, a, st); break;
-        case 2: s = launch_t_stream_m<2>(p, wm, sm, zm, a, st); break;
-        case 3: s = launch_t_stream_m<3>(p, wm, sm, zm, a, st); break;
-        case 4: s = launch_t_stream_m<4>(p, wm, sm, zm, a, st); break;
-        default: return W4_ERR_INVALID_ARG;
-    }
-    if (s != W4_OK) return s;
-    if (p.splits > 1) {
-        const DeviceInfo di = device_info(current_device());
-        const long long total = static_cast<long long>(M) * K;
-        const int blocks = static_cast<int>(std::min<long long>((total + kFinOut - 1) / kFinOut, di.sms * 16));
-        splits_finalize_kernel<<<blocks, 256, 0, st>>>(a.partial, p.splits, M, K, a.bias, a.dX);
-        return launch_status();
-    }
-    return W4_OK;
-}
-
 template <int M, int SZ>
 w4_status launch_t_mma_k(const TMmaPlan& p, const CUtensorMap& wm, const CUtensorMap& sm, const CUtensorMap& zm,
                          const GemvTMmaArgs& a, cudaStream_t st) {
@@ -808,12 +700,10 @@ w4_status run_gemv_t(const void* A, int M, int N, int K, const uint32_t* packed,
                      const void* Z, const Meta& meta, const void* bias, void* Y, void* ws,
                      size_t ws_bytes, cudaStream_t st) {
     const DeviceInfo di = device_info(current_device());
-    if (t_stream_eligible(K, meta)) {
+    if (t_mma_eligible(K, meta)) {
         const int sz = meta.sz_row == 0 ? kSzConst : (meta.G == 1 ? kSzTma1d : kSzTma2d);
         const TMmaPlan mp = plan_t_mma(M, N, K, di.sms, di.max_smem_optin);
         if (mp.ok) return run_gemv_t_mma(mp, sz, M, N, K, A, packed, S, Z, meta, bias, Y, ws, ws_bytes, st);
-        const TStreamPlan tp = plan_t_stream(M, N, K, sz, di.sms);
-        return run_gemv_t_stream(tp, M, N, K, A, packed, S, Z, meta, bias, Y, ws, ws_bytes, st);
     }
     const TPlan p = plan_t(M, N, K, di.sms);
     if (p.ws > ws_bytes || (p.ws > 0 && ws == nullptr)) return W4_ERR_WORKSPACE;
@@ -1006,8 +896,8 @@ w4_status run_gemm_tc(const TcProblem& p, void* ws, size_t ws_bytes, cudaStream_
                      : (pwg ? launch_tc_bn<false, true>(BN, pm, bm, a, grid, smem, st)
                             : launch_tc_bn<false, false>(BN, pm, bm, a, grid, smem, st));
     if (s != W4_OK || plan.F == plan.tiles) return s;
-    const long long elems = static_cast<long long>(plan.tiles - plan.F) * BN * kTcBM;
-    launch_pdl(gemm_tail_finalize_kernel, dim3(static_cast<unsigned>((elems + 255) / 256)), dim3(256), 0, st,
+    const long long threads = static_cast<long long>(plan.tiles - plan.F) * BN * (kTcBM / 4);
+    launch_pdl(gemm_tail_finalize_kernel, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0, st,
                static_cast<const float*>(a.part), plan.F, plan.S, plan.tiles - plan.F, plan.tiles_m, BN, p.M, L_out,
                a.bias, a.Y);
     return launch_status();

@@ -101,8 +101,11 @@ size_t w4_workspace_bytes(int M, int N, int K, int transposed);
  * Fused QKV weights (torchao "Add fused QKV HQQ triton_mm test") are just
  * the row-wise concatenation of the Q, K and V packed weights, scales and
  * zeros; they need no special call.
- * M <= 4 runs the CUDA-core GEMV kernels (same results as w4a16_gemv); M > 4
- * runs the tcgen05 tensor-core kernel.
+ * M <= 4 runs the small-batch GEMV kernels (same results as w4a16_gemv);
+ * M > 4 runs the tcgen05 tensor-core kernel, which needs a workspace only
+ * when it splits the tiles of a last partial wave (or of a grid smaller
+ * than the GPU) into k slices: their fp32 partial tiles, added by a second
+ * kernel.  Results do not depend on timing (fixed summation order).
  * Validation: M, N, K > 0; K % 8 == 0; mode/group rules as for
  * w4_quantize_pack; pointers (bias may be NULL) non-NULL and 16-byte
  * aligned; workspace_bytes >= w4_workspace_bytes(M, N, K, transposed).
@@ -115,10 +118,12 @@ w4_status w4a16_gemm(const void *A, int M, int N, int K, const uint32_t *packed,
                      void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * w4a16_gemv -- the small-batch path on CUDA cores (TensorRT-LLM "Modify
- * small-batched weight only quantization": batch <= 4 GEMV bound by global
- * memory loads).  Same arguments and results as w4a16_gemm; M must be 1..4
- * (W4_ERR_INVALID_ARG otherwise).
+ * w4a16_gemv -- the small-batch path (TensorRT-LLM "Modify small-batched
+ * weight only quantization": a batch <= 4 GEMV is bound by global memory
+ * loads): TMA-streamed packed weights whose integer dot products run as
+ * mma.sync u8 x s8 on the tensor pipe, forward and transposed (other group
+ * lengths or K % 32 != 0 fall back to CUDA-core kernels).  Same arguments
+ * and results as w4a16_gemm; M must be 1..4 (W4_ERR_INVALID_ARG otherwise).
  */
 w4_status w4a16_gemv(const void *A, int M, int N, int K, const uint32_t *packed,
                      const void *scales, const void *zeros, int mode, int group_size,
