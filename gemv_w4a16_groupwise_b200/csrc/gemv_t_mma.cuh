@@ -20,16 +20,19 @@
 // (16 packed words of every row, inside one group) and, per stage, issues
 // 8 mma.sync m16n8k32 (u8 x s8 -> s32):
 //   A (16 x 32, u8)  rows are k, columns are the stage's 32 rows.  Lane
-//                    (gid, tig) reads word column 16 w + 8 S + gid of rows
-//                    8 i + 2 tig + h (i < 4, h < 2), transposes the 4 x 4
+//                    (gid, tig) reads word columns 16 w + 2 gid + S (S < 2,
+//                    one 8-byte load) of rows 8 i + 2 tig + h (i < 4,
+//                    h < 2), transposes the 4 x 4
 //                    bytes of each h with byte permutes, and takes byte p of
 //                    the rows: the low nibbles (code 2p, A row gid) and the
 //                    whole bytes q_2p + 16 q_2p+1 (A row gid + 8).
 //                    A column 4 tig + i + 16 h is stage row 8 i + 2 tig + h.
 //   B (32 x 8, s8)   c of the stage's rows for the warp's group in 16-bit
 //                    fixed point, c' = rint(c 2^(140 - e)) with e the
-//                    largest fp32 exponent of c over the CTA's rows (so
-//                    |c'| <= 2^14), split into digits hi = (c' + 128) >> 8
+//                    largest fp32 exponent of c seen so far in the CTA's
+//                    rows (a running value per m; so |c'| <= 2^14; when it
+//                    rises the integer sums so far move into fp32 sums),
+//                    split into digits hi = (c' + 128) >> 8
 //                    and lo = c' - 256 hi; column 2 m + d is digit d of m.
 //                    Lane r of the warp converts stage row r and leaves its
 //                    digits in a per-warp table laid out as the fragments.
@@ -42,7 +45,7 @@
 //     dX[k + 1] = xs (V_gid+8 - V_gid) / 16 - xs sum_n c' z,
 // the last sum kept by the converting lanes.  Row ranges are split over
 // CTAs so that the grid covers the SMs; the fp32 partials of the splits are
-// added (with the bias) by splits_finalize_kernel in a fixed order.
+// added (with the bias) by splits_finalize_vec4_kernel in a fixed order.
 #pragma once
 
 #include "gemv_mma.cuh"
