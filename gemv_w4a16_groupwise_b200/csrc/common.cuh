@@ -52,14 +52,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return r;
 }
 
-__device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
 __device__ __forceinline__ uint32_t ldg_stream_u32(const void* p) {
     uint32_t v;
     asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
@@ -68,15 +60,6 @@ __device__ __forceinline__ uint32_t ldg_stream_u32(const void* p) {
 
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
     return __ffma2_rn(a, b, c);
-}
-
-// Two codes of a packed word as bf16 "magic" values 128 + q: the low half
-// carries code i (bits 4i..4i+3 of w >> (4i)), the high half code i + 4.
-// Returned as the float pair (128 + q_i, 128 + q_{i+4}), both exact.
-template <int I>
-__device__ __forceinline__ float2 magic_pair(uint32_t w) {
-    const uint32_t v = lop3_and_or(w >> (4 * I), 0x000F000Fu, 0x43004300u);
-    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
 
 }  // namespace w4
