@@ -32,7 +32,7 @@ def bf16_to_f64(bits):
 
 
 def assert_close(y_bits, y_ref64, what=""):
-    """Spec tolerance: |y - y_ref| <= 1e-2 rms(y_ref) + 2^-7 |y_ref| per element."""
+    """The parity tolerance: |y - y_ref| <= 1e-2 rms(y_ref) + 2^-7 |y_ref| per element."""
     y = bf16_to_f64(y_bits)
     ref = np.asarray(y_ref64, dtype=np.float64)
     assert y.shape == ref.shape, (y.shape, ref.shape)
