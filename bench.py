@@ -539,9 +539,7 @@ def run_ours(args):
                 "traffic": (round(traffic / calls) if traffic is not None else None),
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
                                else "fallback 6.65 TB/s",
-                "kernel": "gemv_mma_kernel, timed together with the gemv_xfrag_kernel prep that "
-                          "shapes with a large activation block launch before it "
-                          "(one GEMV call = 1 or 2 launches)",
+                "kernel": "gemv_q8_kernel (one launch per GEMV call in this sweep: no shape splits K)",
                 "per": "GEMV call, averaged over the 40 calls of a step (CUDA events on the launching "
                        "stream around the whole timed region)",
                 "alg_bytes_per_launch": round(alg_per_call),

@@ -12,8 +12,8 @@ Entry points (same names as the C ABI in ``include/w4a16.h``):
   fp16 scales and zeros
 * :func:`w4a16_gemm` -- Y = X . dequant(W)^T (or dX = dY . dequant(W) with
   ``transposed=True``), optional bias
-* :func:`w4a16_gemv` -- the same for M <= 4 (TMA-streamed weights, integer
-  dot products on the tensor pipe)
+* :func:`w4a16_gemv` -- the same for M <= 4 (TMA-streamed weights, exact
+  products on the tensor pipe, fp32 sums)
 * :func:`w4_workspace_bytes`, :func:`w4_device_error`
 """
 from __future__ import annotations
@@ -188,8 +188,8 @@ def w4a16_gemm(A, packed, scales, zeros, mode="groupwise", group_size: int = 128
 
 def w4a16_gemv(A, packed, scales, zeros, mode="groupwise", group_size: int = 128, *, N: int,
                K: int, bias=None, transposed: bool = False, out=None):
-    """Small-batch (M <= 4) path of :func:`w4a16_gemm`: TMA-streamed weights, integer
-    dot products on the tensor pipe (mma.sync u8 x s8), forward and transposed."""
+    """Small-batch (M <= 4) path of :func:`w4a16_gemm`: TMA-streamed weights, exact
+    products on the tensor pipe with fp32 sums, forward and transposed."""
     return _matmul("w4a16_gemv", A, packed, scales, zeros, mode, group_size, N, K, bias,
                    transposed, out)
 

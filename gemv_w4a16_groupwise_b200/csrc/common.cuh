@@ -58,6 +58,10 @@ __device__ __forceinline__ uint32_t ldg_stream_u32(const void* p) {
     return v;
 }
 
+__device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) {
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
     return __ffma2_rn(a, b, c);
 }

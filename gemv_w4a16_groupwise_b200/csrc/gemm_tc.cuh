@@ -133,10 +133,6 @@ __device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t (&r)[8]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) {
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
 // Eight codes of one packed word -> eight bf16 (q - z) * s in k order.
 __device__ __forceinline__ uint4 dequant_word_bf16(uint32_t w, float s, float c_lo, float c_hi) {
     const uint32_t l16 = w << 16, l8 = w << 8, r8 = w >> 8, r16 = w >> 16;

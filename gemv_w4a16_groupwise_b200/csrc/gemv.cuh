@@ -1,9 +1,7 @@
-// CUDA-core pieces of the small-batch (M <= 4) W4A16 products that the
-// streaming GEMV kernels share, plus the kernels that cover what they do
-// not:
+// CUDA-core pieces of the small-batch (M <= 4) W4A16 products: the kernels
+// that cover what the tensor-pipe GEMV kernels do not take, and the split
+// finalize they share:
 //
-//  * helpers for the integer dot products (dp4a with unsigned codes and
-//    signed / unsigned activation bytes, bf16 exponent extraction);
 //  * gemv_fwd_simple_kernel: the forward product for shapes the streaming
 //    kernels do not take (K or the group length not a multiple of 32): one
 //    warp per output row, lanes along K, plain fp32 arithmetic;
@@ -12,8 +10,8 @@
 //  * gemv_t_kernel: the transposed product dX = dY . dequant(W) for M <= 4
 //    on shapes the tensor-pipe kernel does not take.
 //
-// The forward GEMV proper is in gemv_stream.cuh (CUDA cores) and
-// gemv_mma.cuh (tensor pipe); the transposed one in gemv_t_mma.cuh.
+// The forward GEMV proper is in gemv_q8.cuh and gemv_mma.cuh (tensor pipe);
+// the transposed one in gemv_t_mma.cuh.
 #pragma once
 
 #include "tma.cuh"
@@ -30,24 +28,6 @@ struct GemvFwdArgs {
     int N, K, g, G, sz_row;  // group of (n, k): n * sz_row + min(k / g, G - 1)
 };
 
-// dp4a with unsigned codes and signed / unsigned activation bytes
-__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
-    int d;
-    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-__device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t d;
-    asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-
-// Biased exponent of a bf16 (1 for zero and subnormals) and its significand
-// with the implicit bit: value = mant * 2^(e - 134).
-__device__ __forceinline__ int bf16_exp1(uint32_t b) {
-    const int e = (b >> 7) & 0xFF;
-    return e ? e : 1;
-}
 __device__ __forceinline__ float half_to_float_ldg(const __half* p) {
     return __half2float(__ldg(p));
 }
@@ -192,13 +172,15 @@ __global__ void __launch_bounds__(256) gemv_fwd_simple_kernel(const GemvFwdArgs 
 
 // ---------------------------------------------------------------------------
 // Transposed GEMV: dX[m, k] = sum_n dY[m, n] * w_hat[n, k]  (M <= 4)
-// ("Re-write HQQ Fused Gemm Transpose": same packed W, scales and zeros).
-// Lanes own two consecutive packed words (16 k) of a row, so a warp reads
-// 256 contiguous bytes of each row it visits; the 8 warps of a CTA take
-// interleaved rows of the CTA's row range and meet in shared memory.  With
-// c = dY[m, n] * s:   sum_n c (q - z) = sum_n c (off + q) - sum_n c (off + z)
-// so per word only sum_n c and sum_n c z are kept besides the 16 products.
-// Row ranges are split over CTAs; fp32 partials go to the workspace.
+// ("Re-write HQQ Fused Gemm Transpose": same packed W, scales and zeros), for
+// the shapes the tensor-pipe kernel does not take.  Lanes own two
+// consecutive packed words (16 k) of a row, so a warp reads 256 contiguous
+// bytes of each row it visits; the 4 warps of a CTA take interleaved rows of
+// the CTA's row range and meet in shared memory.  Per code the lane forms
+// (q - z) exactly ((2^23 + q) - (2^23 + z) in fp32) and multiplies it by
+// c = dY[m, n] s (exact: 8 x 11 significant bits) in an fp32 fma, so every
+// product is exact and the sums are fp32.  Row ranges are split over CTAs;
+// fp32 partials go to the workspace.
 // ---------------------------------------------------------------------------
 struct GemvTArgs {
     const uint16_t* dY;      // [M, N] bf16
@@ -230,70 +212,39 @@ __global__ void __launch_bounds__(kGemvTThreads)
     const int grp1 = has1 ? min((8 * (j0 + 1)) / a.g, a.G - 1) : 0;
 
     float acc[M][16];
-    float csum[M][2], czsum[M][2];
-#pragma unroll
-    for (int m = 0; m < M; ++m) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) acc[m][e] = 0.0f;
-        csum[m][0] = csum[m][1] = czsum[m][0] = czsum[m][1] = 0.0f;
-    }
-
-    for (int n = r0 + warp; n < r1; n += kGemvTThreads / 32) {
-        const uint32_t* rowp = a.packed + static_cast<size_t>(n) * W8;
-        const uint32_t w0 = has0 ? ldg_stream_u32(rowp + j0) : 0u;
-        const uint32_t w1 = has1 ? ldg_stream_u32(rowp + j0 + 1) : 0u;
-        const float s0 = half_to_float_ldg(a.S + n * a.sz_row + grp0);
-        const float z0 = half_to_float_ldg(a.Z + n * a.sz_row + grp0);
-        const float s1 = half_to_float_ldg(a.S + n * a.sz_row + grp1);
-        const float z1 = half_to_float_ldg(a.Z + n * a.sz_row + grp1);
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-            const float d = bf16_bits_to_float(__ldg(a.dY + static_cast<size_t>(m) * a.N + n));
-            const float c0 = d * s0, c1 = d * s1;
-            csum[m][0] += c0;
-            csum[m][1] += c1;
-            czsum[m][0] = fmaf(c0, z0, czsum[m][0]);
-            czsum[m][1] = fmaf(c1, z1, czsum[m][1]);
-            const float2 cc0 = make_float2(c0, c0), cc1 = make_float2(c1, c1);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t w = h ? w1 : w0;
-                const float2 cc = h ? cc1 : cc0;
-                const uint32_t r8 = w >> 8, l8 = w << 8;
-                // (q3,q4) (q5,q6) (q1,q2) (q0,q7) as (off + q) magic pairs
-                const float2 p0 = make_float2(__uint_as_float(lop3_and_or(w, 0xF000u, 0x45000000u)),
-                                              __uint_as_float(lop3_and_or(w, 0xF0000u, 0x43000000u)));
-                const float2 p1 = make_float2(__uint_as_float(lop3_and_or(r8, 0xF000u, 0x45000000u)),
-                                              __uint_as_float(lop3_and_or(r8, 0xF0000u, 0x43000000u)));
-                const float2 p2 = make_float2(__uint_as_float(lop3_and_or(l8, 0xF000u, 0x45000000u)),
-                                              __uint_as_float(lop3_and_or(l8, 0xF0000u, 0x43000000u)));
-                const float2 p3 =
-                    make_float2(__uint_as_float(lop3_and_or(w << 16, 0xF0000u, 0x43000000u)),
-                                __uint_as_float(lop3_and_or(w >> 16, 0xF000u, 0x45000000u)));
-                float2* A = reinterpret_cast<float2*>(&acc[m][8 * h]);
-                A[0] = ffma2(p0, cc, A[0]);  // k3, k4
-                A[1] = ffma2(p1, cc, A[1]);  // k5, k6
-                A[2] = ffma2(p2, cc, A[2]);  // k1, k2
-                A[3] = ffma2(p3, cc, A[3]);  // k0, k7
-            }
-        }
-    }
-
-    // slot order inside acc[m][8h + slot]: k3,k4,k5,k6,k1,k2,k0,k7 ; offsets
-    // 2048 for odd k, 128 for even k
 #pragma unroll
     for (int m = 0; m < M; ++m)
 #pragma unroll
+        for (int e = 0; e < 16; ++e) acc[m][e] = 0.0f;
+
+    for (int n = r0 + warp; n < r1; n += kGemvTThreads / 32) {
+        const uint32_t* rowp = a.packed + static_cast<size_t>(n) * W8;
+        const uint32_t w[2] = {has0 ? ldg_stream_u32(rowp + j0) : 0u, has1 ? ldg_stream_u32(rowp + j0 + 1) : 0u};
+        const float s[2] = {half_to_float_ldg(a.S + n * a.sz_row + grp0), half_to_float_ldg(a.S + n * a.sz_row + grp1)};
+        // 2^23 + z, so that (2^23 + q) - (2^23 + z) = q - z exactly
+        const float zo[2] = {8388608.0f + half_to_float_ldg(a.Z + n * a.sz_row + grp0),
+                             8388608.0f + half_to_float_ldg(a.Z + n * a.sz_row + grp1)};
+        float qz[16];
+#pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int slot = 0; slot < 8; ++slot) {
-                const int e = (0x70216543 >> (4 * slot)) & 7;  // k offset of the slot
-                const float off = (e & 1) ? 2048.0f : 128.0f;
-                const float v = acc[m][8 * h + slot] - fmaf(off, csum[m][h], czsum[m][h]);
-                red[warp][m][8 * h + e][lane] = v;
-            }
+            for (int e = 0; e < 8; ++e)
+                qz[8 * h + e] = __uint_as_float(0x4B000000u | ((w[h] >> (4 * e)) & 0xFu)) - zo[h];
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const float d = bf16_bits_to_float(__ldg(a.dY + static_cast<size_t>(m) * a.N + n));
+            const float c[2] = {d * s[0], d * s[1]};
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc[m][e] = fmaf(c[e >> 3], qz[e], acc[m][e]);
+        }
+    }
+
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+#pragma unroll
+        for (int e = 0; e < 16; ++e) red[warp][m][e][lane] = acc[m][e];
     __syncthreads();
-    // warps 0..M-1 each finish one m; lanes cover the 16 k of one lane-slot
+    // the warps' sums in warp order; lanes cover the 16 k of one lane-slot
     for (int o = threadIdx.x; o < M * 16 * 32; o += kGemvTThreads) {
         const int m = o / (16 * 32);
         const int rem = o - m * 16 * 32;

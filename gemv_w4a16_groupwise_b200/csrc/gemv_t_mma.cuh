@@ -1,66 +1,63 @@
-// Transposed GEMV for M <= 4 with its integer dot products on the tensor
-// pipe (the fine-tuning backward from the same packed tensors, "Re-write
-// HQQ Fused Gemm Transpose": dX = dY . dequant(W), no repack, no reshaped
-// scales or zeros):
-//     dX[m, k] = sum_n c[m, n, g(k)] (q[n, k] - z[n, g(k)]),
-//     c[m, n, g] = dY[m, n] s[n, g].
+// Transposed GEMV for M <= 4 on the tensor pipe (the fine-tuning backward
+// from the same packed tensors, "Re-write HQQ Fused Gemm Transpose":
+// dX = dY . dequant(W), no repack, no reshaped scales or zeros):
+//     dX[m, k] = sum_n c[m, n] (q[n, k] - z[n, g(k)]),   c[m, n] = dY[m, n] s[n, g(k)].
+//
+// Exact operands.  c is the fp32 product of a bf16 and an fp16 (at most 19
+// significant bits), so it is exactly the sum of three bf16 parts
+// c = c0 + c1 + c2 (c0 = bf16(c), c1 = bf16(c - c0), c2 = c - c0 - c1); the
+// codes enter as exact bf16 (q - z), unpacked from the packed words with one
+// AND-OR (the bf16 pair (128 + q, 128 + q')) and one bf16x2 subtraction of
+// (128 + z, 128 + z').  The mma (m16n8k16, bf16 x bf16 -> fp32) then forms
+// every product exactly and accumulates in fp32; the three parts are
+// separate columns, added once at the end.
 //
 // The reduction runs over weight rows, while a packed word holds 8
-// consecutive k of one row, so the codes are transposed in registers:
+// consecutive k of one row, so the codes are transposed on the way in.
 //
-// Stream.  Each CTA owns a strip of 2048 k (1 KB of every row) and a range
-// of rows.  A producer warp brings the range 32 rows at a time into a
-// CTA-wide ring: one TMA box of 32 rows x 1040 bytes (the packed words seen
-// as 8-byte elements, 130 per row: the strip's 1 KB and the next 16 bytes,
-// which no warp reads), so that rows sit 1040 bytes apart and the words
-// that one load instruction of a warp reads fall into 32 different banks;
-// plus TMA boxes of the 32 rows' scales and zeros.
+// Stream.  Each CTA owns a strip of 16 KW k and a range of rows.  A
+// producer warp brings the range 32 rows at a time into a CTA-wide ring: one
+// TMA box of 32 rows x (8 KW + 16) bytes (the packed words seen as 8-byte
+// elements: the strip's bytes and the next 16, which no warp reads), plus
+// TMA boxes of the 32 rows' scales and zeros.
 //
-// Arithmetic.  Consumer warp w owns k = 128 w .. 128 w + 127 of the strip
-// (16 packed words of every row, inside one group) and, per stage, issues
-// 8 mma.sync m16n8k32 (u8 x s8 -> s32):
-//   A (16 x 32, u8)  rows are k, columns are the stage's 32 rows.  Lane
-//                    (gid, tig) reads word columns 16 w + 2 gid + S (S < 2,
-//                    one 8-byte load) of rows 8 i + 2 tig + h (i < 4,
-//                    h < 2), transposes the 4 x 4
-//                    bytes of each h with byte permutes, and takes byte p of
-//                    the rows: the low nibbles (code 2p, A row gid) and the
-//                    whole bytes q_2p + 16 q_2p+1 (A row gid + 8).
-//                    A column 4 tig + i + 16 h is stage row 8 i + 2 tig + h.
-//   B (32 x 8, s8)   c of the stage's rows for the warp's group in 16-bit
-//                    fixed point, c' = rint(c 2^(140 - e)) with e the
-//                    largest fp32 exponent of c seen so far in the CTA's
-//                    rows (a running value per m; so |c'| <= 2^14; when it
-//                    rises the integer sums so far move into fp32 sums),
-//                    split into digits hi = (c' + 128) >> 8
-//                    and lo = c' - 256 hi; column 2 m + d is digit d of m.
-//                    Lane r of the warp converts stage row r and leaves its
-//                    digits in a per-warp table laid out as the fragments.
-//   D (16 x 8, s32)  accumulates over stages: lane (gid, tig) holds, for
-//                    m = tig, the two digit sums of k = 8 col + 2p (row gid)
-//                    and of the whole bytes (row gid + 8), whose difference
-//                    is 16 x the sums of k + 1.
-// At the end, with xs = 2^(e - 140) and V = 256 D_hi + D_lo per row,
-//     dX[k] = xs V_gid - xs sum_n c' z,
-//     dX[k + 1] = xs (V_gid+8 - V_gid) / 16 - xs sum_n c' z,
-// the last sum kept by the converting lanes.  Row ranges are split over
-// CTAs so that the grid covers the SMs; the fp32 partials of the splits are
-// added (with the bias) by splits_finalize_vec4_kernel in a fixed order.
+// Arithmetic.  Consumer warp w owns k = KW w .. KW w + KW - 1 of the strip
+// (inside one group: KW divides the group length).  Per stage and n-tile t
+// (stage rows 16 t .. 16 t + 15) the mma's 16 reduction columns are the rows
+// 16 t + 4 tig + {0, 1} (register pair 0) and + {2, 3} (pair 1) of lane
+// (gid, tig); its 16 k-rows are, for tile j, k-row gid = nibble j % 4 of the
+// lane's word j / 4 (words 2 gid, 2 gid + 1 of the warp's KW k when KW =
+// 128; word gid when KW = 64) and k-row gid + 8 = nibble j % 4 + 4 of the
+// same word.  So a lane reads one (or two) words of four rows, pairs the rows
+// with one byte permute each, and every (shift, AND-OR, subtract) yields one
+// A register: no codes move between lanes.  B is (c0, c1, c2) of each
+// activation row: columns 3 m' + p of set m / 2 (m' = m % 2), written by the
+// lane that converts stage row r into a per-warp table laid out as the B
+// fragments.  Accumulators stay in registers across all the CTA's stages.
+//
+// At the end a lane adds the three parts of each of its columns with one
+// shuffle, and the lanes holding whole rows write 16 (or 8) consecutive dX,
+// or fp32 partials when the rows are split over CTAs (added, with the bias,
+// by splits_finalize_vec4_kernel in a fixed order).
 #pragma once
 
-#include "gemv_mma.cuh"
+#include "gemv_q8.cuh"
 
 namespace w4 {
 
 constexpr int kTMW = 16;                          // consumer warps
 constexpr int kTMThreads = (kTMW + 1) * 32;       // + the producer warp
 constexpr int kTMRows = 32;                       // weight rows per stage
-constexpr int kTMStrip = 2048;                    // k per CTA strip
-constexpr int kTMPitch = 1040;                    // bytes per row slot: 1 KB of words + 16
-constexpr int kTMBoxX = kTMPitch / 8;             // box width in 8-byte elements
-constexpr int kTMSzOff = kTMRows * kTMPitch;      // scale box, then the zero box 1 KB later
-constexpr int kTMStageBytes = kTMSzOff + 2 * 1024;
-constexpr int kTMTabBytes = 256;                  // per consumer warp: [digit][m][h][tig][i] bytes
+
+// Geometry for a warp k-width KW (128 or 64): strip 16 KW k; a stage row is
+// the strip's 8 KW bytes plus 16.
+__host__ __device__ constexpr int tm_strip(int KW) { return kTMW * KW; }
+__host__ __device__ constexpr int tm_pitch(int KW) { return kTMW * KW / 2 + 16; }
+__host__ __device__ constexpr int tm_sz_off(int KW) { return kTMRows * tm_pitch(KW); }
+__host__ __device__ constexpr int tm_stage_bytes(int KW) { return tm_sz_off(KW) + 2 * 1024; }
+// per warp: B table [set][n-tile][register][lane] u32, then (128 + z) of the
+// stage's rows as bf16
+__host__ __device__ constexpr int tm_tab_bytes(int nset) { return nset * 2 * 2 * 32 * 4 + kTMRows * 2; }
 
 struct GemvTMmaArgs {
     const uint16_t* dY;      // [M, N] bf16
@@ -71,50 +68,45 @@ struct GemvTMmaArgs {
     uint16_t* dX;            // [M, K] bf16
     float* partial;          // [splits, M, K] when splits > 1
     int N, K, g, G, sz_row;
-    int strips;              // ceil(K / 2048)
+    int strips;              // ceil(K / strip)
     int splits;              // row ranges
     int rows_per_split;      // a multiple of 32
     int stages;
 };
 
-// Ring, the warps' digit tables, dY of the split's rows (one float4 per
-// row), barriers and the abort flag.
-__host__ __device__ inline size_t gemv_t_mma_smem_bytes(int stages, int rows_per_split) {
-    return 1024 + static_cast<size_t>(stages) * kTMStageBytes + kTMW * kTMTabBytes +
+// Ring, the warps' tables, dY of the split's rows (one float4 per row),
+// barriers and the abort flag.
+__host__ __device__ inline size_t gemv_t_mma_smem_bytes(int KW, int nset, int stages, int rows_per_split) {
+    return 1024 + static_cast<size_t>(stages) * tm_stage_bytes(KW) + kTMW * tm_tab_bytes(nset) +
            static_cast<size_t>(rows_per_split) * 16 + static_cast<size_t>(stages) * 16 + 16;
 }
 
-// Bytes i of the four words, for i = 0..3: x[i] = {w0.i, w1.i, w2.i, w3.i}.
-__device__ __forceinline__ void transpose_bytes4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
-                                                 uint32_t (&x)[4]) {
-    const uint32_t t0 = prmt(w0, w1, 0x5140u), t1 = prmt(w0, w1, 0x7362u);
-    const uint32_t t2 = prmt(w2, w3, 0x5140u), t3 = prmt(w2, w3, 0x7362u);
-    x[0] = prmt(t0, t2, 0x5410u);
-    x[1] = prmt(t0, t2, 0x7632u);
-    x[2] = prmt(t1, t3, 0x5410u);
-    x[3] = prmt(t1, t3, 0x7632u);
-}
-
-template <int M, int SZ>
+template <int M, int KW, int SZ>
 __global__ void __launch_bounds__(kTMThreads, 1)
     gemv_t_mma_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                       const __grid_constant__ CUtensorMap zmap, const GemvTMmaArgs a) {
     static_assert(M >= 1 && M <= 4, "M");
+    static_assert(KW == 128 || KW == 64, "KW");
     static_assert(SZ == kSzConst || SZ == kSzTma2d || SZ == kSzTma1d, "scale / zero path");
+    constexpr int NSET = (M + 1) / 2;
+    constexpr int NT = KW / 16;                   // k-tiles per warp
+    constexpr int NWD = KW / 64;                  // packed words per row and lane
+    constexpr int kStrip = tm_strip(KW), kPitch = tm_pitch(KW), kSzOff = tm_sz_off(KW);
+    constexpr int kStage = tm_stage_bytes(KW), kTab = tm_tab_bytes(NSET);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int NS = a.stages;
     constexpr uint32_t kSzTx = SZ == kSzTma2d ? 2 * kTMRows * 16 * 2 : SZ == kSzTma1d ? 2 * kTMRows * 2 : 0;
-    uint8_t* ring = base;                                                        // [stage][kTMStageBytes]
-    uint8_t* tabs = ring + NS * kTMStageBytes;                                   // [warp][256]
-    float4* dys = reinterpret_cast<float4*>(tabs + kTMW * kTMTabBytes);          // [row of the split]
+    uint8_t* ring = base;                                                        // [stage][kStage]
+    uint8_t* tabs = ring + NS * kStage;                                          // [warp][kTab]
+    float4* dys = reinterpret_cast<float4*>(tabs + kTMW * kTab);                 // [row of the split]
     uint64_t* full = reinterpret_cast<uint64_t*>(dys + a.rows_per_split);
     uint64_t* empty = full + NS;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NS);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const int strip = blockIdx.x % a.strips, split = blockIdx.x / a.strips;
-    const int k0 = strip * kTMStrip;
+    const int k0 = strip * kStrip;
     const int r0 = split * a.rows_per_split;
     const int r1 = min(a.N, r0 + a.rows_per_split);
     const int nst = r1 > r0 ? (r1 - r0 + kTMRows - 1) / kTMRows : 0;
@@ -136,6 +128,8 @@ __global__ void __launch_bounds__(kTMThreads, 1)
             tma_prefetch_desc(&zmap);
         }
     }
+    // the B tables start at zero: columns no activation row uses stay zero
+    for (int i = threadIdx.x; i < kTMW * kTab / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(tabs)[i] = 0u;
     __syncthreads();
     // launched as a programmatic dependent: let the finalize launch, then
     // wait for the work before this kernel before reading any input
@@ -154,16 +148,16 @@ __global__ void __launch_bounds__(kTMThreads, 1)
                                                                           kErrTimeoutEmpty));
                 if (!ok) break;
             }
-            uint8_t* sd = ring + s * kTMStageBytes;
+            uint8_t* sd = ring + s * kStage;
             const int row0 = r0 + b * kTMRows;
             if (SZ == kSzTma2d)
-                tma_issue_elected<3>(&full[s], kTMRows * kTMPitch + kSzTx, sd, &wmap, k0 / 16, row0,
-                                     sd + kTMSzOff, &smap, x_sz, row0, sd + kTMSzOff + 1024, &zmap, x_sz, row0);
+                tma_issue_elected<3>(&full[s], kTMRows * kPitch + kSzTx, sd, &wmap, k0 / 16, row0, sd + kSzOff,
+                                     &smap, x_sz, row0, sd + kSzOff + 1024, &zmap, x_sz, row0);
             else if (SZ == kSzTma1d)
-                tma_issue_elected<3>(&full[s], kTMRows * kTMPitch + kSzTx, sd, &wmap, k0 / 16, row0,
-                                     sd + kTMSzOff, &smap, row0, 0, sd + kTMSzOff + 1024, &zmap, row0, 0);
+                tma_issue_elected<3>(&full[s], kTMRows * kPitch + kSzTx, sd, &wmap, k0 / 16, row0, sd + kSzOff,
+                                     &smap, row0, 0, sd + kSzOff + 1024, &zmap, row0, 0);
             else
-                tma_issue_elected<1>(&full[s], kTMRows * kTMPitch, sd, &wmap, k0 / 16, row0);
+                tma_issue_elected<1>(&full[s], kTMRows * kPitch, sd, &wmap, k0 / 16, row0);
             if (++s == NS) {
                 s = 0;
                 ++round;
@@ -172,7 +166,7 @@ __global__ void __launch_bounds__(kTMThreads, 1)
     } else {
         // ------------------------------------------------ consumers
         const int gid = lane >> 2, tig = lane & 3;
-        const int kw = k0 + 128 * warp;                  // the warp's first k
+        const int kw = k0 + KW * warp;                   // the warp's first k
         const int grp = group_of(min(kw, a.K - 1));
         float s_const = 0.f, z_const = 0.f;
         if (SZ == kSzConst) {
@@ -191,56 +185,20 @@ __global__ void __launch_bounds__(kTMThreads, 1)
             dys[r] = make_float4(v[0], v[1], v[2], v[3]);
         }
         named_barrier_sync(1, kTMW * 32);
-        // Running exponents: E[m] is the largest fp32 exponent of c seen so
-        // far (at least 14), c' = rint(c 2^(140 - E)), and the integer sums
-        // in acc are in units of xs = 2^(E - 140).  When a stage raises E[m],
-        // the lanes of m first move acc into the fp32 sums fac (in units of
-        // the old xs) and clear it, and every lane rescales its sum of c' z.
-        // The precision of c' is never below that of one exponent for all
-        // of the CTA's rows.
-        // thr[m] = 2^(E[m] - 126): |c| >= thr[m] means an exponent above E[m];
-        // from its bits, 2^(140 - E) = bits 0x86000000 - thr and
-        // 2^(E - 140) = bits thr - 0x07000000
-        float thr[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) thr[m] = __int_as_float((14 + 1) << 23);
-        auto xs_of = [](float th) { return __int_as_float(__float_as_int(th) - 0x07000000); };
-        // this lane's stage row r = 8 i + 2 t + h and its table bytes
-        const int ti = lane >> 3, tt = (lane >> 1) & 3, th = lane & 1;
-        uint8_t* tab = tabs + warp * kTMTabBytes;
-        const int tbyte = th * 16 + tt * 4 + ti;         // + (d * 4 + m) * 32
+        uint8_t* tab = tabs + warp * kTab;
+        uint16_t* tab16 = reinterpret_cast<uint16_t*>(tab);
         const uint32_t* tabw = reinterpret_cast<const uint32_t*>(tab);
-        const int bsel = ((gid & 1) * 4 + (gid >> 1)) * 8 + tig;   // word of b0; b1 is 4 words on
-        float zt[4] = {0.f, 0.f, 0.f, 0.f};
-        int acc[2][4][4];
-        float fac[2][4][2];
+        uint16_t* zzt = reinterpret_cast<uint16_t*>(tab + NSET * 2 * 2 * 32 * 4);
+        // the converting lane's stage row r = lane: its place in the B fragments
+        const int ct = lane >> 4, rr = lane & 15;
+        const int bt = rr >> 2, breg = (rr & 3) >> 1, bhalf = rr & 1;
+        float acc[NSET][NT][4];
 #pragma unroll
-        for (int S = 0; S < 2; ++S)
+        for (int st = 0; st < NSET; ++st)
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[S][p][j] = 0;
-                fac[S][p][0] = fac[S][p][1] = 0.f;
-            }
-        // acc (units xs) -> fac, for the lane's m = tig: rows gid carry the
-        // even codes q_e, rows gid + 8 whole bytes q_e + 16 q_o
-        auto fold = [&](float x) {
-            const float x16 = x * 0.0625f;
-#pragma unroll
-            for (int S = 0; S < 2; ++S)
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const float ve = fmaf(256.0f, static_cast<float>(acc[S][p][0]), static_cast<float>(acc[S][p][1]));
-                    const float vb = fmaf(256.0f, static_cast<float>(acc[S][p][2]), static_cast<float>(acc[S][p][3]));
-                    fac[S][p][0] = fmaf(ve, x, fac[S][p][0]);
-                    fac[S][p][1] = fmaf(vb - ve, x16, fac[S][p][1]);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[S][p][j] = 0;
-                }
-        };
-        auto pick = [&](const auto (&v)[4]) { return tig == 0 ? v[0] : tig == 1 ? v[1] : tig == 2 ? v[2] : v[3]; };
-        // word pair (columns 16 w + 2 gid, + 1) of rows 8 i + 2 tig + h
-        const uint32_t col0 = static_cast<uint32_t>((16 * warp + 2 * gid) * 4 + (2 * tig) * kTMPitch);
+            for (int j = 0; j < NT; ++j) acc[st][j][0] = acc[st][j][1] = acc[st][j][2] = acc[st][j][3] = 0.f;
+        // this lane's words: (2 gid, 2 gid + 1) or gid of the warp's KW k
+        const int wbyte = KW * warp / 2 + (NWD == 2 ? 8 * gid : 4 * gid);
 
         int s = 0;
         uint32_t phase = 0;
@@ -248,126 +206,141 @@ __global__ void __launch_bounds__(kTMThreads, 1)
             const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[s], phase, abort_flag,
                                                                       kErrTimeoutTmaFull));
             if (!ok) break;
-            const uint8_t* sb = ring + s * kTMStageBytes;
+            const uint8_t* sb = ring + s * kStage;
             // ---- this lane's code words first, so that their latency overlaps
-            // the digits: words 2 gid (S = 0) and 2 gid + 1 (S = 1) of the
-            // warp's 16, rows 8 i + 2 tig + h
-            uint2 w[2][4];
+            // the conversion: rows 16 t + 4 tig + i
+            uint32_t wv[2][4][NWD];
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+            for (int t = 0; t < 2; ++t)
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    w[h][i] = *reinterpret_cast<const uint2*>(sb + col0 + (8 * i + h) * kTMPitch);
-            // ---- digits of c for stage row `lane` and the warp's group
+                for (int i = 0; i < 4; ++i) {
+                    const uint8_t* p = sb + (16 * t + 4 * tig + i) * kPitch + wbyte;
+                    if (NWD == 2) {
+                        const uint2 w2 = *reinterpret_cast<const uint2*>(p);
+                        wv[t][i][0] = w2.x;
+                        wv[t][i][NWD - 1] = w2.y;
+                    } else {
+                        wv[t][i][0] = *reinterpret_cast<const uint32_t*>(p);
+                    }
+                }
+            // ---- stage row `lane`: (c0, c1, c2) of each activation row into
+            // the B table, (128 + z) into the zero table
             {
                 float sv, zv;
                 if (SZ == kSzConst) {
                     sv = s_const;
                     zv = z_const;
                 } else if (SZ == kSzTma2d) {
-                    const __half* sh = reinterpret_cast<const __half*>(sb + kTMSzOff);
+                    const __half* sh = reinterpret_cast<const __half*>(sb + kSzOff);
                     sv = __half2float(sh[lane * 16 + grp - x_sz]);
                     zv = __half2float(sh[512 + lane * 16 + grp - x_sz]);
                 } else {
-                    const __half* sh = reinterpret_cast<const __half*>(sb + kTMSzOff);
+                    const __half* sh = reinterpret_cast<const __half*>(sb + kSzOff);
                     sv = __half2float(sh[lane]);
                     zv = __half2float(sh[512 + lane]);
                 }
                 const float4 d4 = dys[b * kTMRows + lane];
-                const float c[4] = {d4.x * sv, d4.y * sv, d4.z * sv, d4.w * sv};
-                const bool up = fabsf(c[0]) >= thr[0] || fabsf(c[1]) >= thr[1] || fabsf(c[2]) >= thr[2] ||
-                                fabsf(c[3]) >= thr[3];
-                if (__any_sync(0xFFFFFFFFu, up)) {              // rare: an exponent rises
-                    float tn[4];
+                const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+                __syncwarp();                              // the last stage's table reads are done
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const int e = min(static_cast<int>(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(c[m]) & 0x7FFFFFFFu) >> 23),
-                                          254);
-                        tn[m] = fmaxf(thr[m], __int_as_float((e + 1) << 23));
-                    }
-                    if (pick(tn) > pick(thr)) fold(xs_of(pick(thr)));
+                for (int m = 0; m < M; ++m) {
+                    const float c = dv[m] * sv;            // exact: 8 x 11 significant bits
+                    const __nv_bfloat16 p0 = __float2bfloat16_rn(c);
+                    const float q1 = c - __bfloat162float(p0);
+                    const __nv_bfloat16 p1 = __float2bfloat16_rn(q1);
+                    const __nv_bfloat16 p2 = __float2bfloat16_rn(q1 - __bfloat162float(p1));
+                    const __nv_bfloat16 pv[3] = {p0, p1, p2};
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        // 2^(E_old - E_new) from the exponent fields (thr may
-                        // be +inf, the bits of E = 254), or 0 below 2^-126
-                        const int f = 127 + ((__float_as_int(thr[m]) - __float_as_int(tn[m])) >> 23);
-                        zt[m] *= f > 0 ? __int_as_float(f << 23) : 0.0f;
-                        thr[m] = tn[m];
+                    for (int p = 0; p < 3; ++p) {
+                        const int col = 3 * (m & 1) + p;
+                        const int idx = ((((m >> 1) * 2 + ct) * 2 + breg) * 32 + col * 4 + bt) * 2 + bhalf;
+                        tab16[idx] = __bfloat16_as_ushort(pv[p]);
                     }
                 }
+                zzt[lane] = __bfloat16_as_ushort(__float2bfloat16_rn(128.0f + zv));
+                __syncwarp();
+            }
+            // ---- the mma: per n-tile, pairs (rows 4 tig, 4 tig + 1) and (+2, +3)
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    // t = 1.5 * 2^23 + c' with c' = rint(c 2^(140 - E)), |c'| <= 2^14,
-                    // in one rounding; the bit pattern of t is 0x4B400000 + c', so
-                    // its low byte is the low digit lo = c' - 256 hi (as a signed
-                    // byte) and byte 1 of bits + 128 is hi = (c' + 128) >> 8
-                    const float t = fmaf(c[m], __int_as_float(0x86000000 - __float_as_int(thr[m])), 12582912.0f);
-                    const uint32_t tb = __float_as_uint(t);
-                    tab[m * 32 + tbyte] = static_cast<uint8_t>((tb + 128u) >> 8);
-                    tab[(4 + m) * 32 + tbyte] = static_cast<uint8_t>(tb);
-                    zt[m] = fmaf(t - 12582912.0f, zv, zt[m]);
+            for (int t = 0; t < 2; ++t) {
+                uint32_t bq[NSET][2];
+#pragma unroll
+                for (int st = 0; st < NSET; ++st) {
+                    bq[st][0] = tabw[((st * 2 + t) * 2 + 0) * 32 + lane];
+                    bq[st][1] = tabw[((st * 2 + t) * 2 + 1) * 32 + lane];
+                }
+                const uint32_t zab = *reinterpret_cast<const uint32_t*>(zzt + 16 * t + 4 * tig);
+                const uint32_t zcd = *reinterpret_cast<const uint32_t*>(zzt + 16 * t + 4 * tig + 2);
+#pragma unroll
+                for (int wd = 0; wd < NWD; ++wd) {
+                    // nibbles 0..3 of rows (A, B) as bf16 pairs in u, 4..7 in v
+                    const uint32_t uab = prmt(wv[t][0][wd], wv[t][1][wd], 0x5410u);
+                    const uint32_t vab = prmt(wv[t][0][wd], wv[t][1][wd], 0x7632u);
+                    const uint32_t ucd = prmt(wv[t][2][wd], wv[t][3][wd], 0x5410u);
+                    const uint32_t vcd = prmt(wv[t][2][wd], wv[t][3][wd], 0x7632u);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t a0 = bf16x2_sub(lop3_and_or(uab >> (4 * q), 0x000F000Fu, 0x43004300u), zab);
+                        const uint32_t a1 = bf16x2_sub(lop3_and_or(vab >> (4 * q), 0x000F000Fu, 0x43004300u), zab);
+                        const uint32_t a2 = bf16x2_sub(lop3_and_or(ucd >> (4 * q), 0x000F000Fu, 0x43004300u), zcd);
+                        const uint32_t a3 = bf16x2_sub(lop3_and_or(vcd >> (4 * q), 0x000F000Fu, 0x43004300u), zcd);
+#pragma unroll
+                        for (int st = 0; st < NSET; ++st)
+                            mma_bf16_16816(acc[st][4 * wd + q], a0, a1, a2, a3, bq[st][0], bq[st][1]);
+                    }
                 }
             }
             __syncwarp();
-            const uint32_t b0 = tabw[bsel], b1 = tabw[bsel + 4];
-            // ---- codes: four nibble pairs of each word
-#pragma unroll
-            for (int S = 0; S < 2; ++S) {
-                uint32_t x0[4], x1[4];
-                if (S == 0) {
-                    transpose_bytes4(w[0][0].x, w[0][1].x, w[0][2].x, w[0][3].x, x0);
-                    transpose_bytes4(w[1][0].x, w[1][1].x, w[1][2].x, w[1][3].x, x1);
-                } else {
-                    transpose_bytes4(w[0][0].y, w[0][1].y, w[0][2].y, w[0][3].y, x0);
-                    transpose_bytes4(w[1][0].y, w[1][1].y, w[1][2].y, w[1][3].y, x1);
-                }
-#pragma unroll
-                for (int p = 0; p < 4; ++p)
-                    mma_u8s8_16832(acc[S][p], x0[p] & 0x0F0F0F0Fu, x0[p], x1[p] & 0x0F0F0F0Fu, x1[p], b0, b1);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            mbar_arrive_elected(&empty[s]);
             if (++s == NS) {
                 s = 0;
                 phase ^= 1u;
             }
         }
-        // ---- outputs: sum_n c' z over the warp, the last fold, 16 k per lane
+        // ---- outputs: the three parts of each activation row meet in lane
+        // tig = 0 (row 2 st) and tig = 1 (row 2 st + 1) of each gid: columns
+        // (0, 1 | 2) and (3 | 4, 5) of the set
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
+        for (int st = 0; st < NSET; ++st) {
+            float v[NT * 2];
 #pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) zt[m] += __shfl_xor_sync(0xFFFFFFFFu, zt[m], o);
-        const float xsm = xs_of(pick(thr));
-        fold(xsm);
-        const float zterm = pick(zt) * xsm;
-        const int k = kw + 16 * gid;                     // words 2 gid, 2 gid + 1
-        if (!*abort_flag && tig < M && k < a.K) {
-            float v[16];
+            for (int j = 0; j < NT; ++j)
 #pragma unroll
-            for (int S = 0; S < 2; ++S)
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    v[8 * S + 2 * p] = fac[S][p][0] - zterm;
-                    v[8 * S + 2 * p + 1] = fac[S][p][1] - zterm;
+                for (int h = 0; h < 2; ++h) {
+                    const float first = acc[st][j][2 * h], second = acc[st][j][2 * h + 1];
+                    const float whole = first + second;
+                    const float recv = __shfl_down_sync(0xFFFFFFFFu, tig == 1 ? first : whole, 1);
+                    v[2 * j + h] = tig == 0 ? whole + recv : second + recv;
                 }
-            if (a.splits == 1) {
-                uint32_t outw[8];
+            const int m = 2 * st + tig;
+            // k of value (j, h): word j / 4, nibble j % 4 + 4 h of the lane's words
+            const int kl = kw + (NWD == 2 ? 16 * gid : 8 * gid);
+            if (!*abort_flag && tig < 2 && m < M && kl < a.K) {
+                float o[8 * NWD];
 #pragma unroll
-                for (int e = 0; e < 16; e += 2) {
-                    float y0 = v[e], y1 = v[e + 1];
-                    if (a.bias) {
-                        y0 += bf16_bits_to_float(a.bias[k + e]);
-                        y1 += bf16_bits_to_float(a.bias[k + e + 1]);
+                for (int j = 0; j < NT; ++j)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) o[8 * (j >> 2) + (j & 3) + 4 * h] = v[2 * j + h];
+                if (a.splits == 1) {
+                    uint32_t outw[4 * NWD];
+#pragma unroll
+                    for (int e = 0; e < 8 * NWD; e += 2) {
+                        float y0 = o[e], y1 = o[e + 1];
+                        if (a.bias) {
+                            y0 += bf16_bits_to_float(a.bias[kl + e]);
+                            y1 += bf16_bits_to_float(a.bias[kl + e + 1]);
+                        }
+                        outw[e / 2] = bf162_bits(__floats2bfloat162_rn(y0, y1));
                     }
-                    outw[e / 2] = bf162_bits(__floats2bfloat162_rn(y0, y1));
-                }
-                uint4* o = reinterpret_cast<uint4*>(a.dX + static_cast<size_t>(tig) * a.K + k);
-                o[0] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-                o[1] = make_uint4(outw[4], outw[5], outw[6], outw[7]);
-            } else {
-                float4* pp = reinterpret_cast<float4*>(a.partial + (static_cast<size_t>(split) * M + tig) * a.K + k);
+                    uint4* op = reinterpret_cast<uint4*>(a.dX + static_cast<size_t>(m) * a.K + kl);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) pp[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    for (int q = 0; q < NWD; ++q)
+                        op[q] = make_uint4(outw[4 * q], outw[4 * q + 1], outw[4 * q + 2], outw[4 * q + 3]);
+                } else {
+                    float4* pp = reinterpret_cast<float4*>(a.partial + (static_cast<size_t>(split) * M + m) * a.K + kl);
+#pragma unroll
+                    for (int q = 0; q < 2 * NWD; ++q) pp[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+                }
             }
         }
     }

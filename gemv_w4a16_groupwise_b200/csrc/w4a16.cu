@@ -12,8 +12,8 @@
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
-#include "gemv_stream.cuh"
 #include "gemv_mma.cuh"
+#include "gemv_q8.cuh"
 #include "gemv_t_mma.cuh"
 #include "quantize.cuh"
 #include "w4a16.h"
@@ -214,19 +214,26 @@ TPlan plan_t(int M, int N, int K, int sms) {
 }
 
 // Tensor-pipe transposed GEMV (gemv_t_mma_kernel): K % 32 == 0 and the
-// tensor-pipe GEMV's scale/zero layouts (g a multiple of 128 with G % 8 == 0,
-// one group per row, or one global pair).  Row ranges are whole 32-row stages; the grid is a whole
-// number of splits per strip, at most one CTA per SM, with the fp32
+// scale/zero layouts its TMA boxes take (g a multiple of 64 with G % 8 == 0,
+// one group per row, or one global pair).  A warp covers KW k of its CTA's
+// strip: 128 for M <= 2 when g allows, else 64 (the accumulators of two mma
+// column sets then fit).  Row ranges are whole 32-row stages; the grid is a
+// whole number of splits per strip, at most one CTA per SM, with the fp32
 // partials held under about a tenth of the weights.
 struct TMmaPlan {
     bool ok = false;
-    int strips = 0, splits = 1, rows_per_split = 0, stages = 0, grid = 0;
+    int KW = 128, strips = 0, splits = 1, rows_per_split = 0, stages = 0, grid = 0;
     size_t smem = 0, ws = 0;
 };
 
-TMmaPlan plan_t_mma(int M, int N, int K, int sms, int max_smem) {
+int t_mma_kw(int M, const Meta& meta) {
+    return (M <= 2 && (meta.G == 1 || meta.g % 128 == 0)) ? 128 : 64;
+}
+
+TMmaPlan plan_t_mma(int M, int N, int K, int KW, int sms, int max_smem) {
     TMmaPlan p;
-    p.strips = (K + kTMStrip - 1) / kTMStrip;
+    p.KW = KW;
+    p.strips = (K + tm_strip(KW) - 1) / tm_strip(KW);
     int splits = std::max(1, sms / p.strips);
     splits = std::min(splits, std::max(1, N / (80 * M)));
     splits = std::min(splits, std::max(1, N / (kTMRows * 4)));   // at least 4 stages of rows per split
@@ -238,10 +245,13 @@ TMmaPlan plan_t_mma(int M, int N, int K, int sms, int max_smem) {
     // the split's dY rows live in shared memory: keep them under 32 KB
     while (static_cast<size_t>(p.rows_per_split) * 16 > 32 * 1024) set_rows(++splits);
     p.grid = p.strips * p.splits;
-    const size_t fixed = gemv_t_mma_smem_bytes(0, p.rows_per_split);
+    const int nset = (M + 1) / 2;
+    const size_t fixed = gemv_t_mma_smem_bytes(KW, nset, 0, p.rows_per_split);
     const size_t avail = max_smem > 0 ? static_cast<size_t>(max_smem) : 232448;
-    p.stages = avail > fixed ? static_cast<int>(std::min<size_t>(8, (avail - fixed) / (kTMStageBytes + 16))) : 0;
-    p.smem = gemv_t_mma_smem_bytes(p.stages, p.rows_per_split);
+    p.stages = avail > fixed
+                   ? static_cast<int>(std::min<size_t>(8, (avail - fixed) / (tm_stage_bytes(KW) + 16)))
+                   : 0;
+    p.smem = gemv_t_mma_smem_bytes(KW, nset, p.stages, p.rows_per_split);
     p.ws = p.splits > 1 ? static_cast<size_t>(p.splits) * M * K * sizeof(float) : 0;
     p.ok = p.stages >= 2;
     return p;
@@ -250,96 +260,30 @@ TMmaPlan plan_t_mma(int M, int N, int K, int sms, int max_smem) {
 bool t_mma_eligible(int K, const Meta& meta) {
     if (K % 32 != 0) return false;
     if (meta.sz_row == 0 || meta.G == 1) return true;
-    return meta.g % 128 == 0 && meta.G % 8 == 0;
+    return meta.g % 64 == 0 && meta.G % 8 == 0;
 }
 
-// Streaming forward GEMV (gemv_stream_kernel): K % 32 == 0 and g % 32 == 0
-// so that every 32-k chunk lies inside one group.  The K slice is the
-// largest whole number of 2048-k boxes whose activation block fits in
-// shared memory next to the TMA ring; the k-parts per round are chosen to
-// even out the work of the persistent CTAs.
-struct StreamPlan {
+// Tensor-pipe forward GEMV (gemv_mma_kernel): K % 32 == 0 and the group
+// length a multiple of 32, or one group per row.  A CTA-wide ring of
+// 16-row x 2048-k stages beside the slice's activation fragments; K is
+// split into slices only when the fragments of all of K leave no room for a
+// ring of 4 stages (then 3).
+struct MmaPlan {
     bool ok = false;
-    int TKC = 0, splits = 1, nbs = 0, KP = 1, RBP = kSW, rounds = 0, units = 0, grid = 0, stages = 2;
-    int szw = 0, warps = kSW, sz = 0;
-    int nrb = 0, cps = 0, nks = 0;             // tensor-pipe kernel: row blocks, CTAs per slice, stages per row block
-    bool mma = false, in_kernel_x = false;
-    size_t smem = 0, xbytes = 0, ws = 0, partial_off = 0;
+    int TKC = 0, splits = 1, nks = 0, nrb = 0, cps = 0, grid = 0, stages = 0;
+    int cls = kCls128, sz = kSzConst, szw = 0;
+    size_t smem = 0, ws = 0;
 };
 
-// szw: scale / zero words per stage row (gemv_stream_sz_words of the group
-// length).  Ring depth first: the deepest ring (4, 3, then 2 stages per
-// warp) whose activation block for all of K still fits; if none does, 2
-// stages and K split into slices.
-StreamPlan plan_stream_szw(int M, int N, int K, int szw, const DeviceInfo& di) {
-    StreamPlan p;
-    p.szw = szw;
-    const int nb_total = (K + kSBK - 1) / kSBK;
-    auto nbs_fit = [&](int stages) {
-        int best = 0;
-        for (int nb = 1; nb <= nb_total; ++nb) {
-            if (gemv_stream_smem_bytes(M, nb * kSBK, stages, szw) > static_cast<size_t>(di.max_smem_optin)) break;
-            best = nb;
-        }
-        return best;
-    };
-    int nbs_max = 0;
-    for (int stages : {4, 3, 2}) {
-        p.stages = stages;
-        nbs_max = nbs_fit(stages);
-        if (nbs_max >= nb_total) break;
-    }
-    if (nbs_max == 0) return p;
-    p.splits = (nb_total + nbs_max - 1) / nbs_max;
-    p.nbs = (nb_total + p.splits - 1) / p.splits;
-    p.TKC = p.nbs * kSBK;
-    const int nrb = (N + kSR - 1) / kSR;
-    double best = 1e300;
-    for (int KP : {1, 2, 4, 8}) {
-        if (KP > p.nbs) break;
-        const int RBP = kSW / KP;
-        const int rounds = (nrb + RBP - 1) / RBP;
-        const int units = p.splits * rounds;
-        const int grid = std::min(units, di.sms);
-        const int per_cta = (units + grid - 1) / grid;
-        // boxes the busiest warp streams, plus the round's barrier and
-        // reduction (about half a box)
-        const double cost = per_cta * ((p.nbs + KP - 1) / KP + 0.5);
-        if (cost < best * 0.999) {
-            best = cost;
-            p.KP = KP;
-            p.RBP = RBP;
-            p.rounds = rounds;
-            p.units = units;
-            p.grid = grid;
-        }
-    }
-    p.smem = gemv_stream_smem_bytes(M, p.TKC, p.stages, szw);
-    p.xbytes = gemv_stream_xblock_bytes(M, p.TKC);
-    p.partial_off = (p.splits * p.xbytes + 255) / 256 * 256;
-    p.ws = p.partial_off + (p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * sizeof(float) : 0);
-    p.ok = true;
-    return p;
-}
-
-StreamPlan plan_stream(int M, int N, int K, const Meta& meta, const DeviceInfo& di) {
-    if (K % 32 != 0 || meta.g % 32 != 0) return StreamPlan{};
-    return plan_stream_szw(M, N, K, gemv_stream_sz_words(meta.g), di);
-}
-
-// Tensor-pipe GEMV (gemv_mma_kernel): group length a multiple of 128, or
-// one group per row.  A CTA-wide ring of 16-row x 2048-k stages beside the
-// slice's activation block; K is split into slices only when the block of
-// all of K leaves no room for a ring of 4 stages (then 3).
-StreamPlan plan_mma(int M, int N, int K, int sz, int szw, const DeviceInfo& di) {
-    StreamPlan p;
-    p.szw = szw;
+MmaPlan plan_mma(int M, int N, int K, int cls, int sz, int szw, const DeviceInfo& di) {
+    MmaPlan p;
+    p.cls = cls;
     p.sz = sz;
-    p.warps = kMThreads / 32;
+    p.szw = szw;
     const int nk_total = (K + kMK - 1) / kMK;
     const size_t cap = static_cast<size_t>(di.max_smem_optin);
-    // the fewest K slices whose activation block leaves room for a ring of
-    // at least 4 stages (deeper rings first, up to 8), else 3
+    // the fewest K slices whose activation fragments leave room for a ring
+    // of at least 4 stages (deeper rings first, up to 8), else 3
     for (int min_st : {4, 3}) {
         for (int splits = 1; splits <= nk_total; ++splits) {
             const int nks = (nk_total + splits - 1) / splits;
@@ -364,223 +308,274 @@ StreamPlan plan_mma(int M, int N, int K, int sz, int szw, const DeviceInfo& di) 
     p.cps = std::max(1, std::min(di.sms / p.splits, p.nrb));
     p.grid = p.splits * p.cps;
     p.smem = gemv_mma_smem_bytes(M, p.TKC, p.stages, sz, szw);
-    p.xbytes = gemv_mma_xblock_bytes(M, p.TKC);
-    // every CTA converts its own activations when that is at most 4 units
-    // (256 k of one row) per consumer warp; else a prep kernel does it once
-    p.in_kernel_x = p.splits == 1 && (p.TKC / 256) * M <= 4 * kMW;
-    auto up = [](size_t v) { return (v + 255) / 256 * 256; };
-    p.partial_off = p.in_kernel_x ? 0 : up(p.splits * p.xbytes);
-    p.ws = p.partial_off + (p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * sizeof(float) : 0);
-    p.mma = true;
+    p.ws = p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * sizeof(float) : 0;
     p.ok = true;
     return p;
 }
 
-bool mma_eligible(int K, const Meta& meta) { return K % 32 == 0 && (meta.G == 1 || meta.g % 128 == 0); }
+bool mma_eligible(int K, const Meta& meta) { return K % 32 == 0 && (meta.G == 1 || meta.g % 32 == 0); }
 
-// How the tensor-pipe GEMV fetches scales and zeros (SzKind).
+// Which packed words a lane holds (WordClass): every k block of one mma
+// step must lie in one group.
+int mma_cls(const Meta& meta) {
+    if (meta.G == 1 || meta.g % 128 == 0) return kCls128;
+    return meta.g % 64 == 0 ? kCls64 : kCls32;
+}
+
+// How the tensor-pipe GEMV fetches scales and zeros (SzKind) and the width
+// that goes with it.
 int mma_sz_kind(const Meta& meta) {
     if (meta.sz_row == 0) return kSzConst;
     if (meta.G == 1) return kSzTma1d;
-    if (meta.G % 8 == 0) return kSzTma2d;
+    if (meta.G % 8 == 0 && gemv_mma_sz_box(meta.g) <= 256) return kSzTma2d;
     return kSzCopy;
 }
+int mma_szw(const Meta& meta, int sz) {
+    return sz == kSzTma2d ? gemv_mma_sz_box(meta.g) : sz == kSzCopy ? gemv_mma_sz_words(meta.g) : 0;
+}
+
+// group of k = (k * mul) >> shift for 0 <= k < 2^31: with l = ceil(log2 g)
+// and mul = floor(2^(31 + l) / g) + 1, k * mul / 2^(31 + l) exceeds k / g
+// by less than 2^-l <= 1 / g, so the floor is exact.
+void group_magic(int g, unsigned long long* mul, int* shift) {
+    int l = 0;
+    while ((1ll << l) < g) ++l;
+    *shift = 31 + l;
+    *mul = (1ull << (31 + l)) / static_cast<unsigned long long>(g) + 1ull;
+}
+
+// Int8 tensor-pipe forward GEMV (gemv_q8_kernel): K % 32 == 0 and the
+// group length a multiple of 128, or one group per row.  The ring is as deep
+// as shared memory allows (up to 8 stages); K is split into slices only to
+// give every SM work when there are fewer row blocks than SMs.
+struct Q8Plan {
+    bool ok = false;
+    int TKC = 0, splits = 1, nks = 0, nrb = 0, cps = 0, grid = 0, stages = 0;
+    int sz = kSzConst, szw = 0;
+    size_t smem = 0, ws = 0;
+};
+
+Q8Plan plan_q8(int M, int N, int K, int sz, int szw, const DeviceInfo& di) {
+    Q8Plan p;
+    p.sz = sz;
+    p.szw = szw;
+    const size_t cap = static_cast<size_t>(di.max_smem_optin);
+    for (int c = 8; c >= 2; --c)
+        if (gemv_q8_smem_bytes(c, sz, szw) <= cap) {
+            p.stages = c;
+            break;
+        }
+    if (p.stages == 0) return p;
+    const int nk_total = (K + kMK - 1) / kMK;
+    p.nrb = (N + kMR - 1) / kMR;
+    int splits = 1;
+    if (2 * p.nrb <= di.sms) splits = std::min(nk_total, std::max(1, di.sms / p.nrb));
+    p.nks = (nk_total + splits - 1) / splits;
+    p.splits = (nk_total + p.nks - 1) / p.nks;
+    p.TKC = p.nks * kMK;
+    p.cps = std::max(1, std::min(di.sms / p.splits, p.nrb));
+    p.grid = p.splits * p.cps;
+    p.smem = gemv_q8_smem_bytes(p.stages, sz, szw);
+    p.ws = p.splits > 1 ? static_cast<size_t>(p.splits) * M * N * sizeof(float) : 0;
+    p.ok = true;
+    return p;
+}
+
+bool q8_eligible(int K, const Meta& meta) { return K % 32 == 0 && (meta.G == 1 || meta.g % 128 == 0); }
 
 size_t gemv_workspace(int M, int N, int K, int transposed, int sms) {
     if (transposed) {
         size_t ws = plan_t(M, N, K, sms).ws;
         if (K % 32 == 0)
-            ws = std::max(ws, plan_t_mma(M, N, K, sms, device_info(current_device()).max_smem_optin).ws);
+            for (int kw : {64, 128})
+                ws = std::max(ws, plan_t_mma(M, N, K, kw, sms, device_info(current_device()).max_smem_optin).ws);
         return ws;
     }
     if (K % 32 != 0) return 0;
-    // the group length picks the kernel and the stage size, and so possibly
-    // the split: cover every choice a group length of 32 .. K can make
+    // the group length sets the stage size, and so possibly the split:
+    // cover every choice a group length of 32 .. K can make
     DeviceInfo di = device_info(current_device());
     di.sms = sms;
-    size_t ws = 0;
-    for (int szw = gemv_stream_sz_words(K); szw <= gemv_stream_sz_words(32); ++szw) {
-        const StreamPlan p = plan_stream_szw(M, N, K, szw, di);
-        if (p.ok) ws = std::max(ws, p.ws);
-    }
-    for (int sz : {kSzConst, kSzTma2d, kSzTma1d}) {
-        const StreamPlan q = plan_mma(M, N, K, sz, 0, di);
+    size_t ws = plan_q8(M, N, K, kSzConst, 0, di).ws;
+    for (int sz : {kSzConst, kSzTma1d}) {
+        const MmaPlan q = plan_mma(M, N, K, kCls128, sz, 0, di);
         if (q.ok) ws = std::max(ws, q.ws);
     }
-    for (int szw = gemv_mma_sz_words(K); szw <= gemv_mma_sz_words(128); ++szw) {
-        const StreamPlan q = plan_mma(M, N, K, kSzCopy, szw, di);
+    for (int szw = 8; szw <= 64; szw += 8) {
+        const MmaPlan q = plan_mma(M, N, K, kCls128, kSzTma2d, szw, di);
+        if (q.ok) ws = std::max(ws, q.ws);
+    }
+    for (int szw = gemv_mma_sz_words(K); szw <= gemv_mma_sz_words(32); ++szw) {
+        const MmaPlan q = plan_mma(M, N, K, kCls128, kSzCopy, szw, di);
         if (q.ok) ws = std::max(ws, q.ws);
     }
     return ws;
 }
 
-template <int M, int GK>
-w4_status launch_gemv_stream_gk(const StreamPlan& p, const CUtensorMap& map, const GemvStreamArgs& a,
-                                cudaStream_t st) {
-    const void* fn = reinterpret_cast<const void*>(gemv_stream_kernel<M, GK>);
-    if (ensure_smem(fn, p.smem) != cudaSuccess) return W4_ERR_CUDA;
-    gemv_stream_kernel<M, GK><<<p.grid, kSW * 32, p.smem, st>>>(map, a);
-    return launch_status();
-}
-
-template <int M>
-w4_status launch_gemv_stream(const StreamPlan& p, const CUtensorMap& map, const GemvStreamArgs& a,
-                             cudaStream_t st) {
-    if (a.G == 1) return launch_gemv_stream_gk<M, kGroupsOne>(p, map, a, st);
-    if (kSBK % a.g == 0) return launch_gemv_stream_gk<M, kGroupsPow2>(p, map, a, st);
-    return launch_gemv_stream_gk<M, kGroupsAny>(p, map, a, st);
-}
-
 // The GEMV is always launched as a programmatic dependent of the work just
-// before it.  After its own prep kernel, its prologue and first weight
-// loads overlap the prep kernel; otherwise only its prologue overlaps the
-// previous kernel's tail, and it waits for that kernel before reading any
-// input.
-template <int M, int GK, int SZ>
-w4_status launch_gemv_mma_k(const StreamPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
+// before it: its prologue overlaps that work's tail, and it waits for that
+// work before reading any input.
+template <int M, int CLS, int SZ>
+w4_status launch_gemv_mma_k(const MmaPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
                             const CUtensorMap& zm, const GemvMmaArgs& a, cudaStream_t st) {
-    auto* fn = gemv_mma_kernel<M, GK, SZ>;
+    auto* fn = gemv_mma_kernel<M, CLS, SZ>;
     if (ensure_smem(reinterpret_cast<const void*>(fn), p.smem) != cudaSuccess) return W4_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.grid);
-    cfg.blockDim = dim3(kMThreads);
-    cfg.dynamicSmemBytes = p.smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, fn, wm, sm, zm, a);
+    launch_pdl(fn, dim3(p.grid), dim3(kMThreads), p.smem, st, wm, sm, zm, a);
     return launch_status();
 }
 
-template <int M, int GK>
-w4_status launch_gemv_mma_gk(const StreamPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
-                             const CUtensorMap& zm, const GemvMmaArgs& a, cudaStream_t st) {
+template <int M, int CLS>
+w4_status launch_gemv_mma_c(const MmaPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
+                            const CUtensorMap& zm, const GemvMmaArgs& a, cudaStream_t st) {
     switch (p.sz) {
-        case kSzConst: return launch_gemv_mma_k<M, GK, kSzConst>(p, wm, sm, zm, a, st);
-        case kSzTma2d: return launch_gemv_mma_k<M, GK, kSzTma2d>(p, wm, sm, zm, a, st);
-        case kSzTma1d: return launch_gemv_mma_k<M, GK, kSzTma1d>(p, wm, sm, zm, a, st);
-        default: return launch_gemv_mma_k<M, GK, kSzCopy>(p, wm, sm, zm, a, st);
+        case kSzConst: return launch_gemv_mma_k<M, CLS, kSzConst>(p, wm, sm, zm, a, st);
+        case kSzTma2d: return launch_gemv_mma_k<M, CLS, kSzTma2d>(p, wm, sm, zm, a, st);
+        case kSzTma1d: return launch_gemv_mma_k<M, CLS, kSzTma1d>(p, wm, sm, zm, a, st);
+        default: return launch_gemv_mma_k<M, CLS, kSzCopy>(p, wm, sm, zm, a, st);
     }
 }
 
 template <int M>
-w4_status launch_gemv_mma_m(const StreamPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
+w4_status launch_gemv_mma_m(const MmaPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
                             const CUtensorMap& zm, const GemvMmaArgs& a, cudaStream_t st) {
-    if (a.G == 1) return launch_gemv_mma_gk<M, kGroupsOne>(p, wm, sm, zm, a, st);
-    if (kSBK % a.g == 0) return launch_gemv_mma_gk<M, kGroupsPow2>(p, wm, sm, zm, a, st);
-    return launch_gemv_mma_gk<M, kGroupsAny>(p, wm, sm, zm, a, st);
+    // group lengths that are a multiple of 128 run the int8 kernel
+    if (p.cls == kCls64) return launch_gemv_mma_c<M, kCls64>(p, wm, sm, zm, a, st);
+    return launch_gemv_mma_c<M, kCls32>(p, wm, sm, zm, a, st);
 }
 
-w4_status launch_gemv_mma(const StreamPlan& p, int M, const CUtensorMap& wm, const void* S, const void* Z,
-                          const GemvMmaArgs& a, cudaStream_t st) {
-    CUtensorMap sm, zm;
-    std::memset(&sm, 0, sizeof sm);
-    std::memset(&zm, 0, sizeof zm);
-    bool ok = true;
-    if (p.sz == kSzTma2d) {
-        ok = make_map_2d(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.G, kMR, 16, 0) &&
-             make_map_2d(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.G, kMR, 16, 0);
-    } else if (p.sz == kSzTma1d) {
-        ok = make_map_row(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, kMR) &&
-             make_map_row(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, kMR);
-    }
-    if (!ok) return W4_ERR_CUDA;
-    switch (M) {
-        case 1: return launch_gemv_mma_m<1>(p, wm, sm, zm, a, st);
-        case 2: return launch_gemv_mma_m<2>(p, wm, sm, zm, a, st);
-        case 3: return launch_gemv_mma_m<3>(p, wm, sm, zm, a, st);
-        default: return launch_gemv_mma_m<4>(p, wm, sm, zm, a, st);
-    }
-}
-
-w4_status run_gemv_stream(const StreamPlan& p, int M, int N, int K, const void* A, const uint32_t* packed,
-                          const void* S, const void* Z, const Meta& meta, const void* bias, void* Y,
-                          void* ws, size_t ws_bytes, cudaStream_t st) {
+w4_status run_gemv_mma(const MmaPlan& p, int M, int N, int K, const void* A, const uint32_t* packed,
+                       const void* S, const void* Z, const Meta& meta, const void* bias, void* Y, void* ws,
+                       size_t ws_bytes, cudaStream_t st) {
     if (p.ws > ws_bytes || (p.ws > 0 && ws == nullptr)) return W4_ERR_WORKSPACE;
     if (ws && !aligned16(ws)) return W4_ERR_ALIGNMENT;
-    uint8_t* xb = static_cast<uint8_t*>(ws);
-    float* partial = p.splits > 1 ? reinterpret_cast<float*>(xb + p.partial_off) : nullptr;
-    CUtensorMap map;
-    if (!make_map_2d(&map, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, p.mma ? kMR : kSR, kSBK / 8, 0))
-        return W4_ERR_CUDA;
+    float* partial = p.splits > 1 ? static_cast<float*>(ws) : nullptr;
+    CUtensorMap wm, sm, zm;
+    std::memset(&sm, 0, sizeof sm);
+    std::memset(&zm, 0, sizeof zm);
+    bool ok = make_map_2d(&wm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, kMR, kMK / 8, 0);
+    if (p.sz == kSzTma2d) {
+        ok = ok && make_map_2d(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, meta.G, kMR, p.szw, 0) &&
+             make_map_2d(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, meta.G, kMR, p.szw, 0);
+    } else if (p.sz == kSzTma1d) {
+        ok = ok && make_map_row(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, kMR) &&
+             make_map_row(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, kMR);
+    }
+    if (!ok) return W4_ERR_CUDA;
+    GemvMmaArgs a;
+    a.X = static_cast<const uint16_t*>(A);
+    a.S = static_cast<const __half*>(S);
+    a.Z = static_cast<const __half*>(Z);
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.Y = static_cast<uint16_t*>(Y);
+    a.partial = partial;
+    a.N = N;
+    a.K = K;
+    a.g = meta.g;
+    a.G = meta.G;
+    a.sz_row = meta.sz_row;
+    group_magic(meta.g, &a.gmul, &a.gshift);
+    a.TKC = p.TKC;
+    a.splits = p.splits;
+    a.nks = p.nks;
+    a.nrb = p.nrb;
+    a.cps = p.cps;
+    a.stages = p.stages;
+    a.szw = p.szw;
+    a.sz_total = meta.sz_row ? static_cast<long long>(N) * meta.sz_row : 1;
     w4_status s = W4_OK;
-    if (p.mma) {
-        if (!p.in_kernel_x) {
-            const long long lanes = static_cast<long long>(p.splits) * (p.TKC / 256) * M * 32;
-            gemv_xfrag_kernel<<<static_cast<int>((lanes + 255) / 256), 256, 0, st>>>(
-                static_cast<const uint16_t*>(A), M, K, p.TKC, p.splits, xb);
-            s = launch_status();
-            if (s != W4_OK) return s;
-        }
-        GemvMmaArgs a;
-        a.X = static_cast<const uint16_t*>(A);
-        a.xblocks = p.in_kernel_x ? nullptr : xb;
-        a.S = static_cast<const __half*>(S);
-        a.Z = static_cast<const __half*>(Z);
-        a.bias = static_cast<const uint16_t*>(bias);
-        a.Y = static_cast<uint16_t*>(Y);
-        a.partial = partial;
-        a.N = N;
-        a.K = K;
-        a.g = meta.g;
-        a.G = meta.G;
-        a.sz_row = meta.sz_row;
-        a.TKC = p.TKC;
-        a.splits = p.splits;
-        a.nks = p.nks;
-        a.nrb = p.nrb;
-        a.cps = p.cps;
-        a.stages = p.stages;
-        a.szw = p.szw;
-        a.sz_total = meta.sz_row ? static_cast<long long>(N) * meta.sz_row : 1;
-        s = launch_gemv_mma(p, M, map, S, Z, a, st);
-    } else {
-        const long long chunks = static_cast<long long>(p.splits) * M * (p.TKC / 32);
-        gemv_xprep_kernel<<<static_cast<int>((chunks + 255) / 256), 256, 0, st>>>(
-            static_cast<const uint16_t*>(A), M, K, p.TKC, p.splits, xb);
-        s = launch_status();
-        if (s != W4_OK) return s;
-        GemvStreamArgs a;
-        a.xblocks = xb;
-        a.S = static_cast<const __half*>(S);
-        a.Z = static_cast<const __half*>(Z);
-        a.bias = static_cast<const uint16_t*>(bias);
-        a.Y = static_cast<uint16_t*>(Y);
-        a.partial = partial;
-        a.N = N;
-        a.K = K;
-        a.g = meta.g;
-        a.G = meta.G;
-        a.sz_row = meta.sz_row;
-        a.TKC = p.TKC;
-        a.splits = p.splits;
-        a.nbs = p.nbs;
-        a.KP = p.KP;
-        a.RBP = p.RBP;
-        a.rounds = p.rounds;
-        a.units = p.units;
-        a.stages = p.stages;
-        a.szw = p.szw;
-        a.sz_total = meta.sz_row ? static_cast<long long>(N) * meta.sz_row : 1;
-        a.M = M;
-        switch (M) {
-            case 1: s = launch_gemv_stream<1>(p, map, a, st); break;
-            case 2: s = launch_gemv_stream<2>(p, map, a, st); break;
-            case 3: s = launch_gemv_stream<3>(p, map, a, st); break;
-            case 4: s = launch_gemv_stream<4>(p, map, a, st); break;
-            default: return W4_ERR_INVALID_ARG;
-        }
+    switch (M) {
+        case 1: s = launch_gemv_mma_m<1>(p, wm, sm, zm, a, st); break;
+        case 2: s = launch_gemv_mma_m<2>(p, wm, sm, zm, a, st); break;
+        case 3: s = launch_gemv_mma_m<3>(p, wm, sm, zm, a, st); break;
+        case 4: s = launch_gemv_mma_m<4>(p, wm, sm, zm, a, st); break;
+        default: return W4_ERR_INVALID_ARG;
     }
     if (s != W4_OK) return s;
     if (p.splits > 1) {
         const DeviceInfo di = device_info(current_device());
         const long long total = static_cast<long long>(M) * N;
         const int blocks = static_cast<int>(std::min<long long>((total + kFinOut - 1) / kFinOut, di.sms * 16));
-        splits_finalize_kernel<<<blocks, 256, 0, st>>>(partial, p.splits, M, N, static_cast<const uint16_t*>(bias),
-                                                        static_cast<uint16_t*>(Y));
+        launch_pdl(splits_finalize_kernel, dim3(blocks), dim3(256), 0, st, static_cast<const float*>(partial),
+                   p.splits, M, N, static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(Y));
+        return launch_status();
+    }
+    return W4_OK;
+}
+
+template <int M, int SZ>
+w4_status launch_q8_k(const Q8Plan& p, const CUtensorMap& wm, const CUtensorMap& sm, const CUtensorMap& zm,
+                      const GemvQ8Args& a, cudaStream_t st) {
+    auto* fn = gemv_q8_kernel<M, SZ>;
+    if (ensure_smem(reinterpret_cast<const void*>(fn), p.smem) != cudaSuccess) return W4_ERR_CUDA;
+    launch_pdl(fn, dim3(p.grid), dim3(kQThreads), p.smem, st, wm, sm, zm, a);
+    return launch_status();
+}
+
+template <int M>
+w4_status launch_q8_m(const Q8Plan& p, const CUtensorMap& wm, const CUtensorMap& sm, const CUtensorMap& zm,
+                      const GemvQ8Args& a, cudaStream_t st) {
+    switch (p.sz) {
+        case kSzConst: return launch_q8_k<M, kSzConst>(p, wm, sm, zm, a, st);
+        case kSzTma2d: return launch_q8_k<M, kSzTma2d>(p, wm, sm, zm, a, st);
+        case kSzTma1d: return launch_q8_k<M, kSzTma1d>(p, wm, sm, zm, a, st);
+        default: return launch_q8_k<M, kSzCopy>(p, wm, sm, zm, a, st);
+    }
+}
+
+w4_status run_gemv_q8(const Q8Plan& p, int M, int N, int K, const void* A, const uint32_t* packed, const void* S,
+                      const void* Z, const Meta& meta, const void* bias, void* Y, void* ws, size_t ws_bytes,
+                      cudaStream_t st) {
+    if (p.ws > ws_bytes || (p.ws > 0 && ws == nullptr)) return W4_ERR_WORKSPACE;
+    if (ws && !aligned16(ws)) return W4_ERR_ALIGNMENT;
+    float* partial = p.splits > 1 ? static_cast<float*>(ws) : nullptr;
+    CUtensorMap wm, sm, zm;
+    std::memset(&sm, 0, sizeof sm);
+    std::memset(&zm, 0, sizeof zm);
+    bool ok = make_map_2d(&wm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, N, K / 8, kMR, kMK / 8, 0);
+    if (p.sz == kSzTma2d) {
+        ok = ok && make_map_2d(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, meta.G, kMR, p.szw, 0) &&
+             make_map_2d(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, meta.G, kMR, p.szw, 0);
+    } else if (p.sz == kSzTma1d) {
+        ok = ok && make_map_row(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, kMR) &&
+             make_map_row(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, kMR);
+    }
+    if (!ok) return W4_ERR_CUDA;
+    GemvQ8Args a;
+    a.X = static_cast<const uint16_t*>(A);
+    a.S = static_cast<const __half*>(S);
+    a.Z = static_cast<const __half*>(Z);
+    a.bias = static_cast<const uint16_t*>(bias);
+    a.Y = static_cast<uint16_t*>(Y);
+    a.partial = partial;
+    a.N = N;
+    a.K = K;
+    a.g = meta.g;
+    a.G = meta.G;
+    a.sz_row = meta.sz_row;
+    group_magic(meta.g, &a.gmul, &a.gshift);
+    a.TKC = p.TKC;
+    a.splits = p.splits;
+    a.nks = p.nks;
+    a.nrb = p.nrb;
+    a.cps = p.cps;
+    a.stages = p.stages;
+    a.szw = p.szw;
+    a.sz_total = meta.sz_row ? static_cast<long long>(N) * meta.sz_row : 1;
+    w4_status s = W4_OK;
+    switch (M) {
+        case 1: s = launch_q8_m<1>(p, wm, sm, zm, a, st); break;
+        case 2: s = launch_q8_m<2>(p, wm, sm, zm, a, st); break;
+        case 3: s = launch_q8_m<3>(p, wm, sm, zm, a, st); break;
+        case 4: s = launch_q8_m<4>(p, wm, sm, zm, a, st); break;
+        default: return W4_ERR_INVALID_ARG;
+    }
+    if (s != W4_OK) return s;
+    if (p.splits > 1) {
+        const DeviceInfo di = device_info(current_device());
+        const long long total = static_cast<long long>(M) * N;
+        const int blocks = static_cast<int>(std::min<long long>((total + kFinOut - 1) / kFinOut, di.sms * 16));
+        launch_pdl(splits_finalize_kernel, dim3(blocks), dim3(256), 0, st, static_cast<const float*>(partial),
+                   p.splits, M, N, static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(Y));
         return launch_status();
     }
     return W4_OK;
@@ -590,14 +585,15 @@ w4_status run_gemv_fwd(const void* A, int M, int N, int K, const uint32_t* packe
                        const void* Z, const Meta& meta, const void* bias, void* Y, void* ws,
                        size_t ws_bytes, cudaStream_t st) {
     const DeviceInfo di = device_info(current_device());
-    {
-        StreamPlan sp;
-        if (mma_eligible(K, meta)) {
-            const int sz = mma_sz_kind(meta);
-            sp = plan_mma(M, N, K, sz, sz == kSzCopy ? gemv_mma_sz_words(meta.g) : 0, di);
-        }
-        if (!sp.ok) sp = plan_stream(M, N, K, meta, di);
-        if (sp.ok) return run_gemv_stream(sp, M, N, K, A, packed, S, Z, meta, bias, Y, ws, ws_bytes, st);
+    if (q8_eligible(K, meta)) {
+        const int sz = mma_sz_kind(meta);
+        const Q8Plan qp = plan_q8(M, N, K, sz, mma_szw(meta, sz), di);
+        if (qp.ok) return run_gemv_q8(qp, M, N, K, A, packed, S, Z, meta, bias, Y, ws, ws_bytes, st);
+    }
+    if (mma_eligible(K, meta)) {
+        const int sz = mma_sz_kind(meta);
+        const MmaPlan mp = plan_mma(M, N, K, mma_cls(meta), sz, mma_szw(meta, sz), di);
+        if (mp.ok) return run_gemv_mma(mp, M, N, K, A, packed, S, Z, meta, bias, Y, ws, ws_bytes, st);
     }
     // K or the group length not a multiple of 32: one warp per output row
     GemvFwdArgs a;
@@ -622,23 +618,31 @@ w4_status run_gemv_fwd(const void* A, int M, int N, int K, const uint32_t* packe
     return launch_status();
 }
 
-template <int M, int SZ>
+template <int M, int KW, int SZ>
 w4_status launch_t_mma_k(const TMmaPlan& p, const CUtensorMap& wm, const CUtensorMap& sm, const CUtensorMap& zm,
                          const GemvTMmaArgs& a, cudaStream_t st) {
-    auto* fn = gemv_t_mma_kernel<M, SZ>;
+    auto* fn = gemv_t_mma_kernel<M, KW, SZ>;
     if (ensure_smem(reinterpret_cast<const void*>(fn), p.smem) != cudaSuccess) return W4_ERR_CUDA;
     launch_pdl(fn, dim3(p.grid), dim3(kTMThreads), p.smem, st, wm, sm, zm, a);
     return launch_status();
 }
 
+template <int M, int KW>
+w4_status launch_t_mma_kw(const TMmaPlan& p, int sz, const CUtensorMap& wm, const CUtensorMap& sm,
+                          const CUtensorMap& zm, const GemvTMmaArgs& a, cudaStream_t st) {
+    switch (sz) {
+        case kSzConst: return launch_t_mma_k<M, KW, kSzConst>(p, wm, sm, zm, a, st);
+        case kSzTma1d: return launch_t_mma_k<M, KW, kSzTma1d>(p, wm, sm, zm, a, st);
+        default: return launch_t_mma_k<M, KW, kSzTma2d>(p, wm, sm, zm, a, st);
+    }
+}
+
 template <int M>
 w4_status launch_t_mma_m(const TMmaPlan& p, int sz, const CUtensorMap& wm, const CUtensorMap& sm,
                          const CUtensorMap& zm, const GemvTMmaArgs& a, cudaStream_t st) {
-    switch (sz) {
-        case kSzConst: return launch_t_mma_k<M, kSzConst>(p, wm, sm, zm, a, st);
-        case kSzTma1d: return launch_t_mma_k<M, kSzTma1d>(p, wm, sm, zm, a, st);
-        default: return launch_t_mma_k<M, kSzTma2d>(p, wm, sm, zm, a, st);
-    }
+    // M = 3, 4 always take KW = 64 (two column sets)
+    if (M <= 2 && p.KW == 128) return launch_t_mma_kw<M, (M <= 2 ? 128 : 64)>(p, sz, wm, sm, zm, a, st);
+    return launch_t_mma_kw<M, 64>(p, sz, wm, sm, zm, a, st);
 }
 
 w4_status run_gemv_t_mma(const TMmaPlan& p, int sz, int M, int N, int K, const void* A, const uint32_t* packed,
@@ -648,8 +652,8 @@ w4_status run_gemv_t_mma(const TMmaPlan& p, int sz, int M, int N, int K, const v
     CUtensorMap wm, sm, zm;
     std::memset(&sm, 0, sizeof sm);
     std::memset(&zm, 0, sizeof zm);
-    // packed rows as K / 16 8-byte elements: boxes of 32 rows x 1040 bytes
-    bool ok = make_map_2d(&wm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, N, K / 16, kTMRows, kTMBoxX, 0);
+    // packed rows as K / 16 8-byte elements: boxes of 32 rows x (strip + 16) bytes
+    bool ok = make_map_2d(&wm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, N, K / 16, kTMRows, tm_pitch(p.KW) / 8, 0);
     if (sz == kSzTma2d)
         ok = ok && make_map_2d(&sm, S, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, meta.G, kTMRows, 16, 0) &&
              make_map_2d(&zm, Z, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, meta.G, kTMRows, 16, 0);
@@ -702,7 +706,7 @@ w4_status run_gemv_t(const void* A, int M, int N, int K, const uint32_t* packed,
     const DeviceInfo di = device_info(current_device());
     if (t_mma_eligible(K, meta)) {
         const int sz = meta.sz_row == 0 ? kSzConst : (meta.G == 1 ? kSzTma1d : kSzTma2d);
-        const TMmaPlan mp = plan_t_mma(M, N, K, di.sms, di.max_smem_optin);
+        const TMmaPlan mp = plan_t_mma(M, N, K, t_mma_kw(M, meta), di.sms, di.max_smem_optin);
         if (mp.ok) return run_gemv_t_mma(mp, sz, M, N, K, A, packed, S, Z, meta, bias, Y, ws, ws_bytes, st);
     }
     const TPlan p = plan_t(M, N, K, di.sms);
@@ -1076,8 +1080,8 @@ w4_status w4a16_gemv_noalloc(const void* X, int M, int N, int K, const uint32_t*
     void* scratch = nullptr;
     s = noalloc_scratch(&scratch);
     if (s != W4_OK) return s;
-    const int sms = device_info(current_device()).sms;
-    if (gemv_workspace(M, N, K, 0, sms) > kNoAllocScratchBytes) return W4_ERR_WORKSPACE;
+    // the chosen plan's workspace is checked against the scratch size
+    // before anything is launched (W4_ERR_WORKSPACE when it does not fit)
     return run_gemv_fwd(X, M, N, K, packed, scales, zeros, meta, bias, Y, scratch,
                         kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
 }

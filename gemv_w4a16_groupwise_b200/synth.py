@@ -102,3 +102,42 @@ def plant_structure(W: np.ndarray, g: int, seed: int) -> np.ndarray:
     last = bf16_bits_to_f32(W[N - 1]).astype(np.float64)
     W[N - 1] = f64_to_bf16_bits(np.abs(last) + 0.1)
     return W
+
+
+def outlier_activations(M: int, K: int, seed: int, exp: int, period: int = 128,
+                        stream: int = STREAM_X) -> tuple[np.ndarray, np.ndarray]:
+    """N(0, 1) bf16 rows with one entry of magnitude 2^exp (random sign) in every
+    ``period`` consecutive entries, at a seeded position; returns (values, the
+    outlier positions along the row).  Activation outliers of this kind are what
+    decode-time LLM activations show."""
+    A = normal_bf16((M, K), 0.0, 1.0, seed, stream)
+    rng = np.random.default_rng([int(seed), 77])
+    blocks = (K + period - 1) // period
+    pos = np.minimum(np.arange(blocks) * period + rng.integers(0, period, blocks), K - 1)
+    sign = np.where(rng.integers(0, 2, (M, blocks)) == 1, np.uint16(0x8000), np.uint16(0))
+    big = f64_to_bf16_bits(np.array([2.0 ** exp]))[0]
+    A[:, pos] = big | sign
+    return A, pos
+
+
+def mixed_range_activations(M: int, K: int, seed: int, lo_exp: int = -20, hi_exp: int = 4,
+                            every: int = 8, stream: int = STREAM_X) -> tuple[np.ndarray, np.ndarray]:
+    """bf16 rows mixing N(0, 2^(2 lo_exp)) values with N(0, 2^(2 hi_exp)) ones at a
+    seeded one in ``every`` positions (the same positions in every row); returns
+    (values, the large positions)."""
+    rng = np.random.default_rng([int(seed), 78])
+    z = rng.standard_normal((M, K))
+    pos = np.flatnonzero(rng.integers(0, every, K) == 0)
+    scale = np.full(K, 2.0 ** lo_exp)
+    scale[pos] = 2.0 ** hi_exp
+    return f64_to_bf16_bits(z * scale[None, :]), pos
+
+
+def spread_rows(W: np.ndarray, seed: int, binades: int = 10) -> np.ndarray:
+    """Copy of bf16 W with each row scaled by a seeded power of two in
+    [2^(-binades/2), 2^(binades/2)], so that the rows' quantization scales
+    spread over ``binades`` binades (exact: powers of two)."""
+    rng = np.random.default_rng([int(seed), 79])
+    e = rng.integers(-(binades // 2), binades // 2 + 1, W.shape[0])
+    v = bf16_bits_to_f32(W).astype(np.float64) * (2.0 ** e)[:, None]
+    return f64_to_bf16_bits(v)

@@ -26,8 +26,10 @@
  *     each comment; the first failure is returned and nothing is launched.
  *     After each launch the library checks cudaGetLastError() and returns
  *     W4_ERR_CUDA if it reports a launch failure.
- *   - The library allocates no device memory.  Kernels that need scratch
- *     take it from the caller's `workspace`; query the size first.
+ *   - The library allocates no device memory at run time.  Kernels that
+ *     need scratch take it from the caller's `workspace`; query the size
+ *     first.  The one exception is w4a16_gemv_noalloc, whose scratch is a
+ *     fixed 8 MiB array compiled into the library (see there).
  *   - Pointers must be 16-byte aligned (W4_ERR_ALIGNMENT otherwise).
  */
 #ifndef W4A16_H
@@ -120,10 +122,19 @@ w4_status w4a16_gemm(const void *A, int M, int N, int K, const uint32_t *packed,
 /*
  * w4a16_gemv -- the small-batch path (TensorRT-LLM "Modify small-batched
  * weight only quantization": a batch <= 4 GEMV is bound by global memory
- * loads): TMA-streamed packed weights whose integer dot products run as
- * mma.sync u8 x s8 on the tensor pipe, forward and transposed (other group
- * lengths or K % 32 != 0 fall back to CUDA-core kernels).  Same arguments
- * and results as w4a16_gemm; M must be 1..4 (W4_ERR_INVALID_ARG otherwise).
+ * loads): TMA-streamed packed weights with their dot products on the tensor
+ * pipe.  Every product of a code and an activation is exact and the sums are
+ * fp32:
+ *   forward, g a multiple of 128 or one group per row: int8 mma on the
+ *     activations as exact 24-bit integers per 128-k granule (three digits);
+ *     a granule whose values span more than 15 binades takes bf16 mma on
+ *     exact (q - z) codes instead;
+ *   forward, other g multiples of 32: bf16 mma on exact (q - z) codes;
+ *   transposed: bf16 mma, dY * s split into three exact bf16 parts;
+ *   K or g not a multiple of 32 (or scale layouts the TMA boxes do not
+ *     take): CUDA-core kernels with exact (q - z) and fp32 fma.
+ * Same arguments and results as w4a16_gemm; M must be 1..4
+ * (W4_ERR_INVALID_ARG otherwise).
  */
 w4_status w4a16_gemv(const void *A, int M, int N, int K, const uint32_t *packed,
                      const void *scales, const void *zeros, int mode, int group_size,
@@ -174,17 +185,21 @@ uint64_t w4_launch_count(void);
  * w4a16_gemv.
  *
  * Limits and sharing:
- *   - A problem whose workspace (the activations in the kernel's
- *     fixed-point form and, when K is split, the fp32 partials) needs more
- *     than 8 MiB (w4_workspace_bytes(M, N, K, 0) > 8 MiB) returns
- *     W4_ERR_WORKSPACE and launches nothing.
+ *   - The scratch holds the fp32 partial sums of a plan that splits K (few
+ *     output rows and a long K, or activations too long for shared
+ *     memory).  Every problem with w4_workspace_bytes(M, N, K, 0) <= 8 MiB
+ *     runs; a larger one runs when the plan for its own group length fits,
+ *     else the call returns W4_ERR_WORKSPACE and launches nothing.
  *   - Every call on a device shares the one array.  Calls that may overlap
  *     on the GPU (other streams, other host threads) race on it and give
  *     wrong results; order them on one stream.  Each call writes all the
  *     scratch it later reads, so nothing needs clearing between calls.
  *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     (cudaGetSymbolAddress) with that device current and keeps it; make
+ *     that first call before any stream capture.  The address is kept for
+ *     the life of the process, so do not call cudaDeviceReset (or otherwise
+ *     destroy the device's primary context) between calls: the array may
+ *     then sit elsewhere.
  */
 w4_status w4a16_gemv_noalloc(const void *X, int M, int N, int K, const uint32_t *packed,
                              const void *scales, const void *zeros, int mode, int group_size,
