@@ -12,9 +12,13 @@ reused only after every other set (>= 350 MB) has streamed through the
 
 The metric is whole-job HBM throughput: algorithmic bytes of the sweep
 (packed weights + fp16 scales/zeros + activations + outputs) / device time.
-Other hot-path rows (quantize-and-pack, transposed GEMV, tensor-core GEMM
-forward / transposed / with bias, fused QKV) are timed once each and
-reported under "rows".
+The same sweep transposed is reported under "sweep_transposed".  Other
+hot-path rows (quantize-and-pack, transposed GEMV, tensor-core GEMM forward /
+transposed / with bias, fused QKV) are timed once each under "rows", and
+every configuration of the workload list (the tiny case, the Llama-3.2-1B
+layers in three modes with quantize-and-pack, the Llama-2-7B QLoRA layers
+forward and transposed, the Llama-3-8B serving layers with bias at M = 1 ..
+1024) under "configs", each against its own roofline.
 
 Multi-GPU: one process per GPU (torchrun); each rank runs the whole sweep on
 its own GPU (independent problems, no data-path collective), value = bytes
@@ -209,23 +213,28 @@ def build_sweep(torch, w4, dev, sizes, seed=1234):
             gen.manual_seed(seed + 7 * M + ws["N"])
             X = torch.randn((M, ws["K"]), generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
             Y = torch.empty((M, ws["N"]), dtype=torch.bfloat16, device=dev)
+            dY = torch.randn((M, ws["N"]), generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+            dX = torch.empty((M, ws["K"]), dtype=torch.bfloat16, device=dev)
             nws = w4.w4_workspace_bytes(M, ws["N"], ws["K"], False)
-            cases.append(dict(M=M, set=ws, X=X, Y=Y, nws=nws,
-                              bytes=case_bytes(M, ws["N"], ws["K"], ws["G"])))
-    max_ws = max(c["nws"] for c in cases)
+            nws_t = w4.w4_workspace_bytes(M, ws["N"], ws["K"], True)
+            cases.append(dict(M=M, set=ws, X=X, Y=Y, dY=dY, dX=dX, nws=nws, nws_t=nws_t,
+                              bytes=case_bytes(M, ws["N"], ws["K"], ws["G"]),
+                              bytes_t=case_bytes(M, ws["N"], ws["K"], ws["G"], out_len=ws["K"])))
+    max_ws = max(max(c["nws"], c["nws_t"]) for c in cases)
     wsbuf = torch.empty(max(max_ws, 16), dtype=torch.uint8, device=dev)
     return cases, wsbuf
 
 
-def make_step(w4, cases, wsbuf, stream_ptr):
+def make_step(w4, cases, wsbuf, stream_ptr, transposed=False):
     lib = w4.library()
+    xk, yk, nk = ("dY", "dX", "nws_t") if transposed else ("X", "Y", "nws")
 
     def step():
         for c in cases:
             s = c["set"]
-            st = lib.w4a16_gemv(c["X"].data_ptr(), c["M"], s["N"], s["K"], s["p"].data_ptr(),
+            st = lib.w4a16_gemv(c[xk].data_ptr(), c["M"], s["N"], s["K"], s["p"].data_ptr(),
                                 s["s"].data_ptr(), s["z"].data_ptr(), w4.MODES[s["mode"]], s["g"],
-                                None, 0, c["Y"].data_ptr(), wsbuf.data_ptr(), c["nws"],
+                                None, 1 if transposed else 0, c[yk].data_ptr(), wsbuf.data_ptr(), c[nk],
                                 stream_ptr())
             if st != 0:
                 raise RuntimeError(f"w4a16_gemv failed: {lib.w4_status_string(st).decode()}")
@@ -355,6 +364,157 @@ def measure_rows(torch, w4, dev, peaks, stream):
     return rows
 
 
+def gemm_roofline(M, N, K, G, peaks, bias=False, out_len=None):
+    """Algorithmic work of one call and the time it needs at the measured
+    peaks: the slower of the tensor-core time for 2 M N K flops and the HBM
+    time for the packed weights, scales, zeros, activations and outputs."""
+    flops = 2.0 * M * N * K
+    byts = case_bytes(M, N, K, G, out_len=out_len) + (2 * (out_len or N) if bias else 0)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = byts / (peaks["hbm_gbs"] * 1e9)
+    return flops, byts, ("tensor" if t_tc >= t_hbm else "hbm"), max(t_tc, t_hbm)
+
+
+def measure_configs(torch, w4, dev, peaks, stream):
+    """Every configuration of the workload list, one timed call each (L2
+    flushed before it): the tiny correctness case, the Llama-3.2-1B layers in
+    three quantization modes with quantize-and-pack of each weight, the
+    Llama-2-7B QLoRA layers forward and transposed, and the Llama-3-8B
+    serving layers with bias at M = 1 .. 1024.  Each row reports the
+    fraction of its own roofline (the slower of tensor-core and HBM time)."""
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+
+    def rnd(shape, std=1.0):
+        return (torch.randn(shape, generator=gen, device=dev, dtype=torch.float32) * std).to(torch.bfloat16)
+
+    def timed(fn, reps=3):
+        fn()
+        ts = []
+        for _ in range(reps):
+            flush_l2(torch, flush)
+            torch.cuda._sleep(1_000_000)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts) * 1e-3          # seconds
+
+    def row(name, M, N, K, mode, g, fn, transposed=False, bias=False):
+        G = 1 if mode != "groupwise" else K // g
+        t = timed(fn)
+        out_len = K if transposed else N
+        flops, byts, bound, t_min = gemm_roofline(M, N, K, G, peaks, bias=bias, out_len=out_len)
+        return {"case": name, "M": M, "N": N, "K": K, "mode": mode, "g": g, "transposed": transposed,
+                "bias": bias, "us": round(t * 1e6, 2), "TFLOP/s": round(flops / t / 1e12, 2),
+                "GB/s": round(byts / t / 1e9, 1), "bound": bound, "frac": round(t_min / t, 4)}
+
+    out = {}
+    with torch.cuda.stream(stream):
+        # tiny correctness case: M = 4, N = 256, K = 512, g = 64, forward and transposed
+        N, K, g = 256, 512, 64
+        W = rnd((N, K), 0.02)
+        P, S, Z = w4.w4_quantize_pack(W, "groupwise", g)
+        X, dY = rnd((4, K)), rnd((4, N))
+        out["config1_tiny"] = [
+            row("tiny fwd", 4, N, K, "groupwise", g, lambda: w4.w4a16_gemv(X, P, S, Z, "groupwise", g, N=N, K=K)),
+            row("tiny t", 4, N, K, "groupwise", g,
+                lambda: w4.w4a16_gemv(dY, P, S, Z, "groupwise", g, N=N, K=K, transposed=True), transposed=True)]
+        # Llama-3.2-1B layers: three modes, M = 128, 512, 2048, and quantize + pack of each W
+        rows, qrows = [], []
+        for (N, K) in ((2048, 2048), (8192, 2048), (2048, 8192), (512, 2048), (128256, 2048)):
+            W = rnd((N, K), 0.02)
+            for mode, g in (("global", 0), ("rowwise", 0), ("groupwise", 64)):
+                G = 1 if mode != "groupwise" else K // g
+                t = timed(lambda: w4.w4_quantize_pack(W, mode, g))
+                qb = 2 * N * K + N * K // 2 + 4 * N * G + (2 * N * K if mode == "global" else 0)
+                qrows.append({"N": N, "K": K, "mode": mode, "g": g, "us": round(t * 1e6, 2),
+                              "GB/s": round(qb / t / 1e9, 1),
+                              "frac": round(qb / t / 1e9 / peaks["hbm_gbs"], 4)})
+                P, S, Z = w4.w4_quantize_pack(W, mode, g)
+                for M in (128, 512, 2048):
+                    X = rnd((M, K))
+                    rows.append(row("llama3.2-1b", M, N, K, mode, g,
+                                    lambda: w4.w4a16_gemm(X, P, S, Z, mode, g, N=N, K=K)))
+                del P, S, Z
+            del W
+        out["config3_llama32_1b"] = rows
+        out["config3_quantize_pack"] = qrows
+        # Llama-2-7B QLoRA layers: forward and transposed, g = 64 and per channel
+        rows = []
+        for (N, K) in ((3 * 4096, 4096), (4096, 4096), (11008, 4096), (4096, 11008)):
+            W = rnd((N, K), 0.02)
+            for mode, g in (("groupwise", 64), ("rowwise", 0)):
+                P, S, Z = w4.w4_quantize_pack(W, mode, g)
+                for M in (1024, 2048):
+                    X, dY = rnd((M, K)), rnd((M, N))
+                    rows.append(row("llama2-7b fwd", M, N, K, mode, g,
+                                    lambda: w4.w4a16_gemm(X, P, S, Z, mode, g, N=N, K=K)))
+                    rows.append(row("llama2-7b t", M, N, K, mode, g,
+                                    lambda: w4.w4a16_gemm(dY, P, S, Z, mode, g, N=N, K=K, transposed=True),
+                                    transposed=True))
+                del P, S, Z
+            del W
+        out["config4_llama2_7b"] = rows
+        # Llama-3-8B serving layers with bias, g = 128, M = 1 .. 1024
+        rows = []
+        for (N, K) in ((6144, 4096), (4096, 4096), (28672, 4096), (4096, 14336)):
+            W = rnd((N, K), 0.02)
+            P, S, Z = w4.w4_quantize_pack(W, "groupwise", 128)
+            b = rnd((N,), 0.01)
+            for M in (1, 4, 16, 64, 256, 1024):
+                X = rnd((M, K))
+                rows.append(row("llama3-8b", M, N, K, "groupwise", 128,
+                                lambda: w4.w4a16_gemm(X, P, S, Z, "groupwise", 128, N=N, K=K, bias=b), bias=True))
+            del W, P, S, Z
+        out["config5_llama3_8b_bias"] = rows
+        del flush
+    torch.cuda.synchronize()
+    return out
+
+
+def host_cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def single_thread_oracle(sizes):
+    """The oracle on one host thread: the tiny correctness case (whole) and
+    one call of the decode sweep per N = K (64 output rows, M = 4)."""
+    code = (
+        "import time, json, oracle\n"
+        "from gemv_w4a16_groupwise_b200 import synth\n"
+        "res = {}\n"
+        "W = synth.weights(256, 512, 0); p, s, z = oracle.quantize_pack(W, 'groupwise', 64)\n"
+        "X = synth.activations(4, 512, 0); t0 = time.perf_counter()\n"
+        "oracle.linear(X, p, s, z, 'groupwise', 64, 256, 512)\n"
+        "res['tiny_fwd_s'] = time.perf_counter() - t0\n"
+        f"for N in {list(sizes)}:\n"
+        "    W = synth.weights(64, N, 1); p, s, z = oracle.quantize_pack(W, 'groupwise', 128)\n"
+        "    X = synth.activations(4, N, 1); t0 = time.perf_counter()\n"
+        "    oracle.linear(X, p, s, z, 'groupwise', 128, 64, N)\n"
+        "    dt = time.perf_counter() - t0\n"
+        "    res[f'sweep_M4_N{N}_64rows_s'] = dt\n"
+        "print(json.dumps(res))\n")
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    try:
+        r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True,
+                           timeout=120)
+        return json.loads(r.stdout.strip().splitlines()[-1])
+    except (subprocess.SubprocessError, ValueError, IndexError):
+        return None
+
+
 def cpu_baseline(seconds_budget, sizes):
     """The oracle, as it stands, on a bounded sample of the sweep: for every
     case it computes R output columns (R sampled weight rows, quantized by the
@@ -449,6 +609,20 @@ def run_ours(args):
     ms_step = max_over_ranks(dist, ms_step, dev)
     value = weak_value(ws_, bytes_step, ms_step)
 
+    # the same sweep, transposed (dX = dY . dequant(W)), timed the same way
+    step_t = make_step(w4, cases, wsbuf, stream_ptr, transposed=True)
+    graph_t = capture(torch, step_t, stream)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            graph_t.replay()
+    ms_t = time_graph(torch, graph_t, max(10, args.steps // 3), stream)
+    bytes_t = sum(c["bytes_t"] for c in cases)
+    sweep_t = {"GB/s": round(bytes_t / (ms_t * 1e-3) / 1e9, 2),
+               "frac": round(bytes_t / (ms_t * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+               "ms_per_step": round(ms_t, 5), "calls": len(cases),
+               "workload": "the decode sweep transposed: dY [M, N] -> dX [M, K], same weights"}
+    del graph_t
+
     # per-case device times (20 back-to-back calls of one case; L2 warm for the
     # small sets -- reported for context, the headline is the cold sweep).
     # The 20 calls sit in one graph, so the host's launch rate does not
@@ -459,7 +633,8 @@ def run_ours(args):
         g1 = capture(torch, one, stream)
         msc = time_graph(torch, g1, 3, stream) / 20
         per_case.append({"M": c["M"], "N": c["set"]["N"], "K": c["set"]["K"], "mode": c["set"]["mode"],
-                         "us": round(msc * 1e3, 2), "GB/s": round(c["bytes"] / msc / 1e6, 1)})
+                         "us": round(msc * 1e3, 2), "GB/s": round(c["bytes"] / msc / 1e6, 1),
+                         "frac": round(c["bytes"] / msc / 1e6 / peaks["hbm_gbs"], 4)})
         del g1
 
     # end to end through the public API with host buffers
@@ -494,9 +669,10 @@ def run_ours(args):
     ms_e2e = max_over_ranks(dist, a0.elapsed_time(a1) / e2e_steps, dev)
     e2e_value = weak_value(ws_, bytes_step, ms_e2e)
 
-    rows = None
+    rows = configs = None
     if not args.no_rows:
         rows = measure_rows(torch, w4, dev, peaks, stream)
+        configs = measure_configs(torch, w4, dev, peaks, stream)
     del graph
 
     err = w4.w4_device_error()
@@ -505,6 +681,8 @@ def run_ours(args):
         cpu = None
         if ws_ == 1 and not args.no_cpu:
             cpu = cpu_baseline(args.cpu_seconds, sizes)
+            cpu["cpu_model"] = host_cpu_model()
+            cpu["single_thread"] = single_thread_oracle(sizes)
         calls = len(cases)
         alg_per_call = bytes_step / calls
         traffic = committed_traffic()
@@ -556,7 +734,9 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "device_error_word": err,
             "cases": per_case,
+            "sweep_transposed": sweep_t,
             "rows": rows,
+            "configs": configs,
         }
     if dist:
         dist.barrier()

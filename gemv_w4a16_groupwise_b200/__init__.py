@@ -72,6 +72,12 @@ def library():
             lib.w4_last_cuda_error.restype = ctypes.c_char_p
             lib.w4_launch_count.argtypes = []
             lib.w4_launch_count.restype = ctypes.c_uint64
+            lib.w4_set_debug_checks.argtypes = [I]
+            lib.w4_set_debug_checks.restype = I
+            lib.w4_debug_set_wait_limit.argtypes = [ctypes.c_ulonglong]
+            lib.w4_debug_set_wait_limit.restype = I
+            lib.w4_debug_withhold_stage.argtypes = [I]
+            lib.w4_debug_withhold_stage.restype = I
             _lib = lib
     return _lib
 
@@ -197,6 +203,25 @@ def w4a16_gemv(A, packed, scales, zeros, mode="groupwise", group_size: int = 128
 def w4_launch_count() -> int:
     """Kernel launches issued by the library in this process (host counter)."""
     return int(library().w4_launch_count())
+
+
+def w4_set_debug_checks(on: bool) -> None:
+    """Debug mode: w4_quantize_pack rejects NaN / Inf weights (W4_ERR_INVALID_ARG)."""
+    library().w4_set_debug_checks(1 if on else 0)
+
+
+def w4_debug_set_wait_limit(ns: int) -> None:
+    """Limit of a kernel's bounded waits on the current device (0 = the default 2 s)."""
+    st = library().w4_debug_set_wait_limit(int(ns))
+    if st != 0:
+        raise W4Error(st, "w4_debug_set_wait_limit")
+
+
+def w4_debug_withhold_stage(stage: int) -> None:
+    """Failure injection: the GEMV producers skip stage `stage` (-1: none)."""
+    st = library().w4_debug_withhold_stage(int(stage))
+    if st != 0:
+        raise W4Error(st, "w4_debug_withhold_stage")
 
 
 def w4_device_error() -> int:

@@ -24,6 +24,15 @@ enum DeviceError : unsigned int {
     kErrTimeoutAccum = 4,       // the epilogue waited too long for the accumulator
 };
 
+// Debug controls, set from the host (w4_debug_set_wait_limit,
+// w4_debug_withhold_stage): how long a bounded wait may last, and a stage
+// index whose copy the GEMV producers leave unissued (-1: none), so that a
+// test can make a wait run out without any fault.
+__device__ unsigned long long g_wait_limit_ns = 2000000000ull;
+__device__ int g_withhold_stage = -1;
+// Set by the debug-mode input check when it meets a NaN or an infinity.
+__device__ unsigned int g_nonfinite;
+
 __device__ __forceinline__ void record_error(unsigned int code) {
     atomicCAS(&g_error_word, 0u, code);
 }

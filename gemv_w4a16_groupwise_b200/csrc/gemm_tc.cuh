@@ -493,6 +493,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // a role gave up: let copies and mma already issued land (bounded)
+        // before the tensor memory and the CTA's shared memory are released
+        const unsigned long long t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 1000000ull) {
+        }
+    }
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();

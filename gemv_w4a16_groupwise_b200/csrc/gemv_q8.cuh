@@ -370,15 +370,16 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
     if (warp == kQW) {
         // ------------------------------------------------------ producer
-        int s = 0;
+        int s = 0, it = 0;
         uint32_t round = 0;
         bool alive = true;
+        const int withhold = g_withhold_stage;     // -1 unless a test injects a lost stage
         for (int c = 0; c < nch && alive; ++c) {
             const int r0 = chunk_lo(c), rc = chunk_lo(c + 1) - r0;
             for (int ks = 0; ks < a.nks && alive; ++ks) {
                 const int k0 = k_slice + ks * kMK;
                 const int x2 = SZ == kSzTma2d ? group_of(k0) & ~7 : 0;
-                for (int r = 0; r < rc; ++r) {
+                for (int r = 0; r < rc; ++r, ++it) {
                     if (round > 0) {
                         alive = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&empty[s], (round - 1) & 1u, abort_flag,
                                                                           kErrTimeoutEmpty));
@@ -386,6 +387,15 @@ __global__ void __launch_bounds__(kQThreads, 1)
                     }
                     uint8_t* sd = ring + s * SB;
                     const int row0 = (r0 + r) * kMR;
+                    if (it == withhold) {
+                        // injected loss: this stage's copy is never issued, so its
+                        // consumers' bounded waits run out; nothing is left in flight
+                        if (++s == NS) {
+                            s = 0;
+                            ++round;
+                        }
+                        continue;
+                    }
                     if (SZ == kSzCopy) {
                         const int arr = lane >> 4, rr = lane & 15;
                         const long long h0 = (static_cast<long long>(row0 + rr) * a.sz_row + group_of(k0)) & ~1ll;

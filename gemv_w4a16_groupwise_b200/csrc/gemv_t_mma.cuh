@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(kTMThreads, 1)
         // that a last stage carries meet c = 0
         int s = 0;
         uint32_t round = 0;
+        const int withhold = g_withhold_stage;     // -1 unless a test injects a lost stage
         for (int b = 0; b < nst; ++b) {
             if (round > 0) {
                 const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&empty[s], (round - 1) & 1u, abort_flag,
@@ -150,6 +151,14 @@ __global__ void __launch_bounds__(kTMThreads, 1)
             }
             uint8_t* sd = ring + s * kStage;
             const int row0 = r0 + b * kTMRows;
+            if (b == withhold) {
+                // injected loss: the copy is never issued (nothing in flight)
+                if (++s == NS) {
+                    s = 0;
+                    ++round;
+                }
+                continue;
+            }
             if (SZ == kSzTma2d)
                 tma_issue_elected<3>(&full[s], kTMRows * kPitch + kSzTx, sd, &wmap, k0 / 16, row0, sd + kSzOff,
                                      &smap, x_sz, row0, sd + kSzOff + 1024, &zmap, x_sz, row0);

@@ -230,4 +230,20 @@ __global__ void __launch_bounds__(256) global_quantize_kernel(
     }
 }
 
+// Debug-mode input check: sets g_nonfinite when any of the n bf16 values is
+// a NaN or an infinity (exponent field all ones).  n is a multiple of 8.
+__global__ void __launch_bounds__(256) nonfinite_check_kernel(const uint16_t* __restrict__ W, long long n) {
+    const long long n8 = n / 8;
+    bool bad = false;
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(W) + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            bad = bad || ((w[j] & 0x7F80u) == 0x7F80u) || ((w[j] & 0x7F800000u) == 0x7F800000u);
+    }
+    if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicOr(&g_nonfinite, 1u);
+}
+
 }  // namespace w4

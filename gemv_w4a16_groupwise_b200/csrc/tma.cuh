@@ -7,9 +7,9 @@
 
 namespace w4 {
 
-// A wait that has not completed after this long is abandoned: the kernel
-// records the reason in g_error_word and unwinds instead of hanging.
-constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
+// A wait that has not completed after g_wait_limit_ns (2 s unless a test
+// shortens it) is abandoned: the kernel records the reason in g_error_word
+// and unwinds instead of hanging.
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -67,18 +67,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, ui
 }
 
 // Wait for the phase with the given parity to complete.  Returns false (and
-// records `err`) when the wait exceeds kWaitTimeoutNs or when another role
+// records `err`) when the wait exceeds g_wait_limit_ns or when another role
 // of the CTA has already raised *abort; the caller then unwinds.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort, unsigned int err) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long start = global_timer_ns();
+    const unsigned long long limit = g_wait_limit_ns;
     for (;;) {
         // suspended for at most 20 us per test, so the abort flag and the
         // time limit are still checked often
         if (mbar_try_wait(bar, parity, 20000u)) return true;
         if (*abort) return false;
-        if (global_timer_ns() - start > kWaitTimeoutNs) {
+        if (global_timer_ns() - start > limit) {
             record_error(err);
             *abort = 1;
             return false;

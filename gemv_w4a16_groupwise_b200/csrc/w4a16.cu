@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "gemm_simple.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "gemv_mma.cuh"
@@ -23,6 +24,7 @@ namespace {
 using namespace w4;
 
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+std::atomic<int> g_debug_checks{0};
 
 // ----------------------------------------------------------------- device info
 struct DeviceInfo {
@@ -828,6 +830,7 @@ TcPlan plan_tc(int M, int N, int K, int transposed, int sms) {
 }
 
 size_t gemm_tc_workspace_bytes(int M, int N, int K, int transposed, int sms) {
+    if (K % 32 != 0 || (transposed && N % 8 != 0)) return 0;   // the plain kernel needs none
     return plan_tc(M, N, K, transposed, sms).ws;
 }
 
@@ -852,9 +855,33 @@ w4_status launch_tc_bn(int BN, const CUtensorMap& pm, const CUtensorMap& bm, con
     }
 }
 
+// Shapes whose rows TMA cannot stream: the plain CUDA-core kernel.
+w4_status run_gemm_simple(const TcProblem& p, cudaStream_t st) {
+    GemmSimpleArgs a;
+    a.A = static_cast<const uint16_t*>(p.A);
+    a.packed = p.packed;
+    a.S = static_cast<const __half*>(p.S);
+    a.Z = static_cast<const __half*>(p.Z);
+    a.bias = static_cast<const uint16_t*>(p.bias);
+    a.Y = static_cast<uint16_t*>(p.Y);
+    a.M = p.M;
+    a.N = p.N;
+    a.K = p.K;
+    a.g = p.g;
+    a.G = p.G;
+    a.sz_row = p.sz_row;
+    const int L = p.transposed ? p.K : p.N;
+    const dim3 grid((L + kGsTile - 1) / kGsTile, (p.M + kGsTile - 1) / kGsTile);
+    if (p.transposed)
+        gemm_simple_kernel<true><<<grid, 256, 0, st>>>(a);
+    else
+        gemm_simple_kernel<false><<<grid, 256, 0, st>>>(a);
+    return launch_status();
+}
+
 w4_status run_gemm_tc(const TcProblem& p, void* ws, size_t ws_bytes, cudaStream_t st) {
-    if (p.K % 32 != 0) return W4_ERR_UNSUPPORTED;      // packed rows must be 16-byte strided
-    if (p.transposed && p.N % 8 != 0) return W4_ERR_UNSUPPORTED;  // dY rows 16-byte strided
+    // packed rows (and dY rows when transposed) must be 16-byte strided for TMA
+    if (p.K % 32 != 0 || (p.transposed && p.N % 8 != 0)) return run_gemm_simple(p, st);
     const DeviceInfo di = device_info(current_device());
     const TcPlan plan = plan_tc(p.M, p.N, p.K, p.transposed, di.sms);
     if (plan.ws > ws_bytes || (plan.ws > 0 && ws == nullptr)) return W4_ERR_WORKSPACE;
@@ -975,6 +1002,23 @@ w4_status w4_quantize_pack(const void* W, int N, int K, int mode, int group_size
     if (workspace_bytes < need || (need > 0 && !workspace)) return W4_ERR_WORKSPACE;
     if (need > 0 && !aligned16(workspace)) return W4_ERR_ALIGNMENT;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (g_debug_checks.load(std::memory_order_relaxed)) {
+        // reject NaN / Inf weights before quantizing (synchronizes the stream)
+        unsigned int flag = 0;
+        if (cudaMemcpyToSymbolAsync(w4::g_nonfinite, &flag, sizeof flag, 0, cudaMemcpyHostToDevice, st) !=
+            cudaSuccess)
+            return W4_ERR_CUDA;
+        const long long n = static_cast<long long>(N) * K;
+        const int blocks = static_cast<int>(std::min<long long>((n / 8 + 255) / 256, 1024));
+        nonfinite_check_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint16_t*>(W), n);
+        s = launch_status();
+        if (s != W4_OK) return s;
+        if (cudaMemcpyFromSymbolAsync(&flag, w4::g_nonfinite, sizeof flag, 0, cudaMemcpyDeviceToHost, st) !=
+                cudaSuccess ||
+            cudaStreamSynchronize(st) != cudaSuccess)
+            return W4_ERR_CUDA;
+        if (flag) return W4_ERR_INVALID_ARG;
+    }
     const uint16_t* w = static_cast<const uint16_t*>(W);
     __half* sc = static_cast<__half*>(scales);
     __half* ze = static_cast<__half*>(zeros);
@@ -1087,6 +1131,29 @@ w4_status w4a16_gemv_noalloc(const void* X, int M, int N, int K, const uint32_t*
 }
 
 const char* w4_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
+
+w4_status w4_set_debug_checks(int on) {
+    g_debug_checks.store(on ? 1 : 0, std::memory_order_relaxed);
+    return W4_OK;
+}
+
+w4_status w4_debug_set_wait_limit(unsigned long long ns) {
+    const unsigned long long v = ns ? ns : 2000000000ull;
+    if (cudaMemcpyToSymbol(w4::g_wait_limit_ns, &v, sizeof v) != cudaSuccess) {
+        g_last_cuda_error = cudaGetLastError();
+        return W4_ERR_CUDA;
+    }
+    return W4_OK;
+}
+
+w4_status w4_debug_withhold_stage(int stage) {
+    const int v = stage < 0 ? -1 : stage;
+    if (cudaMemcpyToSymbol(w4::g_withhold_stage, &v, sizeof v) != cudaSuccess) {
+        g_last_cuda_error = cudaGetLastError();
+        return W4_ERR_CUDA;
+    }
+    return W4_OK;
+}
 
 uint64_t w4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 

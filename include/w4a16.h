@@ -205,6 +205,30 @@ w4_status w4a16_gemv_noalloc(const void *X, int M, int N, int K, const uint32_t 
                              const void *scales, const void *zeros, int mode, int group_size,
                              const void *bias, void *Y, void *stream);
 
+/*
+ * w4_set_debug_checks -- debug mode for input checks (off by default;
+ * process-wide).  When on, w4_quantize_pack first scans W for NaN and
+ * infinities and returns W4_ERR_INVALID_ARG, quantizing nothing, if it
+ * finds any; the scan synchronizes the call's stream, so keep it out of
+ * stream capture.  With it off, non-finite weights give undefined codes.
+ * (vLLM "Adding bias epilogue support for cutlass_scaled_mm": an opaque
+ * "Error Internal" is what distinct statuses avoid.)
+ */
+w4_status w4_set_debug_checks(int on);
+
+/*
+ * Failure injection for testing the bounded waits (current device; both
+ * synchronous).  w4_debug_set_wait_limit sets how long a kernel's bounded
+ * wait may last before the kernel gives up (0 restores the default, 2 s).
+ * w4_debug_withhold_stage makes the producer of every CTA of the GEMV
+ * kernels skip the copy of its stage number `stage` (-1: none, the default)
+ * without issuing it, so the consumers' waits run out, the kernel unwinds,
+ * and w4_device_error reports W4_ERR_TIMEOUT.  Nothing is left in flight and
+ * the context stays usable.  For tests only.
+ */
+w4_status w4_debug_set_wait_limit(unsigned long long ns);
+w4_status w4_debug_withhold_stage(int stage);
+
 #ifdef __cplusplus
 }
 #endif

@@ -154,17 +154,21 @@ def test_gemm_bias(cuda_device, M, transposed):
     assert_close(y, ref, f"gemm bias M={M} t={transposed}")
 
 
-def test_transposed_gemm_needs_aligned_n(cuda_device):
-    """Transposed tensor-core path with N % 8 != 0 is reported, not computed."""
-    w4 = lib()
-    dev = cuda_device
-    N, K = 300, 512
-    W, p, s, z = quantized_case(N, K, "groupwise", 64, 3)
-    dY = to_dev_bf16(synth.grads(16, N, 3), dev)
-    with pytest.raises(w4.W4Error) as ei:
-        w4.w4a16_gemm(dY, to_dev_packed(p, dev), to_dev_f16(s, dev), to_dev_f16(z, dev),
-                      "groupwise", 64, N=N, K=K, transposed=True)
-    assert ei.value.status == 2
+@pytest.mark.parametrize("M,N,K,mode,g,transposed,bias", [
+    (5, 300, 520, "groupwise", 8, False, True),       # K % 32 != 0: packed rows not 16-byte strided
+    (64, 100, 1000, "rowwise", 0, False, False),
+    (130, 257, 264, "global", 0, True, False),         # transposed, N % 8 != 0: dY rows not 16-byte strided
+    (17, 300, 512, "groupwise", 64, True, True),
+    (200, 68, 2056, "groupwise", 8, True, False),      # both
+])
+def test_gemm_shapes_tma_cannot_stream(cuda_device, M, N, K, mode, g, transposed, bias):
+    """Shapes whose rows TMA cannot stream run the plain CUDA-core kernel."""
+    import gemv_w4a16_groupwise_b200 as w4
+    y, ref = run_matmul("w4a16_gemm", M, N, K, mode, g, transposed, bias=bias,
+                        seed=synth.config_seed("simple", M, N, K, mode, g, transposed), dev=cuda_device,
+                        structure=True)
+    assert w4.w4_workspace_bytes(M, N, K, transposed) == 0
+    assert_close(y, ref, f"gemm simple M={M} N={N} K={K} {mode} g={g} t={transposed}")
 
 
 def test_bias_difference(cuda_device):
