@@ -803,9 +803,13 @@ TcPlan plan_tc(int M, int N, int K, int transposed, int sms) {
     const int R = p.tiles % P;
     p.F = p.tiles;
     if (R > 0) {
-        // a tile's time in microseconds, roughly: a 64-k block of 128 x BN
-        // takes ~0.75 us per 256 tokens at the rates this kernel reaches
-        const double tile_us = num_kb * (p.BN / 256.0) * 0.75;
+        // a tile's time in microseconds, roughly: the slower of its tensor
+        // work (a 64-k block of 128 x BN takes ~0.75 us per 256 tokens at the
+        // rates this kernel reaches) and its bytes (128 packed rows and BN
+        // activation rows over the reduction) at one SM's share of HBM
+        // (~40 GB/s); small tiles are bound by the latter
+        const double bytes = static_cast<double>(red) * (kTcBM / 2.0 + 2.0 * p.BN);
+        const double tile_us = std::max(num_kb * (p.BN / 256.0) * 0.75, bytes / 40.0e3);
         double best = 0.0;
         int bestS = 1;
         for (int S = 2; S <= std::min(16, num_kb / 4); ++S) {
