@@ -10,7 +10,9 @@ patterns.
 Functions, in the order the method applies them (each follows the page and
 section named in its docstring):
 
-* :func:`quantize`  -- bf16 W -> uint4 codes, fp16 scales and zeros
+* :func:`quantize`  -- bf16 W -> uint4 codes, fp16 scales and zeros (or, with
+  ``zero="float"`` / ``meta="bf16"``, a fractional zero point / bf16 scales and
+  zeros: the HQQ-style variant)
 * :func:`pack` / :func:`unpack` -- eight codes per uint32 along K
 * :func:`dequant`   -- w_hat = (q - z) * s in fp64
 * :func:`linear`    -- Y = X @ w_hat^T (+ bias), fp64 accumulation
@@ -34,6 +36,9 @@ MODE_GLOBAL = 0
 MODE_ROWWISE = 1
 MODE_GROUPWISE = 2
 MODES = {"global": MODE_GLOBAL, "rowwise": MODE_ROWWISE, "groupwise": MODE_GROUPWISE}
+# format flags or-ed into the mode (see w4a16_oracle.c)
+FLAG_FLOAT_ZERO = 0x10
+FLAG_META_BF16 = 0x20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "w4a16_oracle.c")
@@ -88,8 +93,11 @@ def _c(a, dtype):
     return np.ascontiguousarray(a, dtype=dtype)
 
 
-def _mode(mode):
-    return MODES[mode] if isinstance(mode, str) else int(mode)
+def _mode(mode, zero: str = "int", meta: str = "fp16"):
+    m = MODES[mode] if isinstance(mode, str) else int(mode)
+    if zero not in ("int", "float") or meta not in ("fp16", "bf16"):
+        raise ValueError(f"zero must be 'int' or 'float' and meta 'fp16' or 'bf16', got {zero!r}, {meta!r}")
+    return m | (FLAG_FLOAT_ZERO if zero == "float" else 0) | (FLAG_META_BF16 if meta == "bf16" else 0)
 
 
 def groups_per_row(K: int, mode, g: int) -> int:
@@ -98,7 +106,7 @@ def groups_per_row(K: int, mode, g: int) -> int:
 
 def meta_shape(N: int, K: int, mode, g: int):
     """Shape of the scale / zero arrays: [N,G], [N,1] or [1,1]."""
-    m = _mode(mode)
+    m = _mode(mode) & 0x0F
     if m == MODE_GLOBAL:
         return (1, 1)
     if m == MODE_ROWWISE:
@@ -118,11 +126,14 @@ def f64_to_bf16(x: float) -> int:
     return int(_load().oracle_f64_to_bf16(float(x)))
 
 
-def quantize(W_bf16: np.ndarray, mode, g: int = 0):
-    """Quantize bf16 W [N,K] -> (codes uint8 [N,K], s fp16-bits, z fp16-bits).
+def quantize(W_bf16: np.ndarray, mode, g: int = 0, zero: str = "int", meta: str = "fp16"):
+    """Quantize bf16 W [N,K] -> (codes uint8 [N,K], s bits, z bits).
 
     Asymmetric min-max to uint4 per group (llm-quantization, Objective 1:
     GLOBAL / ROWWISE / GROUPWISE modes), integer zero point, fp16 s and z.
+    ``zero="float"``: fractional zero point z = -min / s and
+    q = clamp(rint(w / s + z), 0, 15) (the HQQ-style quantizer of "Re-write
+    HQQ Fused Gemm Transpose"); ``meta="bf16"``: s and z stored as bf16.
     """
     W = _c(W_bf16, np.uint16)
     N, K = W.shape
@@ -130,7 +141,7 @@ def quantize(W_bf16: np.ndarray, mode, g: int = 0):
     q = np.empty((N, K), np.uint8)
     s = np.empty(shape, np.uint16)
     z = np.empty(shape, np.uint16)
-    rc = _load().oracle_quantize(_ptr(W), N, K, _mode(mode), int(g), _ptr(q), _ptr(s), _ptr(z))
+    rc = _load().oracle_quantize(_ptr(W), N, K, _mode(mode, zero, meta), int(g), _ptr(q), _ptr(s), _ptr(z))
     if rc != 0:
         raise ValueError(f"oracle_quantize: bad arguments N={N} K={K} mode={mode} g={g}")
     return q, s, z
@@ -155,17 +166,17 @@ def unpack(packed: np.ndarray, K: int) -> np.ndarray:
     return out
 
 
-def dequant(packed, s, z, mode, g: int, K: int) -> np.ndarray:
-    """w_hat [N,K] fp64 = (q - z) * s."""
+def dequant(packed, s, z, mode, g: int, K: int, meta: str = "fp16") -> np.ndarray:
+    """w_hat [N,K] fp64 = (q - z) * s (s, z read as fp16, or bf16 with meta="bf16")."""
     p = _c(packed, np.uint32)
     N = p.shape[0]
     out = np.empty((N, K), np.float64)
     _load().oracle_dequant(_ptr(p), _ptr(_c(s, np.uint16)), _ptr(_c(z, np.uint16)), N, K,
-                           _mode(mode), int(g), _ptr(out))
+                           _mode(mode, "int", meta), int(g), _ptr(out))
     return out
 
 
-def linear(X_bf16, packed, s, z, mode, g: int, N: int, K: int, bias=None, cols=None):
+def linear(X_bf16, packed, s, z, mode, g: int, N: int, K: int, bias=None, cols=None, meta: str = "fp16"):
     """Y = X @ w_hat^T (+ bias), fp64 accumulation -> (y64, y_bf16_bits).
 
     With ``cols`` (output column indices n) only those columns are computed.
@@ -179,12 +190,12 @@ def linear(X_bf16, packed, s, z, mode, g: int, N: int, K: int, bias=None, cols=N
     ybf = np.empty((M, nc), np.uint16)
     b = None if bias is None else _c(bias, np.uint16)
     _load().oracle_linear(_ptr(X), M, K, _ptr(_c(packed, np.uint32)), _ptr(_c(s, np.uint16)),
-                          _ptr(_c(z, np.uint16)), N, _mode(mode), int(g), _ptr(b), _ptr(c), nc,
+                          _ptr(_c(z, np.uint16)), N, _mode(mode, "int", meta), int(g), _ptr(b), _ptr(c), nc,
                           _ptr(y64), _ptr(ybf))
     return y64, ybf
 
 
-def linear_t(dY_bf16, packed, s, z, mode, g: int, N: int, K: int, bias=None, cols=None):
+def linear_t(dY_bf16, packed, s, z, mode, g: int, N: int, K: int, bias=None, cols=None, meta: str = "fp16"):
     """dX = dY @ w_hat (+ bias) from the same packed weights -> (x64, x_bf16_bits).
 
     With ``cols`` (output column indices k) only those columns are computed.
@@ -198,12 +209,12 @@ def linear_t(dY_bf16, packed, s, z, mode, g: int, N: int, K: int, bias=None, col
     ybf = np.empty((M, nc), np.uint16)
     b = None if bias is None else _c(bias, np.uint16)
     _load().oracle_linear_t(_ptr(dY), M, N, _ptr(_c(packed, np.uint32)), _ptr(_c(s, np.uint16)),
-                            _ptr(_c(z, np.uint16)), K, _mode(mode), int(g), _ptr(b), _ptr(c), nc,
+                            _ptr(_c(z, np.uint16)), K, _mode(mode, "int", meta), int(g), _ptr(b), _ptr(c), nc,
                             _ptr(y64), _ptr(ybf))
     return y64, ybf
 
 
-def quantize_pack(W_bf16, mode, g: int = 0):
+def quantize_pack(W_bf16, mode, g: int = 0, zero: str = "int", meta: str = "fp16"):
     """quantize then pack: -> (packed uint32 [N,K/8], s, z)."""
-    q, s, z = quantize(W_bf16, mode, g)
+    q, s, z = quantize(W_bf16, mode, g, zero, meta)
     return pack(q), s, z

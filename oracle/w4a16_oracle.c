@@ -17,10 +17,22 @@
  *          q = clamp(rint(w / s) + z, 0, 15)
  *      every step in IEEE fp32, round-half-even, no contraction; clamps are
  *      taken with fmaxf/fminf so that a NaN lands on 0 on every platform.
+ *      Two format flags, or-ed into the mode, give the variants with a
+ *      fractional zero point and with bf16 metadata ("Re-write HQQ Fused
+ *      Gemm Transpose": the HQQ fused GEMM, whose quantizer keeps a float
+ *      zero point; fp16 or bf16 scales are both allowed):
+ *        FLOAT_ZERO  z = meta_rn(-min / s), not rounded to an integer or
+ *                    clamped to [0, 15] (only to the finite range of the
+ *                    metadata type), and q = clamp(rint(w / s + z), 0, 15):
+ *                    the sum is rounded, as round(w / s + z) reads;
+ *        META_BF16   s and z are stored as bf16 instead of fp16: every
+ *                    meta_rn above is a bf16 rounding, and the degenerate
+ *                    group's s is bf16_rn(max(|min|, 2^-14)).
  *   2. pack      -- "packs the quantized matrix into INT8 or INT32": eight
  *      codes per uint32 along K, code i of word j at bits 4i..4i+3, which
  *      is byte-identical to two codes per byte with the low nibble first.
- *   3. dequant   -- w_hat = (q - z) * s   (exact in fp32 and fp64).
+ *   3. dequant   -- w_hat = (q - z) * s   (exact in fp64; also in fp32 when
+ *      z is an integer).
  *   4. matmul    -- Y = X_bf16 @ W_int4^T  (Objective 2), accumulated in
  *      fp64 over ascending k, plus an optional bias per output column
  *      (vLLM "Adding bias epilogue support for cutlass_scaled_mm": bias
@@ -31,9 +43,9 @@
  *      accumulated in fp64 over ascending n.
  *
  * Layouts: W bf16 [N,K] row-major; codes uint8 [N,K]; packed uint32
- * [N,K/8]; scales and zeros fp16 bit patterns [N,G] row-major with G = K/g
- * (ROWWISE [N,1], GLOBAL [1,1]).  bf16 and fp16 values cross this API as
- * uint16 bit patterns.
+ * [N,K/8]; scales and zeros fp16 (or bf16) bit patterns [N,G] row-major
+ * with G = K/g (ROWWISE [N,1], GLOBAL [1,1]).  bf16 and fp16 values cross
+ * this API as uint16 bit patterns.
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fPIC -shared (no -ffast-math).
  * OpenMP runs over output rows or columns only; each output element is
@@ -48,6 +60,9 @@
 #define MODE_GLOBAL 0
 #define MODE_ROWWISE 1
 #define MODE_GROUPWISE 2
+#define MODE_BASE_MASK 0x0F
+#define FLAG_FLOAT_ZERO 0x10   /* fractional zero point */
+#define FLAG_META_BF16 0x20    /* s and z stored as bf16 */
 
 /* Threads an OpenMP region of this library uses (for reporting). */
 int oracle_num_threads(void) { return omp_get_max_threads(); }
@@ -108,10 +123,23 @@ uint16_t oracle_f64_to_bf16(double d)
 
 /* -------------------------------------------------------------- quantize */
 
+/* The metadata type's value of a bit pattern, and the nearest pattern to an
+ * fp32 value (ties to even; bf16 from the exact double of the value). */
+static float meta_value(uint16_t b, int flags)
+{
+    return (flags & FLAG_META_BF16) ? bf16_bits_to_f32(b) : (float)bits_to_f16(b);
+}
+
+static uint16_t meta_rn(float v, int flags)
+{
+    return (flags & FLAG_META_BF16) ? oracle_f64_to_bf16((double)v) : f16_to_bits((_Float16)v);
+}
+
 /* One group of n weights (fp32 values of bf16 inputs) at stride 1.
- * Writes n codes and the fp16 bit patterns of s and z. */
+ * Writes n codes and the bit patterns of s and z (fp16, or bf16 with
+ * FLAG_META_BF16). */
 static void quantize_group(const float *w, long n, uint8_t *q, uint16_t *s_bits,
-                           uint16_t *z_bits)
+                           uint16_t *z_bits, int flags)
 {
     float mn = w[0], mx = w[0];
     for (long i = 1; i < n; ++i) {
@@ -120,9 +148,24 @@ static void quantize_group(const float *w, long n, uint8_t *q, uint16_t *s_bits,
     }
     float range = mx - mn;
     float s32 = range / 15.0f;
-    _Float16 s = (_Float16)s32;
-    if ((float)s == 0.0f) s = (_Float16)fmaxf(fabsf(mn), 0x1p-14f);
-    float sf = (float)s;
+    uint16_t sb = meta_rn(s32, flags);
+    if (meta_value(sb, flags) == 0.0f) sb = meta_rn(fmaxf(fabsf(mn), 0x1p-14f), flags);
+    float sf = meta_value(sb, flags);
+    if (flags & FLAG_FLOAT_ZERO) {
+        /* z = -min / s, kept fractional; only kept finite in its type */
+        const float zmax = (flags & FLAG_META_BF16) ? 0x1.FEp127f : 65504.0f;
+        float z32 = fminf(fmaxf(-mn / sf, -zmax), zmax);
+        uint16_t zb = meta_rn(z32, flags);
+        float zf = meta_value(zb, flags);
+        for (long i = 0; i < n; ++i) {
+            float u = w[i] / sf + zf;
+            float t = fminf(fmaxf(rintf(u), 0.0f), 15.0f);
+            q[i] = (uint8_t)(int)t;
+        }
+        *s_bits = sb;
+        *z_bits = zb;
+        return;
+    }
     float zf = fminf(fmaxf(rintf(-mn / sf), 0.0f), 15.0f);
     int zi = (int)zf;
     for (long i = 0; i < n; ++i) {
@@ -130,13 +173,14 @@ static void quantize_group(const float *w, long n, uint8_t *q, uint16_t *s_bits,
         t = fminf(fmaxf(t, 0.0f), 15.0f);
         q[i] = (uint8_t)(int)t;
     }
-    *s_bits = f16_to_bits(s);
-    *z_bits = f16_to_bits((_Float16)zi);
+    *s_bits = sb;
+    *z_bits = meta_rn((float)zi, flags);
 }
 
 /* Number of groups per row (G) for a mode; 0 on invalid arguments. */
 long oracle_groups_per_row(long K, int mode, long g)
 {
+    mode &= MODE_BASE_MASK;
     if (K <= 0) return 0;
     if (mode == MODE_GLOBAL || mode == MODE_ROWWISE) return 1;
     if (mode != MODE_GROUPWISE || g <= 0 || K % g != 0) return 0;
@@ -149,6 +193,9 @@ long oracle_groups_per_row(long K, int mode, long g)
 int oracle_quantize(const uint16_t *W, long N, long K, int mode, long g, uint8_t *q,
                     uint16_t *s, uint16_t *z)
 {
+    const int flags = mode & ~MODE_BASE_MASK;
+    mode &= MODE_BASE_MASK;
+    if (flags & ~(FLAG_FLOAT_ZERO | FLAG_META_BF16)) return -1;
     long G = oracle_groups_per_row(K, mode, g);
     if (N <= 0 || G == 0) return -1;
     if (mode == MODE_GLOBAL) {
@@ -164,12 +211,14 @@ int oracle_quantize(const uint16_t *W, long N, long K, int mode, long g, uint8_t
          * then quantize every element with them. */
         float ends[2] = {mn, mx};
         uint8_t dummy[2];
-        quantize_group(ends, 2, dummy, &s[0], &z[0]);
-        float sf = (float)bits_to_f16(s[0]);
-        float zf = (float)bits_to_f16(z[0]);
+        quantize_group(ends, 2, dummy, &s[0], &z[0], flags);
+        float sf = meta_value(s[0], flags);
+        float zf = meta_value(z[0], flags);
+        const int fz = (flags & FLAG_FLOAT_ZERO) != 0;
 #pragma omp parallel for schedule(static)
         for (long i = 0; i < total; ++i) {
-            float t = rintf(bf16_bits_to_f32(W[i]) / sf) + zf;
+            float w = bf16_bits_to_f32(W[i]);
+            float t = fz ? rintf(w / sf + zf) : rintf(w / sf) + zf;
             t = fminf(fmaxf(t, 0.0f), 15.0f);
             q[i] = (uint8_t)(int)t;
         }
@@ -190,7 +239,7 @@ int oracle_quantize(const uint16_t *W, long N, long K, int mode, long g, uint8_t
             for (long gi = 0; gi < G; ++gi) {
                 const uint16_t *src = W + n * K + gi * gl;
                 for (long i = 0; i < gl; ++i) buf[i] = bf16_bits_to_f32(src[i]);
-                quantize_group(buf, gl, q + n * K + gi * gl, &s[n * G + gi], &z[n * G + gi]);
+                quantize_group(buf, gl, q + n * K + gi * gl, &s[n * G + gi], &z[n * G + gi], flags);
             }
         }
         if (heap) __builtin_free(heap);
@@ -226,12 +275,14 @@ void oracle_unpack(const uint32_t *packed, long N, long K, uint8_t *q)
 static void group_params(const uint16_t *s, const uint16_t *z, long n, long k, long K, int mode,
                          long g, double *sd, double *zd)
 {
+    const int flags = mode & ~MODE_BASE_MASK;
     long idx;
+    mode &= MODE_BASE_MASK;
     if (mode == MODE_GLOBAL) idx = 0;
     else if (mode == MODE_ROWWISE) idx = n;
     else idx = n * (K / g) + k / g;
-    *sd = (double)(float)bits_to_f16(s[idx]);
-    *zd = (double)(float)bits_to_f16(z[idx]);
+    *sd = (double)meta_value(s[idx], flags);
+    *zd = (double)meta_value(z[idx], flags);
 }
 
 /* One dequantized row: out[k] = (q[n,k] - z) * s, for k in [0, K). */

@@ -368,3 +368,202 @@ def test_quantization_mae_soft_band():
         wh = oracle.dequant(oracle.pack(q), s, z, m, g, 2048)
         mae = float(np.mean(np.abs(wv - wh)))
         assert 0.75 * page_mae <= mae <= 1.25 * page_mae, (mode, g, mae, page_mae)
+
+
+# ----------------------------------------------------------------------------
+# Variant: fractional zero point and bf16 scales / zeros (the HQQ-style
+# quantizer of "Re-write HQQ Fused Gemm Transpose"; fp16 or bf16 metadata).
+# Reading: s = meta((max - min) / 15); z = meta(-min / s), not rounded to an
+# integer and not clamped to [0, 15]; q = clamp(rint(w / s + z), 0, 15).
+# ----------------------------------------------------------------------------
+def meta_value(bits, meta):
+    b = np.asarray(bits, dtype=np.uint16)
+    if meta == "bf16":
+        return bf16_value(b)
+    return b.view(np.float16).astype(np.float64)
+
+
+ROW_C = [-0.15625, 0.78125, 0.0, 0.03125, 0.1, -0.1, 0.5, 0.25]
+# bf16 inputs: 0.1 -> 0.10009765625 (= 205 * 2^-11), the rest exact.
+# min -0.15625, max 0.78125: range 0.9375 = 15/16 -> s = 1/16 exactly (fp16 0x2C00,
+# bf16 0x3D80); z = 0.15625 * 16 = 2.5 exactly (fp16 0x4100, bf16 0x4020).
+# w/s + z = 0, 15, 2.5, 3, 4.1015625, 0.8984375, 10.5, 6.5 -> rint (ties to even):
+ROW_C_Q = [0, 15, 2, 3, 4, 1, 10, 6]
+# the integer-zero reading differs: z = rint(2.5) = 2, rint(w/s) + 2 = 0, 14, 2, 2, 4, 0, 10, 6
+ROW_C_Q_INT = [0, 14, 2, 2, 4, 0, 10, 6]
+ROW_D = [1.0, 1.5, 2.0, 1.25, 1.75, 1.0, 2.0, 1.5]
+# all positive: s = fp16(1/15) = 0.066650390625 (0x2C44); -min/s = -15.00366...
+# -> fp16 (step 2^-7 in [8, 16)) = -15.0 (0xCB80); w/s - 15 = 0.0037, 7.5055, 15.0073,
+# 3.7546, 11.2564, ... -> q = 0, 8, 15, 4, 11, 0, 15, 8: the whole code range is used,
+# where the clamped integer zero point maps every w to 15.
+ROW_D_Q = [0, 8, 15, 4, 11, 0, 15, 8]
+
+
+@pytest.mark.parametrize("meta,s_bits,z_bits", [("fp16", 0x2C00, 0x4100), ("bf16", 0x3D80, 0x4020)])
+def test_golden_float_zero_example(meta, s_bits, z_bits):
+    q, s, z = oracle.quantize(bf16([ROW_C]), "groupwise", 8, zero="float", meta=meta)
+    assert q.tolist() == [ROW_C_Q]
+    assert s.ravel().tolist() == [s_bits] and z.ravel().tolist() == [z_bits]
+    assert oracle.pack(q).ravel().tolist() == [0x6A1432F0]
+    wh = oracle.dequant(oracle.pack(q), s, z, "groupwise", 8, 8, meta=meta)
+    assert wh.ravel().tolist() == [(c - 2.5) / 16 for c in ROW_C_Q]
+    qi, _, zi = oracle.quantize(bf16([ROW_C]), "groupwise", 8, zero="int", meta=meta)
+    assert qi.tolist() == [ROW_C_Q_INT] and meta_value(zi, meta).ravel().tolist() == [2.0]
+
+
+def test_golden_float_zero_all_positive_group():
+    q, s, z = oracle.quantize(bf16([ROW_D]), "groupwise", 8, zero="float")
+    assert s.ravel().tolist() == [0x2C44] and z.ravel().tolist() == [0xCB80]
+    assert q.tolist() == [ROW_D_Q]
+    wh = oracle.dequant(oracle.pack(q), s, z, "groupwise", 8, 8)
+    assert np.abs(wh - bf16_value(bf16([ROW_D]))).max() <= 0.5 * 0.066650390625 + 1e-12
+    # constant groups reconstruct exactly: s = |w|, z = -sign(w)
+    q, s, z = oracle.quantize(bf16([[0.5] * 8, [-3.0] * 8, [0.0] * 8]), "groupwise", 8, zero="float")
+    wh = oracle.dequant(oracle.pack(q), s, z, "groupwise", 8, 8)
+    assert wh.tolist() == [[0.5] * 8, [-3.0] * 8, [0.0] * 8]
+
+
+@pytest.mark.parametrize("meta", ["fp16", "bf16"])
+@pytest.mark.parametrize("g", [8, 16, 64])
+def test_float_zero_exact_round_trip(meta, g):
+    """w = (q - z) * 2^-e with a fractional z on a quarter grid: exactly representable;
+    quantize must return q, z and 2^-e."""
+    rng = np.random.default_rng(31 + g)
+    N, G = 24, 5
+    K = G * g
+    q = rng.integers(0, 16, size=(N, K))
+    q[:, ::g] = 0
+    q[:, 1::g] = 15
+    z = rng.integers(-60, 121, size=(N, G)) / 4.0          # -15 .. 30 in quarter steps
+    e = rng.integers(-3, 20, size=(N, G))
+    w = (q - np.repeat(z, g, axis=1)) * np.ldexp(1.0, -np.repeat(e, g, axis=1))
+    W = bf16(w)
+    assert (bf16_value(W) == w).all()
+    q2, s2, z2 = oracle.quantize(W, "groupwise", g, zero="float", meta=meta)
+    assert (q2 == q).all()
+    assert (meta_value(z2, meta) == z).all()
+    assert (meta_value(s2, meta) == np.ldexp(1.0, -e)).all()
+    wh = oracle.dequant(oracle.pack(q2), s2, z2, "groupwise", g, K, meta=meta)
+    assert (wh == w).all()
+
+
+@pytest.mark.parametrize("meta", ["fp16", "bf16"])
+def test_float_zero_brute_force_codes(meta):
+    """Each code is the nearest of the 16 levels to u = fp32(fp32(w / s) + z), found by
+    exhaustive search (ties to the even level), and z is within one rounding of -min/s."""
+    g = 16
+    W = synth.normal_bf16((40, 4 * g), 0.0, 0.02, seed=9, stream=2)
+    W[3, :g] = bf16(np.abs(synth.bf16_bits_to_f32(W[3, :g])) + 0.05)     # all positive
+    W[4, g:2 * g] = bf16(-np.abs(synth.bf16_bits_to_f32(W[4, g:2 * g])) - 0.05)
+    q, s, z = oracle.quantize(W, "groupwise", g, zero="float", meta=meta)
+    wv = synth.bf16_bits_to_f32(W)
+    zrel = 2.0 ** -8 if meta == "bf16" else 2.0 ** -11          # half a step of the type
+    for n in range(W.shape[0]):
+        for gi in range(4):
+            sl = slice(gi * g, (gi + 1) * g)
+            sv = np.float32(meta_value(s[n, gi], meta))
+            zv = np.float32(meta_value(z[n, gi], meta))
+            exact = -Fraction(float(wv[n, sl].min())) / Fraction(float(sv))
+            assert abs(Fraction(float(zv)) - exact) <= abs(exact) * Fraction(zrel) * Fraction(1001, 1000)
+            for w, code in zip(wv[n, sl], q[n, sl]):
+                u = np.float32(np.float32(w) / sv) + zv
+                d = [abs(Fraction(float(u)) - lv) for lv in range(16)]
+                best = min(range(16), key=lambda lv: (d[lv], lv % 2))
+                assert code == best
+
+
+@pytest.mark.parametrize("meta", ["fp16", "bf16"])
+@pytest.mark.parametrize("mode,g", [("groupwise", 32), ("groupwise", 128), ("rowwise", 0), ("global", 0)])
+def test_float_zero_error_bound(meta, mode, g):
+    """|w - w_hat| <= (1/2 + |z - (-min/s)|) s: half a step plus the zero point's rounding,
+    for every group, with or without zero inside it."""
+    K = 512
+    W = synth.normal_bf16((64, K), 0.0, 0.02, seed=22, stream=2)
+    W[:8] = bf16(np.abs(synth.bf16_bits_to_f32(W[:8])) + 0.01)          # groups away from zero
+    q, s, z = oracle.quantize(W, mode, g, zero="float", meta=meta)
+    wh = oracle.dequant(oracle.pack(q), s, z, mode, g, K, meta=meta)
+    w = bf16_value(W)
+    gl = {"groupwise": g, "rowwise": K, "global": K}[mode]
+    sv, zv = meta_value(s, meta), meta_value(z, meta)
+    if mode == "global":
+        sk, zk = np.full(W.shape, sv[0, 0]), np.full(W.shape, zv[0, 0])
+        mn = np.full(W.shape, w.min())
+    else:
+        sk, zk = np.repeat(sv, gl, axis=1), np.repeat(zv, gl, axis=1)
+        mn = np.repeat(w.reshape(64, -1, gl).min(axis=2), gl, axis=1)
+    zerr = np.abs(zk + mn / sk)
+    err = np.abs(w - wh)
+    assert (err <= (0.5 + zerr + 2.0 ** -12) * sk).all()
+    # the zero point follows the group: codes 0 and 15 are both used in most groups
+    if mode == "groupwise":
+        used = (q.reshape(64, -1, g).min(axis=2) == 0) & (q.reshape(64, -1, g).max(axis=2) == 15)
+        assert used.mean() > 0.9
+
+
+def test_float_zero_reduces_to_integer_zero_when_min_is_on_the_grid():
+    """If -min/s is an integer in [0, 15] and no w/s sits on a half step, both readings
+    give the same codes, scale and zero value."""
+    rng = np.random.default_rng(17)
+    g, G, N = 16, 4, 12
+    zi = rng.integers(0, 16, size=(N, G))
+    e = rng.integers(2, 12, size=(N, G))
+    lev = rng.integers(0, 16, size=(N, G * g)).astype(np.float64)
+    frac = rng.uniform(-0.4, 0.4, size=lev.shape)
+    frac[:, ::g] = 0.0
+    lev[:, ::g] = 0.0                      # the minimum sits on level 0 ...
+    frac[:, 1::g] = 0.0
+    lev[:, 1::g] = 15.0                    # ... and the maximum on level 15
+    t = np.clip(lev + frac, 0.0, 15.0) - np.repeat(zi, g, axis=1)
+    w = bf16_value(bf16(t * np.ldexp(1.0, -np.repeat(e, g, axis=1))))
+    W = bf16(w)
+    for meta in ("fp16", "bf16"):
+        qf, sf, zf = oracle.quantize(W, "groupwise", g, zero="float", meta=meta)
+        qi, si, zi2 = oracle.quantize(W, "groupwise", g, zero="int", meta=meta)
+        assert (qf == qi).all() and (sf == si).all()
+        assert (meta_value(zf, meta) == meta_value(zi2, meta)).all()
+        assert (meta_value(zf, meta) == zi).all()
+
+
+def test_bf16_metadata_matches_fp16_where_both_are_exact():
+    """With power-of-two scales and integer zeros the bf16-metadata quantizer returns the
+    same codes and values as the fp16 one (only the bit patterns differ)."""
+    rng = np.random.default_rng(23)
+    g, G, N = 32, 3, 10
+    q = rng.integers(0, 16, size=(N, G * g))
+    q[:, ::g] = 0
+    q[:, 1::g] = 15
+    z = rng.integers(0, 16, size=(N, G))
+    e = rng.integers(-2, 14, size=(N, G))
+    w = (q - np.repeat(z, g, axis=1)) * np.ldexp(1.0, -np.repeat(e, g, axis=1))
+    W = bf16(w)
+    q16, s16, z16 = oracle.quantize(W, "groupwise", g)
+    qb, sb, zb = oracle.quantize(W, "groupwise", g, meta="bf16")
+    assert (q16 == qb).all()
+    assert (meta_value(s16, "fp16") == meta_value(sb, "bf16")).all()
+    assert (meta_value(z16, "fp16") == meta_value(zb, "bf16")).all()
+    # bf16 rounds the scale to 8 significant bits: a non-power-of-two range shows it
+    qb, sb, _ = oracle.quantize(bf16([ROW_A]), "groupwise", 8, meta="bf16")
+    assert sb.ravel().tolist() == [0x3E4D]          # 0.2 -> 205 * 2^-10 = 0.2001953125
+
+
+@pytest.mark.parametrize("zero,meta", [("float", "fp16"), ("float", "bf16"), ("int", "bf16")])
+def test_variant_matmul_one_hot_and_adjoint(zero, meta):
+    """linear / linear_t read the variant's metadata: one-hot rows return the dequantized
+    weights, and <X W^T, dY> = <X, dY W>."""
+    seed = 0
+    X = synth.activations(4, 512, seed)
+    W = synth.weights(256, 512, seed)
+    dY = synth.grads(4, 256, seed)
+    p, s, z = oracle.quantize_pack(W, "groupwise", 64, zero=zero, meta=meta)
+    wh = oracle.dequant(p, s, z, "groupwise", 64, 512, meta=meta)
+    ks = [0, 63, 64, 511]
+    E = np.zeros((len(ks), 512))
+    E[np.arange(len(ks)), ks] = 1.0
+    y64, _ = oracle.linear(bf16(E), p, s, z, "groupwise", 64, 256, 512, meta=meta)
+    assert (y64 == wh[:, ks].T).all()
+    y64, _ = oracle.linear(X, p, s, z, "groupwise", 64, 256, 512, meta=meta)
+    x64, _ = oracle.linear_t(dY, p, s, z, "groupwise", 64, 256, 512, meta=meta)
+    lhs = float(np.sum(y64 * bf16_value(dY)))
+    rhs = float(np.sum(bf16_value(X) * x64))
+    assert abs(lhs - rhs) <= 1e-9 * (abs(lhs) + 1.0)
+    assert np.allclose(y64, bf16_value(X) @ wh.T, rtol=1e-12, atol=1e-12)
