@@ -379,8 +379,9 @@ def measure_configs(torch, w4, dev, peaks, stream):
     """Every configuration of the workload list, one timed call each (L2
     flushed before it): the tiny correctness case, the Llama-3.2-1B layers in
     three quantization modes with quantize-and-pack of each weight, the
-    Llama-2-7B QLoRA layers forward and transposed, and the Llama-3-8B
-    serving layers with bias at M = 1 .. 1024.  Each row reports the
+    Llama-2-7B QLoRA layers forward and transposed, the Llama-3-8B serving
+    layers with bias at M = 1 .. 1024, and the fractional-zero variant (fp16
+    and bf16 metadata) on decode and training shapes.  Each row reports the
     fraction of its own roofline (the slower of tensor-core and HBM time)."""
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     gen = torch.Generator(device=dev)
@@ -472,6 +473,30 @@ def measure_configs(torch, w4, dev, peaks, stream):
                                 lambda: w4.w4a16_gemm(X, P, S, Z, "groupwise", 128, N=N, K=K, bias=b), bias=True))
             del W, P, S, Z
         out["config5_llama3_8b_bias"] = rows
+        # the HQQ-style variant: fractional zero point, fp16 and bf16 scales / zeros,
+        # quantize + pack and the decode / training products on the same shapes
+        rows = []
+        for (N, K, g) in ((16384, 16384, 128), (8192, 8192, 128), (11008, 4096, 64)):
+            W = rnd((N, K), 0.02)
+            for meta in ("fp16", "bf16"):
+                t = timed(lambda: w4.w4_quantize_pack(W, "groupwise", g, zero="float", meta=meta))
+                qb = 2 * N * K + N * K // 2 + 4 * N * (K // g)
+                rows.append({"case": f"quantize float-zero {meta}", "N": N, "K": K, "g": g, "us": round(t * 1e6, 2),
+                             "GB/s": round(qb / t / 1e9, 1), "frac": round(qb / t / 1e9 / peaks["hbm_gbs"], 4)})
+                P, S, Z = w4.w4_quantize_pack(W, "groupwise", g, zero="float", meta=meta)
+                Ms = (1, 4) if N == K else (2048,)
+                for M in Ms:
+                    X, dY = rnd((M, K)), rnd((M, N))
+                    r = row(f"float-zero {meta} fwd", M, N, K, "groupwise", g,
+                            lambda: w4.w4a16_gemm(X, P, S, Z, "groupwise", g, N=N, K=K, zero="float"))
+                    rows.append(r)
+                    r = row(f"float-zero {meta} t", M, N, K, "groupwise", g,
+                            lambda: w4.w4a16_gemm(dY, P, S, Z, "groupwise", g, N=N, K=K, transposed=True,
+                                                  zero="float"), transposed=True)
+                    rows.append(r)
+                del P, S, Z
+            del W
+        out["variant_float_zero"] = rows
         del flush
     torch.cuda.synchronize()
     return out

@@ -9,7 +9,8 @@ or without the built library every call raises.
 Entry points (same names as the C ABI in ``include/w4a16.h``):
 
 * :func:`w4_quantize_pack` -- bf16 W [N, K] -> packed int4 (int32 [N, K/8]),
-  fp16 scales and zeros
+  fp16 scales and zeros (``zero="float"``: fractional zero point;
+  ``meta="bf16"``: bf16 scales and zeros)
 * :func:`w4a16_gemm` -- Y = X . dequant(W)^T (or dX = dY . dequant(W) with
   ``transposed=True``), optional bias
 * :func:`w4a16_gemv` -- the same for M <= 4 (TMA-streamed weights, exact
@@ -28,6 +29,8 @@ W4_MODE_GLOBAL = 0
 W4_MODE_ROWWISE = 1
 W4_MODE_GROUPWISE = 2
 MODES = {"global": W4_MODE_GLOBAL, "rowwise": W4_MODE_ROWWISE, "groupwise": W4_MODE_GROUPWISE}
+W4_ZERO_FLOAT = 0x10
+W4_META_BF16 = 0x20
 
 _lock = threading.Lock()
 _lib = None
@@ -87,8 +90,17 @@ def _torch():
     return torch
 
 
-def _mode(mode) -> int:
-    return MODES[mode] if isinstance(mode, str) else int(mode)
+def _mode(mode, zero: str = "int", meta: str = "fp16") -> int:
+    """The C mode argument: base mode or-ed with the format flags."""
+    m = MODES[mode] if isinstance(mode, str) else int(mode)
+    if zero not in ("int", "float") or meta not in ("fp16", "bf16"):
+        raise ValueError(f"zero must be 'int' or 'float' and meta 'fp16' or 'bf16', got {zero!r}, {meta!r}")
+    return m | (W4_ZERO_FLOAT if zero == "float" else 0) | (W4_META_BF16 if meta == "bf16" else 0)
+
+
+def _meta_dtype(meta: str):
+    torch = _torch()
+    return torch.bfloat16 if meta == "bf16" else torch.float16
 
 
 def _check_cuda(t, name, dtype, shape=None):
@@ -111,7 +123,7 @@ def _stream_ptr(device):
 
 
 def meta_shape(N: int, K: int, mode, group_size: int):
-    m = _mode(mode)
+    m = _mode(mode) & 0x0F
     if m == W4_MODE_GLOBAL:
         return (1, 1)
     if m == W4_MODE_ROWWISE:
@@ -129,23 +141,31 @@ def w4_workspace_bytes(M: int, N: int, K: int, transposed: bool = False) -> int:
     return int(library().w4_workspace_bytes(M, N, K, int(bool(transposed))))
 
 
-def w4_quantize_pack(W, mode="groupwise", group_size: int = 128, out=None):
-    """Quantize bf16 W [N, K] (CUDA) -> (packed int32 [N, K/8], scales fp16, zeros fp16)."""
+def w4_quantize_pack(W, mode="groupwise", group_size: int = 128, out=None, zero: str = "int",
+                     meta: str = "fp16"):
+    """Quantize bf16 W [N, K] (CUDA) -> (packed int32 [N, K/8], scales, zeros).
+
+    ``zero="float"`` keeps a fractional zero point (the HQQ-style quantizer);
+    ``meta="bf16"`` stores scales and zeros as bf16 instead of fp16.
+    """
     torch = _torch()
     _check_cuda(W, "W", torch.bfloat16)
     N, K = W.shape
     shape = meta_shape(N, K, mode, group_size)
     dev = W.device
+    mdt = _meta_dtype(meta)
     if out is None:
         packed = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
-        scales = torch.empty(shape, dtype=torch.float16, device=dev)
-        zeros = torch.empty(shape, dtype=torch.float16, device=dev)
+        scales = torch.empty(shape, dtype=mdt, device=dev)
+        zeros = torch.empty(shape, dtype=mdt, device=dev)
     else:
         packed, scales, zeros = out
+        _check_cuda(scales, "scales", mdt, shape)
+        _check_cuda(zeros, "zeros", mdt, shape)
     nws = w4_quantize_workspace_bytes(N, K, mode)
     ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
     with torch.cuda.device(dev):
-        st = library().w4_quantize_pack(W.data_ptr(), N, K, _mode(mode), int(group_size),
+        st = library().w4_quantize_pack(W.data_ptr(), N, K, _mode(mode, zero, meta), int(group_size),
                                         packed.data_ptr(), scales.data_ptr(), zeros.data_ptr(),
                                         ws.data_ptr(), nws, _stream_ptr(dev))
     if st != 0:
@@ -153,12 +173,14 @@ def w4_quantize_pack(W, mode="groupwise", group_size: int = 128, out=None):
     return packed, scales, zeros
 
 
-def _matmul(fname, A, packed, scales, zeros, mode, group_size, N, K, bias, transposed, out):
+def _matmul(fname, A, packed, scales, zeros, mode, group_size, N, K, bias, transposed, out, zero):
     torch = _torch()
     _check_cuda(A, "A", torch.bfloat16)
     _check_cuda(packed, "packed", torch.int32, (N, K // 8))
-    _check_cuda(scales, "scales", torch.float16, meta_shape(N, K, mode, group_size))
-    _check_cuda(zeros, "zeros", torch.float16, meta_shape(N, K, mode, group_size))
+    # the metadata type follows the scales' dtype (fp16 or bf16)
+    meta = "bf16" if isinstance(scales, torch.Tensor) and scales.dtype == torch.bfloat16 else "fp16"
+    _check_cuda(scales, "scales", _meta_dtype(meta), meta_shape(N, K, mode, group_size))
+    _check_cuda(zeros, "zeros", _meta_dtype(meta), meta_shape(N, K, mode, group_size))
     if A.dim() != 2:
         raise ValueError("A must be 2-D")
     M = A.shape[0]
@@ -177,7 +199,7 @@ def _matmul(fname, A, packed, scales, zeros, mode, group_size, N, K, bias, trans
     with torch.cuda.device(dev):
         st = getattr(library(), fname)(
             A.data_ptr(), M, N, K, packed.data_ptr(), scales.data_ptr(), zeros.data_ptr(),
-            _mode(mode), int(group_size), None if bias is None else bias.data_ptr(),
+            _mode(mode, zero, meta), int(group_size), None if bias is None else bias.data_ptr(),
             int(bool(transposed)), out.data_ptr(), None if ws is None else ws.data_ptr(), nws,
             _stream_ptr(dev))
     if st != 0:
@@ -186,18 +208,21 @@ def _matmul(fname, A, packed, scales, zeros, mode, group_size, N, K, bias, trans
 
 
 def w4a16_gemm(A, packed, scales, zeros, mode="groupwise", group_size: int = 128, *, N: int,
-               K: int, bias=None, transposed: bool = False, out=None):
-    """Y = A . dequant(W)^T  (A [M, K])  or, transposed, dX = A . dequant(W)  (A [M, N])."""
+               K: int, bias=None, transposed: bool = False, out=None, zero: str = "int"):
+    """Y = A . dequant(W)^T  (A [M, K])  or, transposed, dX = A . dequant(W)  (A [M, N]).
+
+    ``zero`` must name the quantizer's zero point ("int" or "float"); bf16 scales
+    and zeros are recognised by their dtype."""
     return _matmul("w4a16_gemm", A, packed, scales, zeros, mode, group_size, N, K, bias,
-                   transposed, out)
+                   transposed, out, zero)
 
 
 def w4a16_gemv(A, packed, scales, zeros, mode="groupwise", group_size: int = 128, *, N: int,
-               K: int, bias=None, transposed: bool = False, out=None):
+               K: int, bias=None, transposed: bool = False, out=None, zero: str = "int"):
     """Small-batch (M <= 4) path of :func:`w4a16_gemm`: TMA-streamed weights, exact
     products on the tensor pipe with fp32 sums, forward and transposed."""
     return _matmul("w4a16_gemv", A, packed, scales, zeros, mode, group_size, N, K, bias,
-                   transposed, out)
+                   transposed, out, zero)
 
 
 def w4_launch_count() -> int:

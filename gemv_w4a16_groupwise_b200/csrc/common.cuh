@@ -47,6 +47,19 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
     return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
 
+// Format flags of the scale / zero metadata, or-ed into the mode (the same
+// values as W4_ZERO_FLOAT and W4_META_BF16 of the public header).
+constexpr int kFmtZeroFloat = 0x10;   // fractional zero point
+constexpr int kFmtMetaBf16 = 0x20;    // scales and zeros stored as bf16
+
+// Value of a scale or zero stored as fp16 bits, or bf16 bits.
+__device__ __forceinline__ float meta_to_float(uint16_t b, bool bf16) {
+    return bf16 ? bf16_bits_to_float(b) : __half2float(__ushort_as_half(b));
+}
+__device__ __forceinline__ float meta_to_float(__half h, bool bf16) {
+    return meta_to_float(__half_as_ushort(h), bf16);
+}
+
 __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
     // (a & mask) | orv in one instruction
     uint32_t r;
@@ -74,5 +87,7 @@ __device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) {
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
     return __ffma2_rn(a, b, c);
 }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 
 }  // namespace w4

@@ -3,7 +3,8 @@
 // transposed mode, dY rows not 16-byte strided (N % 8 != 0).  A CTA computes
 // a 64 x 64 tile of the output from 32-long slices of the reduction staged in
 // shared memory: the activations as fp32 and the weights dequantized to
-// (q - z) s in fp32 (exact: a 5-bit integer times an 11-bit significand);
+// (q - z) s in fp32 (exact for an integer z: a 5-bit integer times an 11-bit
+// significand; a fractional z rounds it once);
 // each thread keeps 4 x 4 outputs and adds x w_hat with fp32 fma (every
 // product exact), in ascending reduction order, then adds the bias and
 // rounds once to bf16.
@@ -23,6 +24,7 @@ struct GemmSimpleArgs {
     const uint16_t* bias;     // [output columns] bf16 or nullptr
     uint16_t* Y;              // [M, output columns] bf16
     int M, N, K, g, G, sz_row;
+    int fmt;                  // format flags: kFmtZeroFloat, kFmtMetaBf16
 };
 
 constexpr int kGsTile = 64;   // output tile (rows of A x output columns)
@@ -53,8 +55,9 @@ __global__ void __launch_bounds__(256) gemm_simple_kernel(const GemmSimpleArgs a
             if (n < a.N && k < a.K) {
                 const uint32_t word = __ldg(a.packed + static_cast<size_t>(n) * W8 + k / 8);
                 const int grp = a.G == 1 ? 0 : k / a.g;
-                const float s = __half2float(a.S[static_cast<size_t>(n) * a.sz_row + grp]);
-                const float z = __half2float(a.Z[static_cast<size_t>(n) * a.sz_row + grp]);
+                const bool mbf = (a.fmt & kFmtMetaBf16) != 0;
+                const float s = meta_to_float(a.S[static_cast<size_t>(n) * a.sz_row + grp], mbf);
+                const float z = meta_to_float(a.Z[static_cast<size_t>(n) * a.sz_row + grp], mbf);
                 w = (static_cast<float>((word >> (4 * (k & 7))) & 0xFu) - z) * s;
             }
             ws[rr][i] = w;

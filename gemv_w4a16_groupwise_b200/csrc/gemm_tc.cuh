@@ -36,7 +36,9 @@
 // 2048) with one lop3, and one packed FMA per pair gives
 //     (off + q) * s - (off + z) * s = (q - z) * s
 // exactly in fp32 (both products need at most 23 significand bits), which
-// cvt.rn.bf16x2 rounds once.
+// cvt.rn.bf16x2 rounds once.  A fractional zero point (more significand
+// bits) takes (off + q) - (off + z) and then the product with s instead,
+// the product rounded in fp32 before the bf16 rounding.
 #pragma once
 
 #include "tma.cuh"
@@ -54,6 +56,7 @@ constexpr int kTcPBytes = kTcBM * kTcBK / 2;   // 4 KB packed tile
 struct TcArgs {
     const __half* S;
     const __half* Z;
+    int fmt;              // format flags: kFmtZeroFloat, kFmtMetaBf16
     const uint16_t* bias;
     uint16_t* Y;
     float* part;          // [(tiles - F) * nslice][BN][128] fp32 partial tiles of the split tail
@@ -71,6 +74,7 @@ struct TcProblem {
     const void* S;
     const void* Z;
     int g, G, sz_row;
+    int fmt;
     const void* bias;
     int transposed;
     void* Y;
@@ -134,7 +138,7 @@ __device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t (&r)[8]) {
 }
 
 // Eight codes of one packed word -> eight bf16 (q - z) * s in k order.
-__device__ __forceinline__ uint4 dequant_word_bf16(uint32_t w, float s, float c_lo, float c_hi) {
+__device__ __forceinline__ uint4 dequant_word_bf16(uint32_t w, float s, float c_lo, float c_hi, bool fz) {
     const uint32_t l16 = w << 16, l8 = w << 8, r8 = w >> 8, r16 = w >> 16;
     const float2 ss = make_float2(s, s);
     const float2 cc = make_float2(c_lo, c_hi);
@@ -147,10 +151,19 @@ __device__ __forceinline__ uint4 dequant_word_bf16(uint32_t w, float s, float c_
                                    __uint_as_float(lop3_and_or(r8, 0xF000u, 0x45000000u)));
     const float2 v67 = make_float2(__uint_as_float(lop3_and_or(r8, 0xF0000u, 0x43000000u)),
                                    __uint_as_float(lop3_and_or(r16, 0xF000u, 0x45000000u)));
-    const float2 f01 = ffma2(v01, ss, cc);
-    const float2 f23 = ffma2(v23, ss, cc);
-    const float2 f45 = ffma2(v45, ss, cc);
-    const float2 f67 = ffma2(v67, ss, cc);
+    float2 f01, f23, f45, f67;
+    if (!fz) {
+        f01 = ffma2(v01, ss, cc);
+        f23 = ffma2(v23, ss, cc);
+        f45 = ffma2(v45, ss, cc);
+        f67 = ffma2(v67, ss, cc);
+    } else {
+        // cc = -(off + z) here
+        f01 = fmul2(fadd2(v01, cc), ss);
+        f23 = fmul2(fadd2(v23, cc), ss);
+        f45 = fmul2(fadd2(v45, cc), ss);
+        f67 = fmul2(fadd2(v67, cc), ss);
+    }
     uint4 out;
     out.x = bf162_bits(__floats2bfloat162_rn(f01.x, f01.y));
     out.y = bf162_bits(__floats2bfloat162_rn(f23.x, f23.y));
@@ -332,6 +345,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int gshift = -1;                                  // log2(g) when g is a power of two
         if ((a.g & (a.g - 1)) == 0) gshift = __ffs(a.g) - 1;
         auto group_of = [&](int k) { return min(gshift >= 0 ? (k >> gshift) : k / a.g, a.G - 1); };
+        const bool mbf = (a.fmt & kFmtMetaBf16) != 0;
+        const bool fz = (a.fmt & kFmtZeroFloat) != 0;
         // Scale / zero of one stage (tile i, block kb); with g a multiple of
         // 32 the thread's 4 words share one group.
         constexpr int NG = PWG ? 4 : 1;
@@ -345,8 +360,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int j = 0; j < NG; ++j) {
                 const int grp = group_of(8 * (kw0 + j));
-                sv[j] = __half2float(__ldg(sp + grp));
-                zv[j] = __half2float(__ldg(zp + grp));
+                sv[j] = meta_to_float(__ldg(reinterpret_cast<const unsigned short*>(sp + grp)), mbf);
+                zv[j] = meta_to_float(__ldg(reinterpret_cast<const unsigned short*>(zp + grp)), mbf);
             }
         };
         // (ci, ckb): unit and k-block of this group's current stage; cb1 is
@@ -398,7 +413,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const float sj = sv[PWG ? j : 0], zj = zv[PWG ? j : 0];
                     uint4 out = make_uint4(0u, 0u, 0u, 0u);
                     if (row_ok && (kw0 + j) < W8)
-                        out = dequant_word_bf16(w, sj, -(128.0f + zj) * sj, -(2048.0f + zj) * sj);
+                        out = fz ? dequant_word_bf16(w, sj, -(128.0f + zj), -(2048.0f + zj), true)
+                                 : dequant_word_bf16(w, sj, -(128.0f + zj) * sj, -(2048.0f + zj) * sj, false);
                     *reinterpret_cast<uint4*>(st + off[j]) = out;
                 }
                 fence_proxy_async_smem();

@@ -26,10 +26,12 @@ struct GemvFwdArgs {
     const uint16_t* bias;    // [N] bf16 or nullptr
     uint16_t* Y;             // [M, N] bf16
     int N, K, g, G, sz_row;  // group of (n, k): n * sz_row + min(k / g, G - 1)
+    int fmt;                 // format flags: kFmtZeroFloat, kFmtMetaBf16
 };
 
-__device__ __forceinline__ float half_to_float_ldg(const __half* p) {
-    return __half2float(__ldg(p));
+// A scale or zero (fp16 or bf16 bits) through the read-only cache.
+__device__ __forceinline__ float meta_ldg(const __half* p, bool bf16) {
+    return meta_to_float(__ldg(reinterpret_cast<const unsigned short*>(p)), bf16);
 }
 
 
@@ -145,8 +147,9 @@ __global__ void __launch_bounds__(256) gemv_fwd_simple_kernel(const GemvFwdArgs 
     for (int j = lane; j < W8; j += 32) {
         const uint32_t w = __ldg(packed + static_cast<size_t>(n) * W8 + j);
         const int grp = min((8 * j) / a.g, a.G - 1);
-        const float s = half_to_float_ldg(a.S + n * a.sz_row + grp);
-        const float z = half_to_float_ldg(a.Z + n * a.sz_row + grp);
+        const bool mbf = (a.fmt & kFmtMetaBf16) != 0;
+        const float s = meta_ldg(a.S + n * a.sz_row + grp, mbf);
+        const float z = meta_ldg(a.Z + n * a.sz_row + grp, mbf);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const float wv = (static_cast<float>((w >> (4 * e)) & 0xF) - z) * s;
@@ -179,8 +182,9 @@ __global__ void __launch_bounds__(256) gemv_fwd_simple_kernel(const GemvFwdArgs 
 // the CTA's row range and meet in shared memory.  Per code the lane forms
 // (q - z) exactly ((2^23 + q) - (2^23 + z) in fp32) and multiplies it by
 // c = dY[m, n] s (exact: 8 x 11 significant bits) in an fp32 fma, so every
-// product is exact and the sums are fp32.  Row ranges are split over CTAs;
-// fp32 partials go to the workspace.
+// product is exact and the sums are fp32.  A fractional zero point takes
+// (128 + q) - (128 + z) instead, q - z rounded at most once.  Row ranges are
+// split over CTAs; fp32 partials go to the workspace.
 // ---------------------------------------------------------------------------
 struct GemvTArgs {
     const uint16_t* dY;      // [M, N] bf16
@@ -192,6 +196,7 @@ struct GemvTArgs {
     float* partial;          // [splits, M, K] when splits > 1
     int N, K, g, G, sz_row;
     int rows_per_split, splits;
+    int fmt;                 // format flags: kFmtZeroFloat, kFmtMetaBf16
 };
 
 constexpr int kGemvTThreads = 128;
@@ -220,16 +225,22 @@ __global__ void __launch_bounds__(kGemvTThreads)
     for (int n = r0 + warp; n < r1; n += kGemvTThreads / 32) {
         const uint32_t* rowp = a.packed + static_cast<size_t>(n) * W8;
         const uint32_t w[2] = {has0 ? ldg_stream_u32(rowp + j0) : 0u, has1 ? ldg_stream_u32(rowp + j0 + 1) : 0u};
-        const float s[2] = {half_to_float_ldg(a.S + n * a.sz_row + grp0), half_to_float_ldg(a.S + n * a.sz_row + grp1)};
-        // 2^23 + z, so that (2^23 + q) - (2^23 + z) = q - z exactly
-        const float zo[2] = {8388608.0f + half_to_float_ldg(a.Z + n * a.sz_row + grp0),
-                             8388608.0f + half_to_float_ldg(a.Z + n * a.sz_row + grp1)};
+        const bool mbf = (a.fmt & kFmtMetaBf16) != 0;
+        const float s[2] = {meta_ldg(a.S + n * a.sz_row + grp0, mbf), meta_ldg(a.S + n * a.sz_row + grp1, mbf)};
+        // off + z, so that (off + q) - (off + z) = q - z: off = 2^23 for an
+        // integer z (exact), 128 for a fractional one (exact unless z has
+        // bits below 2^-16)
+        const float off = (a.fmt & kFmtZeroFloat) ? 128.0f : 8388608.0f;
+        const uint32_t ob = (a.fmt & kFmtZeroFloat) ? 0x43000000u : 0x4B000000u;
+        const int qsh = (a.fmt & kFmtZeroFloat) ? 16 : 0;     // code position in (off + q)
+        const float zo[2] = {off + meta_ldg(a.Z + n * a.sz_row + grp0, mbf),
+                             off + meta_ldg(a.Z + n * a.sz_row + grp1, mbf)};
         float qz[16];
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                qz[8 * h + e] = __uint_as_float(0x4B000000u | ((w[h] >> (4 * e)) & 0xFu)) - zo[h];
+                qz[8 * h + e] = __uint_as_float(ob | (((w[h] >> (4 * e)) & 0xFu) << qsh)) - zo[h];
 #pragma unroll
         for (int m = 0; m < M; ++m) {
             const float d = bf16_bits_to_float(__ldg(a.dY + static_cast<size_t>(m) * a.N + n));

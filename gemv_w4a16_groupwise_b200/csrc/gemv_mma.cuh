@@ -145,6 +145,18 @@ __device__ __forceinline__ void unpack_word_bf16(uint32_t w, uint32_t zz, uint32
     p[3] = bf16x2_sub(lop3_and_or(w >> 12, 0x000F000Fu, 0x43004300u), zz);
 }
 
+// The same registers for a fractional zero point, where q - z is not a
+// bf16 value: (128 + q) - (128 + z) in fp32 (zo = 128 + z), rounded once to
+// bf16.
+__device__ __forceinline__ void unpack_word_bf16_rounded(uint32_t w, float zo, uint32_t (&p)[4]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float lo = __uint_as_float(lop3_and_or(w << (16 - 4 * i), 0x000F0000u, 0x43000000u));
+        const float hi = __uint_as_float(lop3_and_or(w >> (4 * i), 0x000F0000u, 0x43000000u));
+        p[i] = bf162_bits(__floats2bfloat162_rn(lo - zo, hi - zo));
+    }
+}
+
 // How the scales and zeros reach a stage:
 //   kSzConst  one scale and zero for the whole matrix (global mode): read
 //             once per thread, no per-stage data;
@@ -202,12 +214,13 @@ struct GemvMmaArgs {
     int stages;               // ring depth
     int szw;                  // 2-D box: groups per row; copy path: words per row and stage
     long long sz_total;       // halves in each of S and Z (N * sz_row, or 1)
+    int fmt;                  // format flags: kFmtZeroFloat, kFmtMetaBf16
 };
 
 // Work split: each CTA of a slice takes a contiguous range of whole row
 // blocks (balanced to within one row block) and walks them row block by row
 // block, stage by stage along its K slice.
-template <int M, int CLS, int SZ>
+template <int M, int CLS, int SZ, bool FZ>
 __global__ void __launch_bounds__(kMThreads, 1)
     gemv_mma_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                     const __grid_constant__ CUtensorMap zmap, const GemvMmaArgs a) {
@@ -353,11 +366,14 @@ __global__ void __launch_bounds__(kMThreads, 1)
         if (items > 0) convert_x_block<M, CLS>(a.X, a.K, k_slice, a.nks, warp, lane, xw);
         __syncwarp();
 
-        float s_const = 0.f;
+        const bool mbf = (a.fmt & kFmtMetaBf16) != 0;
+        constexpr bool fz = FZ;     // a.fmt & kFmtZeroFloat, as a template argument
+        float s_const = 0.f, zo_const = 0.f;
         uint32_t zz_const = 0u;
         if (SZ == kSzConst) {
-            s_const = __half2float(a.S[0]);
-            zz_const = bf16x2_splat(128.0f + __half2float(a.Z[0]));
+            s_const = meta_to_float(a.S[0], mbf);
+            zo_const = 128.0f + meta_to_float(a.Z[0], mbf);
+            zz_const = bf16x2_splat(zo_const);
         }
         float y0a = 0.f, y0b = 0.f, y1a = 0.f, y1b = 0.f;   // rows gid / gid + 8, m = 2 tig / 2 tig + 1
         int rb = rb_lo, ks = 0, rbi = 0;
@@ -404,7 +420,7 @@ __global__ void __launch_bounds__(kMThreads, 1)
                     for (int i = 0; i < 4; ++i) bq[i] = xq[i * kLB];
                 }
                 // ---- scales and zeros of rows gid and gid + 8, per k block
-                float sv[NB][2];
+                float sv[NB][2], zo[NB][2];
                 uint32_t zz[NB][2];
 #pragma unroll
                 for (int b = 0; b < NB; ++b) {
@@ -412,24 +428,25 @@ __global__ void __launch_bounds__(kMThreads, 1)
                     if (SZ == kSzConst) {
                         sv[b][0] = sv[b][1] = s_const;
                         zz[b][0] = zz[b][1] = zz_const;
+                        zo[b][0] = zo[b][1] = zo_const;
                         continue;
                     }
                     const __half* sh = reinterpret_cast<const __half*>(sb + kMWBytes);
                     if (SZ == kSzTma1d) {
-                        sv[b][0] = __half2float(sh[gid]);
-                        sv[b][1] = __half2float(sh[gid + 8]);
-                        zv0 = __half2float(sh[64 + gid]);
-                        zv1 = __half2float(sh[64 + gid + 8]);
+                        sv[b][0] = meta_to_float(sh[gid], mbf);
+                        sv[b][1] = meta_to_float(sh[gid + 8], mbf);
+                        zv0 = meta_to_float(sh[64 + gid], mbf);
+                        zv1 = meta_to_float(sh[64 + gid + 8], mbf);
                     } else {
                         const int grp = group_of(kg + b * (128 / NB));
                         const int fg = group_of(k0);
                         if (SZ == kSzTma2d) {
                             const int gi = grp - (fg & ~7);
                             const int w2 = a.szw;
-                            sv[b][0] = __half2float(sh[gid * w2 + gi]);
-                            sv[b][1] = __half2float(sh[(gid + 8) * w2 + gi]);
-                            zv0 = __half2float(sh[kMR * w2 + gid * w2 + gi]);
-                            zv1 = __half2float(sh[kMR * w2 + (gid + 8) * w2 + gi]);
+                            sv[b][0] = meta_to_float(sh[gid * w2 + gi], mbf);
+                            sv[b][1] = meta_to_float(sh[(gid + 8) * w2 + gi], mbf);
+                            zv0 = meta_to_float(sh[kMR * w2 + gid * w2 + gi], mbf);
+                            zv1 = meta_to_float(sh[kMR * w2 + (gid + 8) * w2 + gi], mbf);
                         } else {
                             // row r's words start at half (row r, first group)
                             // rounded down to even
@@ -437,14 +454,16 @@ __global__ void __launch_bounds__(kMThreads, 1)
                             const int o0 = grp - fg + ((((row0 + gid) & a.sz_row) ^ fg) & 1);
                             const int o1 = grp - fg + ((((row0 + gid + 8) & a.sz_row) ^ fg) & 1);
                             const int w2 = 2 * a.szw;
-                            sv[b][0] = __half2float(sh[gid * w2 + o0]);
-                            sv[b][1] = __half2float(sh[(gid + 8) * w2 + o1]);
-                            zv0 = __half2float(sh[(kMR + gid) * w2 + o0]);
-                            zv1 = __half2float(sh[(kMR + gid + 8) * w2 + o1]);
+                            sv[b][0] = meta_to_float(sh[gid * w2 + o0], mbf);
+                            sv[b][1] = meta_to_float(sh[(gid + 8) * w2 + o1], mbf);
+                            zv0 = meta_to_float(sh[(kMR + gid) * w2 + o0], mbf);
+                            zv1 = meta_to_float(sh[(kMR + gid + 8) * w2 + o1], mbf);
                         }
                     }
-                    zz[b][0] = bf16x2_splat(128.0f + zv0);
-                    zz[b][1] = bf16x2_splat(128.0f + zv1);
+                    zo[b][0] = 128.0f + zv0;
+                    zo[b][1] = 128.0f + zv1;
+                    zz[b][0] = bf16x2_splat(zo[b][0]);
+                    zz[b][1] = bf16x2_splat(zo[b][1]);
                 }
                 // ---- eight mma steps, one accumulator per k block
                 float d[NB][4];
@@ -455,8 +474,13 @@ __global__ void __launch_bounds__(kMThreads, 1)
                     constexpr int kPer = 4 / NB;
                     const int b = i / kPer;
                     uint32_t pa[4], pb[4];
-                    unpack_word_bf16(wa[i], zz[b][0], pa);
-                    unpack_word_bf16(wb[i], zz[b][1], pb);
+                    if (!fz) {
+                        unpack_word_bf16(wa[i], zz[b][0], pa);
+                        unpack_word_bf16(wb[i], zz[b][1], pb);
+                    } else {
+                        unpack_word_bf16_rounded(wa[i], zo[b][0], pa);
+                        unpack_word_bf16_rounded(wb[i], zo[b][1], pb);
+                    }
                     mma_bf16_16816(d[b], pa[0], pb[0], pa[1], pb[1], bq[i].x, bq[i].y);
                     mma_bf16_16816(d[b], pa[2], pb[2], pa[3], pb[3], bq[i].z, bq[i].w);
                 }

@@ -269,7 +269,7 @@ __device__ __forceinline__ void q8_bf16_fragments(const uint16_t* __restrict__ X
 // scale.  Kept out of line so that the int8 path keeps its registers.
 template <int M, int NSET>
 __device__ __noinline__ float2 q8_bf16_stage(const uint16_t* __restrict__ X, int K, int kg, int lane, uint4 wa,
-                                             uint4 wb, uint32_t zz0, uint32_t zz1) {
+                                             uint4 wb, uint32_t zz0, uint32_t zz1, bool fz, float zo0, float zo1) {
     uint32_t hx[16];
     q8_bf16_fragments<M>(X, K, kg, lane, hx);
     float dh[4] = {0.f, 0.f, 0.f, 0.f};
@@ -277,8 +277,13 @@ __device__ __noinline__ float2 q8_bf16_stage(const uint16_t* __restrict__ X, int
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         uint32_t pa[4], pb[4];
-        unpack_word_bf16(wa4[i], zz0, pa);
-        unpack_word_bf16(wb4[i], zz1, pb);
+        if (!fz) {
+            unpack_word_bf16(wa4[i], zz0, pa);
+            unpack_word_bf16(wb4[i], zz1, pb);
+        } else {
+            unpack_word_bf16_rounded(wa4[i], zo0, pa);
+            unpack_word_bf16_rounded(wb4[i], zo1, pb);
+        }
         mma_bf16_16816(dh, pa[0], pb[0], pa[1], pb[1], hx[4 * i], hx[4 * i + 1]);
         mma_bf16_16816(dh, pa[2], pb[2], pa[3], pb[3], hx[4 * i + 2], hx[4 * i + 3]);
     }
@@ -314,9 +319,10 @@ struct GemvQ8Args {
     int stages;               // ring depth
     int szw;                  // 2-D box: groups per row; copy path: words per row and stage
     long long sz_total;       // halves in each of S and Z (N * sz_row, or 1)
+    int fmt;                  // format flags: kFmtZeroFloat, kFmtMetaBf16
 };
 
-template <int M, int SZ>
+template <int M, int SZ, bool FZ>
 __global__ void __launch_bounds__(kQThreads, 1)
     gemv_q8_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                    const __grid_constant__ CUtensorMap zmap, const GemvQ8Args a) {
@@ -429,14 +435,19 @@ __global__ void __launch_bounds__(kQThreads, 1)
         // ------------------------------------------------------ consumers
         uint32_t* tab = tabs + warp * kQTabWords;
         float2* yw = reinterpret_cast<float2*>(ysum + warp * kQYWords) + lane;   // [row block] stride 32
-        float s_const = 0.f;
+        const bool mbf = (a.fmt & kFmtMetaBf16) != 0;
+        // a fractional zero point z is taken as zi + (z - zi), zi = clamp(rint(z), 0, 15):
+        // the integer part goes through the exact integer sums, the rest is an fp32
+        // correction of the fold
+        constexpr bool fz = FZ;     // a.fmt & kFmtZeroFloat, as a template argument
+        float s_const = 0.f, z_const = 0.f;
         int z16_const = 0;
         uint32_t zz_const = 0u;
         if (SZ == kSzConst) {
-            const float zf = __half2float(a.Z[0]);
-            s_const = __half2float(a.S[0]);
-            z16_const = __float_as_int(fmaf(zf, 16.0f, 12582912.0f)) - 0x4B400000;
-            zz_const = bf16x2_splat(128.0f + zf);
+            z_const = meta_to_float(a.Z[0], mbf);
+            s_const = meta_to_float(a.S[0], mbf);
+            z16_const = __float_as_int(fmaf(z_const, 16.0f, 12582912.0f)) - 0x4B400000;
+            zz_const = bf16x2_splat(128.0f + z_const);
         }
         const uint8_t* ra_base = ring + gid * 1024 + warp * 64 + tig * 16;
 #pragma unroll
@@ -483,7 +494,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
                         float s0, s1, z0, z1;
                         if (SZ == kSzConst) {
                             s0 = s1 = s_const;
-                            z0 = z1 = 0.f;
+                            z0 = z1 = z_const;
                         } else {
                             const __half* sh = reinterpret_cast<const __half*>(sb + kMWBytes);
                             int o0 = so0, o1 = so1;
@@ -495,10 +506,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
                                 o0 = gid * w2 + grp - fg + ((((row0 + gid) & a.sz_row) ^ fg) & 1);
                                 o1 = (gid + 8) * w2 + grp - fg + ((((row0 + gid + 8) & a.sz_row) ^ fg) & 1);
                             }
-                            s0 = __half2float(sh[o0]);
-                            s1 = __half2float(sh[o1]);
-                            z0 = __half2float(sh[zo + o0]);
-                            z1 = __half2float(sh[zo + o1]);
+                            s0 = meta_to_float(sh[o0], mbf);
+                            s1 = meta_to_float(sh[o1], mbf);
+                            z0 = meta_to_float(sh[zo + o0], mbf);
+                            z1 = meta_to_float(sh[zo + o1], mbf);
                         }
                         if (!xg.bf16) {
                             // ---- int8 path: four mma per set, exact integer sums
@@ -521,20 +532,33 @@ __global__ void __launch_bounds__(kQThreads, 1)
                                     mma_u8s8_16832(dd[st], o0, o1, o2, o3, xg.b[st][4 * pr + 2], xg.b[st][4 * pr + 3]);
                                 }
                             }
-                            const int zq0 = SZ == kSzConst ? z16_const
-                                                           : __float_as_int(fmaf(z0, 16.0f, 12582912.0f)) - 0x4B400000;
-                            const int zq1 = SZ == kSzConst ? z16_const
-                                                           : __float_as_int(fmaf(z1, 16.0f, 12582912.0f)) - 0x4B400000;
+                            int zq0, zq1;          // 16 z (16 zi for a fractional zero), an integer
+                            float zr0 = 0.f, zr1 = 0.f;   // 16 (z - zi)
+                            if (!fz) {
+                                zq0 = SZ == kSzConst ? z16_const
+                                                     : __float_as_int(fmaf(z0, 16.0f, 12582912.0f)) - 0x4B400000;
+                                zq1 = SZ == kSzConst ? z16_const
+                                                     : __float_as_int(fmaf(z1, 16.0f, 12582912.0f)) - 0x4B400000;
+                            } else {
+                                const float zi0 = fminf(fmaxf(rintf(z0), 0.f), 15.f);
+                                const float zi1 = fminf(fmaxf(rintf(z1), 0.f), 15.f);
+                                zq0 = __float_as_int(fmaf(zi0, 16.0f, 12582912.0f)) - 0x4B400000;
+                                zq1 = __float_as_int(fmaf(zi1, 16.0f, 12582912.0f)) - 0x4B400000;
+                                zr0 = 16.0f * (z0 - zi0);
+                                zr1 = 16.0f * (z1 - zi1);
+                            }
                             float f[2];
 #pragma unroll
                             for (int h = 0; h < 2; ++h) {
                                 const int z16 = h ? zq1 : zq0;
+                                const float zr = h ? zr1 : zr0;
                                 // V = 16 sum q d of the lane's two columns of set 0
                                 const int va = 16 * de[0][2 * h] + dd[0][2 * h];
                                 const int vb = 16 * de[0][2 * h + 1] + dd[0][2 * h + 1];
                                 if (NSET == 1) {
                                     // (c2, d1) lanes: 256 V_c2 + V_d1; d0 lanes: V_d0 (vb = 0)
                                     f[h] = static_cast<float>(xg.khi * va + vb - z16 * xg.thi);
+                                    if (fz) f[h] = fmaf(-zr, static_cast<float>(xg.thi), f[h]);
                                 } else {
                                     const int wa_ = 16 * de[NSET - 1][2 * h] + dd[NSET - 1][2 * h];
                                     const int wb_ = 16 * de[NSET - 1][2 * h + 1] + dd[NSET - 1][2 * h + 1];
@@ -544,8 +568,13 @@ __global__ void __launch_bounds__(kQThreads, 1)
                                     const int mine = odd ? wa_ : 256 * va + vb;
                                     const int other = __shfl_xor_sync(0xFFFFFFFFu, odd ? va : 256 * wa_ + wb_, 1);
                                     const int hi = odd ? other : mine, lo = odd ? mine : other;
-                                    f[h] = fmaf(static_cast<float>(hi - z16 * xg.thi), 256.0f,
-                                                static_cast<float>(lo - z16 * xg.tlo));
+                                    float fh = static_cast<float>(hi - z16 * xg.thi);
+                                    float fl = static_cast<float>(lo - z16 * xg.tlo);
+                                    if (fz) {
+                                        fh = fmaf(-zr, static_cast<float>(xg.thi), fh);
+                                        fl = fmaf(-zr, static_cast<float>(xg.tlo), fl);
+                                    }
+                                    f[h] = fmaf(fh, 256.0f, fl);
                                 }
                             }
                             yv.x = fmaf(s0 * xg.xs, f[0], yv.x);
@@ -554,7 +583,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
                             // ---- bf16 path (rare): exact (q - z) x bf16 activations, fp32 sums
                             const uint32_t zz0 = SZ == kSzConst ? zz_const : bf16x2_splat(128.0f + z0);
                             const uint32_t zz1 = SZ == kSzConst ? zz_const : bf16x2_splat(128.0f + z1);
-                            const float2 d = q8_bf16_stage<M, NSET>(a.X, a.K, kg, lane, wa, wb, zz0, zz1);
+                            const float2 d = q8_bf16_stage<M, NSET>(a.X, a.K, kg, lane, wa, wb, zz0, zz1, fz,
+                                                                    128.0f + z0, 128.0f + z1);
                             yv.x = fmaf(s0, d.x, yv.x);
                             yv.y = fmaf(s1, d.y, yv.y);
                         }

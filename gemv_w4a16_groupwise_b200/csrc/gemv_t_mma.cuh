@@ -72,6 +72,7 @@ struct GemvTMmaArgs {
     int splits;              // row ranges
     int rows_per_split;      // a multiple of 32
     int stages;
+    int fmt;                 // format flags: kFmtZeroFloat, kFmtMetaBf16
 };
 
 // Ring, the warps' tables, dY of the split's rows (one float4 per row),
@@ -81,7 +82,7 @@ __host__ __device__ inline size_t gemv_t_mma_smem_bytes(int KW, int nset, int st
            static_cast<size_t>(rows_per_split) * 16 + static_cast<size_t>(stages) * 16 + 16;
 }
 
-template <int M, int KW, int SZ>
+template <int M, int KW, int SZ, bool FZ>
 __global__ void __launch_bounds__(kTMThreads, 1)
     gemv_t_mma_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                       const __grid_constant__ CUtensorMap zmap, const GemvTMmaArgs a) {
@@ -177,10 +178,17 @@ __global__ void __launch_bounds__(kTMThreads, 1)
         const int gid = lane >> 2, tig = lane & 3;
         const int kw = k0 + KW * warp;                   // the warp's first k
         const int grp = group_of(min(kw, a.K - 1));
+        const bool mbf = (a.fmt & kFmtMetaBf16) != 0;
+        // a fractional zero point z is taken as zi + (z - zi), zi = clamp(rint(z), 0, 15):
+        // the codes enter the mma as the exact bf16 q - zi, and since the
+        // warp's k columns share one group, the rest is one fp32 sum per
+        // activation row, sum_n c[n] (z - zi)[n], taken off every output
+        constexpr bool fz = FZ;     // a.fmt & kFmtZeroFloat, as a template argument
+        float corr[4] = {0.f, 0.f, 0.f, 0.f};
         float s_const = 0.f, z_const = 0.f;
         if (SZ == kSzConst) {
-            s_const = __half2float(a.S[0]);
-            z_const = __half2float(a.Z[0]);
+            s_const = meta_to_float(a.S[0], mbf);
+            z_const = meta_to_float(a.Z[0], mbf);
         }
         // dY of the CTA's rows into shared memory, one float4 per row (absent
         // m and rows past r1 read as 0, so rows a stage carries past r1 add
@@ -241,19 +249,26 @@ __global__ void __launch_bounds__(kTMThreads, 1)
                     zv = z_const;
                 } else if (SZ == kSzTma2d) {
                     const __half* sh = reinterpret_cast<const __half*>(sb + kSzOff);
-                    sv = __half2float(sh[lane * 16 + grp - x_sz]);
-                    zv = __half2float(sh[512 + lane * 16 + grp - x_sz]);
+                    sv = meta_to_float(sh[lane * 16 + grp - x_sz], mbf);
+                    zv = meta_to_float(sh[512 + lane * 16 + grp - x_sz], mbf);
                 } else {
                     const __half* sh = reinterpret_cast<const __half*>(sb + kSzOff);
-                    sv = __half2float(sh[lane]);
-                    zv = __half2float(sh[512 + lane]);
+                    sv = meta_to_float(sh[lane], mbf);
+                    zv = meta_to_float(sh[512 + lane], mbf);
                 }
                 const float4 d4 = dys[b * kTMRows + lane];
                 const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+                float zfr = 0.f;
+                if (fz) {
+                    const float zi = fminf(fmaxf(rintf(zv), 0.f), 15.f);
+                    zfr = zv - zi;                         // exact
+                    zv = zi;
+                }
                 __syncwarp();                              // the last stage's table reads are done
 #pragma unroll
                 for (int m = 0; m < M; ++m) {
                     const float c = dv[m] * sv;            // exact: 8 x 11 significant bits
+                    if (fz) corr[m] = fmaf(c, zfr, corr[m]);
                     const __nv_bfloat16 p0 = __float2bfloat16_rn(c);
                     const float q1 = c - __bfloat162float(p0);
                     const __nv_bfloat16 p1 = __float2bfloat16_rn(q1);
@@ -306,6 +321,12 @@ __global__ void __launch_bounds__(kTMThreads, 1)
                 phase ^= 1u;
             }
         }
+        if (fz) {
+#pragma unroll
+            for (int m = 0; m < M; ++m)
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) corr[m] += __shfl_xor_sync(0xFFFFFFFFu, corr[m], o);
+        }
         // ---- outputs: the three parts of each activation row meet in lane
         // tig = 0 (row 2 st) and tig = 1 (row 2 st + 1) of each gid: columns
         // (0, 1 | 2) and (3 | 4, 5) of the set
@@ -330,6 +351,11 @@ __global__ void __launch_bounds__(kTMThreads, 1)
                 for (int j = 0; j < NT; ++j)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) o[8 * (j >> 2) + (j & 3) + 4 * h] = v[2 * j + h];
+                if (fz) {
+                    const float cm = m == 0 ? corr[0] : m == 1 ? corr[1] : m == 2 ? corr[2] : corr[3];
+#pragma unroll
+                    for (int e = 0; e < 8 * NWD; ++e) o[e] -= cm;
+                }
                 if (a.splits == 1) {
                     uint32_t outw[4 * NWD];
 #pragma unroll

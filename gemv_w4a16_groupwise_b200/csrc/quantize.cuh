@@ -10,6 +10,11 @@
 //     q = clamp(rint(w / s) + z, 0, 15)
 // Clamps use fmaxf/fminf (a NaN lands on 0) and then convert to int, so a
 // negative zero never reaches the stored fp16 zero point.
+// Format flags (or-ed into the mode) give the HQQ-style variant of
+// "Re-write HQQ Fused Gemm Transpose" and bf16 metadata:
+//     fractional zero:  z = meta(-min / s) (kept finite in its type, not
+//                       rounded or clamped), q = clamp(rint(w / s + z), 0, 15)
+//     bf16 metadata:    every fp16 rounding above is a bf16 rounding.
 #pragma once
 
 #include "common.cuh"
@@ -17,24 +22,36 @@
 namespace w4 {
 
 struct GroupParams {
-    __half s;
-    float sf;   // float(s)
-    float rs;   // 1 / sf, correctly rounded
-    int z;
-    float zf;   // float(z)
+    uint16_t sb, zb;   // stored bits of s and z (fp16, or bf16)
+    float sf;          // value of s
+    float rs;          // 1 / sf, correctly rounded
+    float zf;          // value of z (an integer unless the zero is fractional)
+    bool fz;           // fractional zero point
 };
 
-__device__ __forceinline__ GroupParams group_params_from_range(float mn, float mx) {
+// Nearest value of the metadata type (fp16 or bf16), as stored bits.
+__device__ __forceinline__ uint16_t meta_bits_rn(float v, bool bf16) {
+    return bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(v)) : __half_as_ushort(__float2half_rn(v));
+}
+
+__device__ __forceinline__ GroupParams group_params_from_range(float mn, float mx, int flags) {
     GroupParams p;
+    const bool bf = (flags & kFmtMetaBf16) != 0;
+    p.fz = (flags & kFmtZeroFloat) != 0;
     const float range = __fsub_rn(mx, mn);
-    __half s = __float2half_rn(__fdiv_rn(range, 15.0f));
-    if (__half2float(s) == 0.0f) s = __float2half_rn(fmaxf(fabsf(mn), 0x1p-14f));
-    p.s = s;
-    p.sf = __half2float(s);
+    uint16_t sb = meta_bits_rn(__fdiv_rn(range, 15.0f), bf);
+    if (meta_to_float(sb, bf) == 0.0f) sb = meta_bits_rn(fmaxf(fabsf(mn), 0x1p-14f), bf);
+    p.sb = sb;
+    p.sf = meta_to_float(sb, bf);
     p.rs = __frcp_rn(p.sf);
-    const float zf = fminf(fmaxf(rintf(__fdiv_rn(-mn, p.sf)), 0.0f), 15.0f);
-    p.z = static_cast<int>(zf);
-    p.zf = static_cast<float>(p.z);
+    if (p.fz) {
+        const float zmax = bf ? 0x1.FEp127f : 65504.0f;      // largest finite value of the type
+        p.zb = meta_bits_rn(fminf(fmaxf(__fdiv_rn(-mn, p.sf), -zmax), zmax), bf);
+        p.zf = meta_to_float(p.zb, bf);
+    } else {
+        p.zf = fminf(fmaxf(rintf(__fdiv_rn(-mn, p.sf)), 0.0f), 15.0f);
+        p.zb = meta_bits_rn(static_cast<float>(static_cast<int>(p.zf)), bf);   // no negative zero
+    }
     return p;
 }
 
@@ -53,8 +70,22 @@ __device__ __forceinline__ float rint_quotient(float w, const GroupParams& p) {
     return rintf(__fdiv_rn(w, p.sf));
 }
 
+// rint(fp32(fp32(w / s) + z)) for a fractional z, through the same
+// reciprocal: t = w * (1/s) is within 2^-22 |t| of fp32(w / s), so u = t + z
+// is within 2^-22 |t| + one ulp of u of the exact sum's fp32 value; when u
+// is farther than that from every half-integer both round alike, else the
+// division and the sum are done exactly.
+__device__ __forceinline__ float rint_shifted_quotient(float w, const GroupParams& p) {
+    const float t = w * p.rs;
+    const float u = __fadd_rn(t, p.zf);
+    const float k = rintf(u);
+    const float margin = (fabsf(t) + 4.0f * fabsf(u)) * 0x1p-22f;
+    if (fabsf(u - k) < 0.5f - margin) return k;
+    return rintf(__fadd_rn(__fdiv_rn(w, p.sf), p.zf));
+}
+
 __device__ __forceinline__ uint32_t quantize_code(float w, const GroupParams& p) {
-    float t = __fadd_rn(rint_quotient(w, p), p.zf);
+    float t = p.fz ? rint_shifted_quotient(w, p) : __fadd_rn(rint_quotient(w, p), p.zf);
     t = fminf(fmaxf(t, 0.0f), 15.0f);
     // t is an integer in [0, 15]: adding 2^23 leaves it in the low mantissa bits
     return __float_as_uint(__fadd_rn(t, 8388608.0f)) & 0xFu;
@@ -83,7 +114,7 @@ __device__ __forceinline__ uint32_t pack8(const float (&v)[8], const GroupParams
 template <int LPG, int WPT>
 __global__ void __launch_bounds__(256) quantize_segmented_kernel(
     const uint16_t* __restrict__ W, long long total_words, uint32_t* __restrict__ packed,
-    __half* __restrict__ scales, __half* __restrict__ zeros) {
+    uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros, int flags) {
     const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     const long long w0 = t * WPT;                      // first word of the thread
     const bool active = w0 < total_words;
@@ -104,7 +135,7 @@ __global__ void __launch_bounds__(256) quantize_segmented_kernel(
         mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
         mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
     }
-    const GroupParams p = group_params_from_range(mn, mx);
+    const GroupParams p = group_params_from_range(mn, mx, flags);
     if (!active) return;
     if (WPT == 2) {
         *reinterpret_cast<uint2*>(packed + w0) = make_uint2(pack8(v[0], p), pack8(v[1], p));
@@ -114,8 +145,8 @@ __global__ void __launch_bounds__(256) quantize_segmented_kernel(
     }
     if ((threadIdx.x & (LPG - 1)) == 0) {
         const long long grp = t / LPG;
-        scales[grp] = p.s;
-        zeros[grp] = __int2half_rn(p.z);
+        scales[grp] = p.sb;
+        zeros[grp] = p.zb;
     }
 }
 
@@ -124,7 +155,7 @@ __global__ void __launch_bounds__(256) quantize_segmented_kernel(
 // (the re-read is an L2 hit for all but the longest rows).
 __global__ void __launch_bounds__(256) quantize_warp_group_kernel(
     const uint16_t* __restrict__ W, long long num_groups, int words_per_group,
-    uint32_t* __restrict__ packed, __half* __restrict__ scales, __half* __restrict__ zeros) {
+    uint32_t* __restrict__ packed, uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros, int flags) {
     const int lane = threadIdx.x & 31;
     const long long grp =
         static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
@@ -146,15 +177,15 @@ __global__ void __launch_bounds__(256) quantize_warp_group_kernel(
         mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
         mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
     }
-    const GroupParams p = group_params_from_range(mn, mx);
+    const GroupParams p = group_params_from_range(mn, mx, flags);
     for (int c = lane; c < words_per_group; c += 32) {
         float v[8];
         unpack8_bf16(__ldg(src + c), v);
         packed[base + c] = pack8(v, p);
     }
     if (lane == 0) {
-        scales[grp] = p.s;
-        zeros[grp] = __int2half_rn(p.z);
+        scales[grp] = p.sb;
+        zeros[grp] = p.zb;
     }
 }
 
@@ -199,8 +230,8 @@ __global__ void __launch_bounds__(256) global_minmax_kernel(const uint16_t* __re
 // grid-stride share of W; block 0 stores s and z.
 __global__ void __launch_bounds__(256) global_quantize_kernel(
     const uint16_t* __restrict__ W, long long total_words, const float2* __restrict__ partial,
-    int num_partial, uint32_t* __restrict__ packed, __half* __restrict__ scales,
-    __half* __restrict__ zeros) {
+    int num_partial, uint32_t* __restrict__ packed, uint16_t* __restrict__ scales,
+    uint16_t* __restrict__ zeros, int flags) {
     __shared__ GroupParams sp;
     if (threadIdx.x < 32) {
         float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
@@ -214,13 +245,13 @@ __global__ void __launch_bounds__(256) global_quantize_kernel(
             mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
             mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
         }
-        if (threadIdx.x == 0) sp = group_params_from_range(mn, mx);
+        if (threadIdx.x == 0) sp = group_params_from_range(mn, mx, flags);
     }
     __syncthreads();
     const GroupParams p = sp;
     if (blockIdx.x == 0 && threadIdx.x == 0) {
-        scales[0] = p.s;
-        zeros[0] = __int2half_rn(p.z);
+        scales[0] = p.sb;
+        zeros[0] = p.zb;
     }
     for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
          t < total_words; t += static_cast<long long>(gridDim.x) * blockDim.x) {

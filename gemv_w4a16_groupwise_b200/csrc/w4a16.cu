@@ -166,23 +166,25 @@ struct Meta {
     int g;       // group length along K (K for ROWWISE / GLOBAL)
     int G;       // groups per row
     int sz_row;  // row stride of the scale / zero arrays
+    int fmt;     // format flags of the mode (kFmtZeroFloat, kFmtMetaBf16)
 };
 
+// The mode argument: a base mode or-ed with format flags.
+constexpr int kModeBaseMask = 0x0F;
+
 w4_status check_mode(int K, int mode, int group_size, Meta* meta) {
-    if (mode == W4_MODE_GLOBAL) {
-        *meta = Meta{K, 1, 0};
-        return W4_OK;
+    const int fmt = mode & ~kModeBaseMask;
+    if (fmt & ~(W4_ZERO_FLOAT | W4_META_BF16)) return W4_ERR_INVALID_ARG;
+    static_assert(W4_ZERO_FLOAT == kFmtZeroFloat && W4_META_BF16 == kFmtMetaBf16, "format flags");
+    switch (mode & kModeBaseMask) {
+        case W4_MODE_GLOBAL: *meta = Meta{K, 1, 0, fmt}; return W4_OK;
+        case W4_MODE_ROWWISE: *meta = Meta{K, 1, 1, fmt}; return W4_OK;
+        case W4_MODE_GROUPWISE:
+            if (group_size < 8 || group_size % 8 != 0 || K % group_size != 0) return W4_ERR_INVALID_ARG;
+            *meta = Meta{group_size, K / group_size, K / group_size, fmt};
+            return W4_OK;
+        default: return W4_ERR_INVALID_ARG;
     }
-    if (mode == W4_MODE_ROWWISE) {
-        *meta = Meta{K, 1, 1};
-        return W4_OK;
-    }
-    if (mode == W4_MODE_GROUPWISE) {
-        if (group_size < 8 || group_size % 8 != 0 || K % group_size != 0) return W4_ERR_INVALID_ARG;
-        *meta = Meta{group_size, K / group_size, K / group_size};
-        return W4_OK;
-    }
-    return W4_ERR_INVALID_ARG;
 }
 
 std::atomic<uint64_t> g_launches{0};
@@ -417,32 +419,32 @@ size_t gemv_workspace(int M, int N, int K, int transposed, int sms) {
 // The GEMV is always launched as a programmatic dependent of the work just
 // before it: its prologue overlaps that work's tail, and it waits for that
 // work before reading any input.
-template <int M, int CLS, int SZ>
+template <int M, int CLS, int SZ, bool FZ>
 w4_status launch_gemv_mma_k(const MmaPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
                             const CUtensorMap& zm, const GemvMmaArgs& a, cudaStream_t st) {
-    auto* fn = gemv_mma_kernel<M, CLS, SZ>;
+    auto* fn = gemv_mma_kernel<M, CLS, SZ, FZ>;
     if (ensure_smem(reinterpret_cast<const void*>(fn), p.smem) != cudaSuccess) return W4_ERR_CUDA;
     launch_pdl(fn, dim3(p.grid), dim3(kMThreads), p.smem, st, wm, sm, zm, a);
     return launch_status();
 }
 
-template <int M, int CLS>
+template <int M, int CLS, bool FZ>
 w4_status launch_gemv_mma_c(const MmaPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
                             const CUtensorMap& zm, const GemvMmaArgs& a, cudaStream_t st) {
     switch (p.sz) {
-        case kSzConst: return launch_gemv_mma_k<M, CLS, kSzConst>(p, wm, sm, zm, a, st);
-        case kSzTma2d: return launch_gemv_mma_k<M, CLS, kSzTma2d>(p, wm, sm, zm, a, st);
-        case kSzTma1d: return launch_gemv_mma_k<M, CLS, kSzTma1d>(p, wm, sm, zm, a, st);
-        default: return launch_gemv_mma_k<M, CLS, kSzCopy>(p, wm, sm, zm, a, st);
+        case kSzConst: return launch_gemv_mma_k<M, CLS, kSzConst, FZ>(p, wm, sm, zm, a, st);
+        case kSzTma2d: return launch_gemv_mma_k<M, CLS, kSzTma2d, FZ>(p, wm, sm, zm, a, st);
+        case kSzTma1d: return launch_gemv_mma_k<M, CLS, kSzTma1d, FZ>(p, wm, sm, zm, a, st);
+        default: return launch_gemv_mma_k<M, CLS, kSzCopy, FZ>(p, wm, sm, zm, a, st);
     }
 }
 
-template <int M>
+template <int M, bool FZ>
 w4_status launch_gemv_mma_m(const MmaPlan& p, const CUtensorMap& wm, const CUtensorMap& sm,
                             const CUtensorMap& zm, const GemvMmaArgs& a, cudaStream_t st) {
     // group lengths that are a multiple of 128 run the int8 kernel
-    if (p.cls == kCls64) return launch_gemv_mma_c<M, kCls64>(p, wm, sm, zm, a, st);
-    return launch_gemv_mma_c<M, kCls32>(p, wm, sm, zm, a, st);
+    if (p.cls == kCls64) return launch_gemv_mma_c<M, kCls64, FZ>(p, wm, sm, zm, a, st);
+    return launch_gemv_mma_c<M, kCls32, FZ>(p, wm, sm, zm, a, st);
 }
 
 w4_status run_gemv_mma(const MmaPlan& p, int M, int N, int K, const void* A, const uint32_t* packed,
@@ -475,6 +477,7 @@ w4_status run_gemv_mma(const MmaPlan& p, int M, int N, int K, const void* A, con
     a.g = meta.g;
     a.G = meta.G;
     a.sz_row = meta.sz_row;
+    a.fmt = meta.fmt;
     group_magic(meta.g, &a.gmul, &a.gshift);
     a.TKC = p.TKC;
     a.splits = p.splits;
@@ -485,11 +488,12 @@ w4_status run_gemv_mma(const MmaPlan& p, int M, int N, int K, const void* A, con
     a.szw = p.szw;
     a.sz_total = meta.sz_row ? static_cast<long long>(N) * meta.sz_row : 1;
     w4_status s = W4_OK;
+    const bool fz = (meta.fmt & kFmtZeroFloat) != 0;
     switch (M) {
-        case 1: s = launch_gemv_mma_m<1>(p, wm, sm, zm, a, st); break;
-        case 2: s = launch_gemv_mma_m<2>(p, wm, sm, zm, a, st); break;
-        case 3: s = launch_gemv_mma_m<3>(p, wm, sm, zm, a, st); break;
-        case 4: s = launch_gemv_mma_m<4>(p, wm, sm, zm, a, st); break;
+        case 1: s = fz ? launch_gemv_mma_m<1, true>(p, wm, sm, zm, a, st) : launch_gemv_mma_m<1, false>(p, wm, sm, zm, a, st); break;
+        case 2: s = fz ? launch_gemv_mma_m<2, true>(p, wm, sm, zm, a, st) : launch_gemv_mma_m<2, false>(p, wm, sm, zm, a, st); break;
+        case 3: s = fz ? launch_gemv_mma_m<3, true>(p, wm, sm, zm, a, st) : launch_gemv_mma_m<3, false>(p, wm, sm, zm, a, st); break;
+        case 4: s = fz ? launch_gemv_mma_m<4, true>(p, wm, sm, zm, a, st) : launch_gemv_mma_m<4, false>(p, wm, sm, zm, a, st); break;
         default: return W4_ERR_INVALID_ARG;
     }
     if (s != W4_OK) return s;
@@ -504,23 +508,23 @@ w4_status run_gemv_mma(const MmaPlan& p, int M, int N, int K, const void* A, con
     return W4_OK;
 }
 
-template <int M, int SZ>
+template <int M, int SZ, bool FZ>
 w4_status launch_q8_k(const Q8Plan& p, const CUtensorMap& wm, const CUtensorMap& sm, const CUtensorMap& zm,
                       const GemvQ8Args& a, cudaStream_t st) {
-    auto* fn = gemv_q8_kernel<M, SZ>;
+    auto* fn = gemv_q8_kernel<M, SZ, FZ>;
     if (ensure_smem(reinterpret_cast<const void*>(fn), p.smem) != cudaSuccess) return W4_ERR_CUDA;
     launch_pdl(fn, dim3(p.grid), dim3(kQThreads), p.smem, st, wm, sm, zm, a);
     return launch_status();
 }
 
-template <int M>
+template <int M, bool FZ>
 w4_status launch_q8_m(const Q8Plan& p, const CUtensorMap& wm, const CUtensorMap& sm, const CUtensorMap& zm,
                       const GemvQ8Args& a, cudaStream_t st) {
     switch (p.sz) {
-        case kSzConst: return launch_q8_k<M, kSzConst>(p, wm, sm, zm, a, st);
-        case kSzTma2d: return launch_q8_k<M, kSzTma2d>(p, wm, sm, zm, a, st);
-        case kSzTma1d: return launch_q8_k<M, kSzTma1d>(p, wm, sm, zm, a, st);
-        default: return launch_q8_k<M, kSzCopy>(p, wm, sm, zm, a, st);
+        case kSzConst: return launch_q8_k<M, kSzConst, FZ>(p, wm, sm, zm, a, st);
+        case kSzTma2d: return launch_q8_k<M, kSzTma2d, FZ>(p, wm, sm, zm, a, st);
+        case kSzTma1d: return launch_q8_k<M, kSzTma1d, FZ>(p, wm, sm, zm, a, st);
+        default: return launch_q8_k<M, kSzCopy, FZ>(p, wm, sm, zm, a, st);
     }
 }
 
@@ -554,6 +558,7 @@ w4_status run_gemv_q8(const Q8Plan& p, int M, int N, int K, const void* A, const
     a.g = meta.g;
     a.G = meta.G;
     a.sz_row = meta.sz_row;
+    a.fmt = meta.fmt;
     group_magic(meta.g, &a.gmul, &a.gshift);
     a.TKC = p.TKC;
     a.splits = p.splits;
@@ -564,11 +569,12 @@ w4_status run_gemv_q8(const Q8Plan& p, int M, int N, int K, const void* A, const
     a.szw = p.szw;
     a.sz_total = meta.sz_row ? static_cast<long long>(N) * meta.sz_row : 1;
     w4_status s = W4_OK;
+    const bool fz = (meta.fmt & kFmtZeroFloat) != 0;
     switch (M) {
-        case 1: s = launch_q8_m<1>(p, wm, sm, zm, a, st); break;
-        case 2: s = launch_q8_m<2>(p, wm, sm, zm, a, st); break;
-        case 3: s = launch_q8_m<3>(p, wm, sm, zm, a, st); break;
-        case 4: s = launch_q8_m<4>(p, wm, sm, zm, a, st); break;
+        case 1: s = fz ? launch_q8_m<1, true>(p, wm, sm, zm, a, st) : launch_q8_m<1, false>(p, wm, sm, zm, a, st); break;
+        case 2: s = fz ? launch_q8_m<2, true>(p, wm, sm, zm, a, st) : launch_q8_m<2, false>(p, wm, sm, zm, a, st); break;
+        case 3: s = fz ? launch_q8_m<3, true>(p, wm, sm, zm, a, st) : launch_q8_m<3, false>(p, wm, sm, zm, a, st); break;
+        case 4: s = fz ? launch_q8_m<4, true>(p, wm, sm, zm, a, st) : launch_q8_m<4, false>(p, wm, sm, zm, a, st); break;
         default: return W4_ERR_INVALID_ARG;
     }
     if (s != W4_OK) return s;
@@ -609,6 +615,7 @@ w4_status run_gemv_fwd(const void* A, int M, int N, int K, const uint32_t* packe
     a.g = meta.g;
     a.G = meta.G;
     a.sz_row = meta.sz_row;
+    a.fmt = meta.fmt;
     const int blocks = static_cast<int>((static_cast<long long>(N) * 32 + 255) / 256);
     switch (M) {
         case 1: gemv_fwd_simple_kernel<1><<<blocks, 256, 0, st>>>(a, packed); break;
@@ -620,31 +627,31 @@ w4_status run_gemv_fwd(const void* A, int M, int N, int K, const uint32_t* packe
     return launch_status();
 }
 
-template <int M, int KW, int SZ>
+template <int M, int KW, int SZ, bool FZ>
 w4_status launch_t_mma_k(const TMmaPlan& p, const CUtensorMap& wm, const CUtensorMap& sm, const CUtensorMap& zm,
                          const GemvTMmaArgs& a, cudaStream_t st) {
-    auto* fn = gemv_t_mma_kernel<M, KW, SZ>;
+    auto* fn = gemv_t_mma_kernel<M, KW, SZ, FZ>;
     if (ensure_smem(reinterpret_cast<const void*>(fn), p.smem) != cudaSuccess) return W4_ERR_CUDA;
     launch_pdl(fn, dim3(p.grid), dim3(kTMThreads), p.smem, st, wm, sm, zm, a);
     return launch_status();
 }
 
-template <int M, int KW>
+template <int M, int KW, bool FZ>
 w4_status launch_t_mma_kw(const TMmaPlan& p, int sz, const CUtensorMap& wm, const CUtensorMap& sm,
                           const CUtensorMap& zm, const GemvTMmaArgs& a, cudaStream_t st) {
     switch (sz) {
-        case kSzConst: return launch_t_mma_k<M, KW, kSzConst>(p, wm, sm, zm, a, st);
-        case kSzTma1d: return launch_t_mma_k<M, KW, kSzTma1d>(p, wm, sm, zm, a, st);
-        default: return launch_t_mma_k<M, KW, kSzTma2d>(p, wm, sm, zm, a, st);
+        case kSzConst: return launch_t_mma_k<M, KW, kSzConst, FZ>(p, wm, sm, zm, a, st);
+        case kSzTma1d: return launch_t_mma_k<M, KW, kSzTma1d, FZ>(p, wm, sm, zm, a, st);
+        default: return launch_t_mma_k<M, KW, kSzTma2d, FZ>(p, wm, sm, zm, a, st);
     }
 }
 
-template <int M>
+template <int M, bool FZ>
 w4_status launch_t_mma_m(const TMmaPlan& p, int sz, const CUtensorMap& wm, const CUtensorMap& sm,
                          const CUtensorMap& zm, const GemvTMmaArgs& a, cudaStream_t st) {
     // M = 3, 4 always take KW = 64 (two column sets)
-    if (M <= 2 && p.KW == 128) return launch_t_mma_kw<M, (M <= 2 ? 128 : 64)>(p, sz, wm, sm, zm, a, st);
-    return launch_t_mma_kw<M, 64>(p, sz, wm, sm, zm, a, st);
+    if (M <= 2 && p.KW == 128) return launch_t_mma_kw<M, (M <= 2 ? 128 : 64), FZ>(p, sz, wm, sm, zm, a, st);
+    return launch_t_mma_kw<M, 64, FZ>(p, sz, wm, sm, zm, a, st);
 }
 
 w4_status run_gemv_t_mma(const TMmaPlan& p, int sz, int M, int N, int K, const void* A, const uint32_t* packed,
@@ -676,16 +683,18 @@ w4_status run_gemv_t_mma(const TMmaPlan& p, int sz, int M, int N, int K, const v
     a.g = meta.g;
     a.G = meta.G;
     a.sz_row = meta.sz_row;
+    a.fmt = meta.fmt;
     a.strips = p.strips;
     a.splits = p.splits;
     a.rows_per_split = p.rows_per_split;
     a.stages = p.stages;
     w4_status s = W4_OK;
+    const bool fz = (meta.fmt & kFmtZeroFloat) != 0;
     switch (M) {
-        case 1: s = launch_t_mma_m<1>(p, sz, wm, sm, zm, a, st); break;
-        case 2: s = launch_t_mma_m<2>(p, sz, wm, sm, zm, a, st); break;
-        case 3: s = launch_t_mma_m<3>(p, sz, wm, sm, zm, a, st); break;
-        case 4: s = launch_t_mma_m<4>(p, sz, wm, sm, zm, a, st); break;
+        case 1: s = fz ? launch_t_mma_m<1, true>(p, sz, wm, sm, zm, a, st) : launch_t_mma_m<1, false>(p, sz, wm, sm, zm, a, st); break;
+        case 2: s = fz ? launch_t_mma_m<2, true>(p, sz, wm, sm, zm, a, st) : launch_t_mma_m<2, false>(p, sz, wm, sm, zm, a, st); break;
+        case 3: s = fz ? launch_t_mma_m<3, true>(p, sz, wm, sm, zm, a, st) : launch_t_mma_m<3, false>(p, sz, wm, sm, zm, a, st); break;
+        case 4: s = fz ? launch_t_mma_m<4, true>(p, sz, wm, sm, zm, a, st) : launch_t_mma_m<4, false>(p, sz, wm, sm, zm, a, st); break;
         default: return W4_ERR_INVALID_ARG;
     }
     if (s != W4_OK) return s;
@@ -726,6 +735,7 @@ w4_status run_gemv_t(const void* A, int M, int N, int K, const uint32_t* packed,
     a.g = meta.g;
     a.G = meta.G;
     a.sz_row = meta.sz_row;
+    a.fmt = meta.fmt;
     a.rows_per_split = p.rows_per_split;
     a.splits = p.splits;
     const dim3 grid((K / 8 + kGemvTWordsPerCta - 1) / kGemvTWordsPerCta, p.splits);
@@ -874,6 +884,7 @@ w4_status run_gemm_simple(const TcProblem& p, cudaStream_t st) {
     a.g = p.g;
     a.G = p.G;
     a.sz_row = p.sz_row;
+    a.fmt = p.fmt;
     const int L = p.transposed ? p.K : p.N;
     const dim3 grid((L + kGsTile - 1) / kGsTile, (p.M + kGsTile - 1) / kGsTile);
     if (p.transposed)
@@ -916,6 +927,7 @@ w4_status run_gemm_tc(const TcProblem& p, void* ws, size_t ws_bytes, cudaStream_
     a.g = p.g;
     a.G = p.G;
     a.sz_row = p.sz_row;
+    a.fmt = p.fmt;
     a.stages = stages;
     a.part = static_cast<float*>(ws);
     a.F = plan.F;
@@ -989,7 +1001,7 @@ const char* w4_status_string(int status) {
 size_t w4_quantize_workspace_bytes(int N, int K, int mode) {
     (void)N;
     (void)K;
-    return mode == W4_MODE_GLOBAL ? 1024 * sizeof(float2) : 0;
+    return (mode & kModeBaseMask) == W4_MODE_GLOBAL ? 1024 * sizeof(float2) : 0;
 }
 
 w4_status w4_quantize_pack(const void* W, int N, int K, int mode, int group_size, uint32_t* packed,
@@ -1024,11 +1036,12 @@ w4_status w4_quantize_pack(const void* W, int N, int K, int mode, int group_size
         if (flag) return W4_ERR_INVALID_ARG;
     }
     const uint16_t* w = static_cast<const uint16_t*>(W);
-    __half* sc = static_cast<__half*>(scales);
-    __half* ze = static_cast<__half*>(zeros);
+    uint16_t* sc = static_cast<uint16_t*>(scales);
+    uint16_t* ze = static_cast<uint16_t*>(zeros);
+    const int fmt = meta.fmt;
     const long long total_words = static_cast<long long>(N) * (K / 8);
     const DeviceInfo di = device_info(current_device());
-    if (mode == W4_MODE_GLOBAL) {
+    if ((mode & kModeBaseMask) == W4_MODE_GLOBAL) {
         const int blocks = static_cast<int>(
             std::min<long long>(1024, std::min<long long>((total_words + 255) / 256, di.sms * 4)));
         float2* part = static_cast<float2*>(workspace);
@@ -1037,7 +1050,7 @@ w4_status w4_quantize_pack(const void* W, int N, int K, int mode, int group_size
         if (s != W4_OK) return s;
         const int qblocks =
             static_cast<int>(std::min<long long>((total_words + 255) / 256, di.sms * 8));
-        global_quantize_kernel<<<qblocks, 256, 0, st>>>(w, total_words, part, blocks, packed, sc, ze);
+        global_quantize_kernel<<<qblocks, 256, 0, st>>>(w, total_words, part, blocks, packed, sc, ze, fmt);
         return launch_status();
     }
     // words per group: two words per thread (one for g = 8), lanes of a group
@@ -1046,17 +1059,17 @@ w4_status w4_quantize_pack(const void* W, int N, int K, int mode, int group_size
     const int wpt = lpg >= 2 ? 2 : 1;
     const int blocks = static_cast<int>((total_words / wpt + 255) / 256);
     switch (lpg) {
-        case 1: quantize_segmented_kernel<1, 1><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
-        case 2: quantize_segmented_kernel<1, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
-        case 4: quantize_segmented_kernel<2, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
-        case 8: quantize_segmented_kernel<4, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
-        case 16: quantize_segmented_kernel<8, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
-        case 32: quantize_segmented_kernel<16, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
-        case 64: quantize_segmented_kernel<32, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze); break;
+        case 1: quantize_segmented_kernel<1, 1><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
+        case 2: quantize_segmented_kernel<1, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
+        case 4: quantize_segmented_kernel<2, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
+        case 8: quantize_segmented_kernel<4, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
+        case 16: quantize_segmented_kernel<8, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
+        case 32: quantize_segmented_kernel<16, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
+        case 64: quantize_segmented_kernel<32, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
         default: {
             const long long groups = total_words / lpg;
             const int gblocks = static_cast<int>((groups + 7) / 8);
-            quantize_warp_group_kernel<<<gblocks, 256, 0, st>>>(w, groups, lpg, packed, sc, ze);
+            quantize_warp_group_kernel<<<gblocks, 256, 0, st>>>(w, groups, lpg, packed, sc, ze, fmt);
         }
     }
     return launch_status();
@@ -1108,6 +1121,7 @@ w4_status w4a16_gemm(const void* A, int M, int N, int K, const uint32_t* packed,
     pr.g = meta.g;
     pr.G = meta.G;
     pr.sz_row = meta.sz_row;
+    pr.fmt = meta.fmt;
     pr.bias = bias;
     pr.transposed = transposed;
     pr.Y = Y;

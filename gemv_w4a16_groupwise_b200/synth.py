@@ -104,6 +104,20 @@ def plant_structure(W: np.ndarray, g: int, seed: int) -> np.ndarray:
     return W
 
 
+def offset_groups(W: np.ndarray, g: int, seed: int, share: float = 0.25, amp: float = 0.08) -> np.ndarray:
+    """Copy of bf16 W where a seeded ``share`` of the g-long groups is shifted by an
+    offset uniform in [-amp, amp] (groups that do not straddle zero, whose min-max
+    zero point then lies far outside the code range)."""
+    W = np.array(W, dtype=np.uint16, copy=True)
+    N, K = W.shape
+    rng = np.random.default_rng([int(seed), 55])
+    G = K // g
+    pick = rng.random((N, G)) < share
+    off = rng.uniform(-amp, amp, (N, G)) * pick
+    vals = bf16_bits_to_f32(W).astype(np.float64) + np.repeat(off, g, axis=1)
+    return f64_to_bf16_bits(vals)
+
+
 def outlier_activations(M: int, K: int, seed: int, exp: int, period: int = 128,
                         stream: int = STREAM_X) -> tuple[np.ndarray, np.ndarray]:
     """N(0, 1) bf16 rows with one entry of magnitude 2^exp (random sign) in every

@@ -59,6 +59,25 @@ typedef enum w4_mode {
 } w4_mode;
 
 /*
+ * Format flags, or-ed into the `mode` argument of every call (the quantizer
+ * and the matmuls must be given the same ones).  Without flags the zero
+ * point is an integer in [0, 15] and s, z are fp16.
+ *   W4_ZERO_FLOAT  fractional zero point, the HQQ-style quantizer ("Re-write
+ *                  HQQ Fused Gemm Transpose": its fused GEMM keeps a float
+ *                  zero):  z = meta(-min / s), neither rounded to an integer
+ *                  nor clamped to [0, 15] (only kept finite in its type), and
+ *                  q = clamp(rint(w / s + z), 0, 15).
+ *   W4_META_BF16   s and z are stored as bf16 instead of fp16 (every fp16
+ *                  rounding of the quantizer becomes a bf16 rounding).
+ * With W4_ZERO_FLOAT, q - z is no longer a small integer: the kernels round
+ * it once (to bf16 on the bf16-mma and tensor-core paths, in fp32 on the
+ * CUDA-core ones), except the int8 forward GEMV and the transposed GEMV,
+ * which keep the integer part zi = clamp(rint(z), 0, 15) exact and add the
+ * rest, (z - zi) times the activation sum, in fp32.
+ */
+enum { W4_ZERO_FLOAT = 0x10, W4_META_BF16 = 0x20 };
+
+/*
  * Workspace bytes w4_quantize_pack needs for (N, K, mode): non-zero only for
  * GLOBAL, whose min/max runs as a separate grid-wide pass.
  */
@@ -72,11 +91,15 @@ size_t w4_quantize_workspace_bytes(int N, int K, int mode);
  *     s = fp16((max - min) / 15); if s == 0: s = fp16(max(|min|, 2^-14))
  *     z = clamp(rint(-min / s), 0, 15)
  *     q = clamp(rint(w / s) + z, 0, 15)
- * in IEEE fp32 with round-half-even; results are bit-exact against the
- * CPU oracle.  Inputs must be finite and satisfy (max - min) / 15 <= 65504.
+ * in IEEE fp32 with round-half-even (with the format flags above: the
+ * fractional zero point and / or bf16 metadata); results are bit-exact
+ * against the CPU oracle.  Inputs must be finite and, for fp16 metadata,
+ * satisfy (max - min) / 15 <= 65504.
  *
- * Outputs: packed uint32 [N, K/8]; scales, zeros fp16 (see conventions).
- * Validation: N, K > 0; K % 8 == 0; mode in range; GROUPWISE needs
+ * Outputs: packed uint32 [N, K/8]; scales, zeros fp16 or bf16 bits (see
+ * conventions).
+ * Validation: N, K > 0; K % 8 == 0; mode in range (unknown flag bits are
+ * W4_ERR_INVALID_ARG); GROUPWISE needs
  * group_size >= 8, group_size % 8 == 0, K % group_size == 0; pointers
  * non-NULL and 16-byte aligned; workspace_bytes >=
  * w4_quantize_workspace_bytes(N, K, mode).
