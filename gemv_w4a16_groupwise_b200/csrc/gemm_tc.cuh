@@ -172,7 +172,7 @@ __device__ __forceinline__ uint4 dequant_word_bf16(uint32_t w, float s, float c_
     return out;
 }
 
-template <bool TR, int BN, bool PWG>
+template <bool TR, int BN, bool PWG, bool FZ>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap pmap, const __grid_constant__ CUtensorMap bmap,
                    const TcArgs a) {
@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if ((a.g & (a.g - 1)) == 0) gshift = __ffs(a.g) - 1;
         auto group_of = [&](int k) { return min(gshift >= 0 ? (k >> gshift) : k / a.g, a.G - 1); };
         const bool mbf = (a.fmt & kFmtMetaBf16) != 0;
-        const bool fz = (a.fmt & kFmtZeroFloat) != 0;
+        constexpr bool fz = FZ;     // a.fmt & kFmtZeroFloat, as a template argument
         // Scale / zero of one stage (tile i, block kb); with g a multiple of
         // 32 the thread's 4 words share one group.
         constexpr int NG = PWG ? 4 : 1;

@@ -848,25 +848,32 @@ size_t gemm_tc_workspace_bytes(int M, int N, int K, int transposed, int sms) {
     return plan_tc(M, N, K, transposed, sms).ws;
 }
 
-template <bool TR, int BN, bool PWG>
+template <bool TR, int BN, bool PWG, bool FZ>
 w4_status launch_tc(const CUtensorMap& pm, const CUtensorMap& bm, const TcArgs& a, dim3 grid,
                     size_t smem, cudaStream_t st) {
-    const void* fn = reinterpret_cast<const void*>(gemm_tc_kernel<TR, BN, PWG>);
+    const void* fn = reinterpret_cast<const void*>(gemm_tc_kernel<TR, BN, PWG, FZ>);
     if (ensure_smem(fn, smem) != cudaSuccess) return W4_ERR_CUDA;
-    gemm_tc_kernel<TR, BN, PWG><<<grid, kTcThreads, smem, st>>>(pm, bm, a);
+    gemm_tc_kernel<TR, BN, PWG, FZ><<<grid, kTcThreads, smem, st>>>(pm, bm, a);
     return launch_status();
 }
 
-template <bool TR, bool PWG>
+template <bool TR, bool PWG, bool FZ>
 w4_status launch_tc_bn(int BN, const CUtensorMap& pm, const CUtensorMap& bm, const TcArgs& a,
                        dim3 grid, size_t smem, cudaStream_t st) {
     switch (BN) {
-        case 16: return launch_tc<TR, 16, PWG>(pm, bm, a, grid, smem, st);
-        case 32: return launch_tc<TR, 32, PWG>(pm, bm, a, grid, smem, st);
-        case 64: return launch_tc<TR, 64, PWG>(pm, bm, a, grid, smem, st);
-        case 128: return launch_tc<TR, 128, PWG>(pm, bm, a, grid, smem, st);
-        default: return launch_tc<TR, 256, PWG>(pm, bm, a, grid, smem, st);
+        case 16: return launch_tc<TR, 16, PWG, FZ>(pm, bm, a, grid, smem, st);
+        case 32: return launch_tc<TR, 32, PWG, FZ>(pm, bm, a, grid, smem, st);
+        case 64: return launch_tc<TR, 64, PWG, FZ>(pm, bm, a, grid, smem, st);
+        case 128: return launch_tc<TR, 128, PWG, FZ>(pm, bm, a, grid, smem, st);
+        default: return launch_tc<TR, 256, PWG, FZ>(pm, bm, a, grid, smem, st);
     }
+}
+
+template <bool TR, bool PWG>
+w4_status launch_tc_fz(bool fz, int BN, const CUtensorMap& pm, const CUtensorMap& bm, const TcArgs& a,
+                       dim3 grid, size_t smem, cudaStream_t st) {
+    return fz ? launch_tc_bn<TR, PWG, true>(BN, pm, bm, a, grid, smem, st)
+              : launch_tc_bn<TR, PWG, false>(BN, pm, bm, a, grid, smem, st);
 }
 
 // Shapes whose rows TMA cannot stream: the plain CUDA-core kernel.
@@ -938,10 +945,11 @@ w4_status run_gemm_tc(const TcProblem& p, void* ws, size_t ws_bytes, cudaStream_
     // persistent: one CTA per SM (or per work unit, when there are fewer)
     const dim3 grid(static_cast<unsigned>(plan.grid));
     const bool pwg = (p.g % 32) != 0;
-    w4_status s = tr ? (pwg ? launch_tc_bn<true, true>(BN, pm, bm, a, grid, smem, st)
-                            : launch_tc_bn<true, false>(BN, pm, bm, a, grid, smem, st))
-                     : (pwg ? launch_tc_bn<false, true>(BN, pm, bm, a, grid, smem, st)
-                            : launch_tc_bn<false, false>(BN, pm, bm, a, grid, smem, st));
+    const bool fz = (p.fmt & kFmtZeroFloat) != 0;
+    w4_status s = tr ? (pwg ? launch_tc_fz<true, true>(fz, BN, pm, bm, a, grid, smem, st)
+                            : launch_tc_fz<true, false>(fz, BN, pm, bm, a, grid, smem, st))
+                     : (pwg ? launch_tc_fz<false, true>(fz, BN, pm, bm, a, grid, smem, st)
+                            : launch_tc_fz<false, false>(fz, BN, pm, bm, a, grid, smem, st));
     if (s != W4_OK || plan.F == plan.tiles) return s;
     const long long threads = static_cast<long long>(plan.tiles - plan.F) * BN * (kTcBM / 4);
     launch_pdl(gemm_tail_finalize_kernel, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0, st,
