@@ -51,6 +51,12 @@ def split_range(total: int, world: int, rank: int, quantum: int = 1) -> tuple[in
     return lo * quantum, hi * quantum
 
 
+def _own(t):
+    """A copy of a slice in storage of its own: slices of the full layer can start off
+    the 16-byte alignment the library requires, fresh allocations do not."""
+    return t.clone(memory_format=_torch().contiguous_format)
+
+
 def _mode_base(mode) -> str:
     if isinstance(mode, str):
         return mode
@@ -78,7 +84,7 @@ def shard_columns(packed, scales, zeros, mode, group_size: int, N: int, K: int, 
         s, z = scales, zeros
     else:
         s, z = scales[lo:hi], zeros[lo:hi]
-    return Shard(packed[lo:hi].contiguous(), s.contiguous(), z.contiguous(), hi - lo, K, lo, hi)
+    return Shard(_own(packed[lo:hi]), _own(s), _own(z), hi - lo, K, lo, hi)
 
 
 def shard_rows(packed, scales, zeros, mode, group_size: int, N: int, K: int, rank: int,
@@ -90,10 +96,10 @@ def shard_rows(packed, scales, zeros, mode, group_size: int, N: int, K: int, ran
     if quantum % 8:
         raise ValueError("the group length must be a multiple of 8")
     lo, hi = split_range(K, world, rank, quantum)
-    p = packed[:, lo // 8:hi // 8].contiguous()
+    p = _own(packed[:, lo // 8:hi // 8])
     if base == "groupwise":
-        s = scales[:, lo // group_size:hi // group_size].contiguous()
-        z = zeros[:, lo // group_size:hi // group_size].contiguous()
+        s = _own(scales[:, lo // group_size:hi // group_size])
+        z = _own(zeros[:, lo // group_size:hi // group_size])
     else:
         s, z = scales, zeros
     return Shard(p, s, z, N, hi - lo, lo, hi)
@@ -147,7 +153,7 @@ class ColumnParallelW4A16:
         self.mode, self.g, self.N, self.K, self.zero = mode, group_size, N, K, zero
         self.shard = shard_columns(packed, scales, zeros, mode, group_size, N, K, self.rank, self.comm.world)
         self.sizes = [split_range(N, self.comm.world, r) for r in range(self.comm.world)]
-        self.bias = None if bias is None else bias[self.shard.lo:self.shard.hi].contiguous()
+        self.bias = None if bias is None else _own(bias[self.shard.lo:self.shard.hi])
         self.matmul = matmul or _default_matmul()
 
     def forward(self, X, gather: bool = True):
@@ -164,7 +170,7 @@ class ColumnParallelW4A16:
         """dY [M, N] (whole, or this rank's [M, N1 - N0]) -> dX [M, K], summed over ranks."""
         torch = _torch()
         sh = self.shard
-        d = dY[:, sh.lo:sh.hi].contiguous() if dY.shape[1] == self.N and self.comm.world > 1 else dY
+        d = _own(dY[:, sh.lo:sh.hi]) if dY.shape[1] == self.N and self.comm.world > 1 else dY
         part = self.matmul(d, sh.packed, sh.scales, sh.zeros, self.mode, self.g, N=sh.N, K=self.K,
                            transposed=True, zero=self.zero)
         return self.comm.all_reduce_sum(part).to(torch.bfloat16)
@@ -189,7 +195,7 @@ class RowParallelW4A16:
         """X [M, K] (whole) or this rank's X [M, K1 - K0] -> Y [M, N] (all-reduced, + bias once)."""
         torch = _torch()
         sh = self.shard
-        x = X[:, sh.lo:sh.hi].contiguous() if X.shape[1] == self.K and self.comm.world > 1 else X
+        x = _own(X[:, sh.lo:sh.hi]) if X.shape[1] == self.K and self.comm.world > 1 else X
         part = self.matmul(x, sh.packed, sh.scales, sh.zeros, self.mode, self.g, N=self.N, K=sh.K,
                            zero=self.zero)
         y = self.comm.all_reduce_sum(part)
