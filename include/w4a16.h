@@ -156,6 +156,8 @@ w4_status w4a16_gemm(const void *A, int M, int N, int K, const uint32_t *packed,
  *   transposed: bf16 mma, dY * s split into three exact bf16 parts;
  *   K or g not a multiple of 32 (or scale layouts the TMA boxes do not
  *     take): CUDA-core kernels with exact (q - z) and fp32 fma.
+ * With W4_ZERO_FLOAT the int8 and transposed paths keep the integer part of
+ * z exact and add the rest in fp32; the other paths round q - z once.
  * Same arguments and results as w4a16_gemm; M must be 1..4
  * (W4_ERR_INVALID_ARG otherwise).
  */
@@ -209,8 +211,8 @@ uint64_t w4_launch_count(void);
  *
  * Limits and sharing:
  *   - The scratch holds the fp32 partial sums of a plan that splits K (few
- *     output rows and a long K, or activations too long for shared
- *     memory).  Every problem with w4_workspace_bytes(M, N, K, 0) <= 8 MiB
+ *     output rows and a long K).  Every problem with
+ *     w4_workspace_bytes(M, N, K, 0) <= 8 MiB
  *     runs; a larger one runs when the plan for its own group length fits,
  *     else the call returns W4_ERR_WORKSPACE and launches nothing.
  *   - Every call on a device shares the one array.  Calls that may overlap
