@@ -18,7 +18,8 @@ transposed / with bias, fused QKV) are timed once each under "rows", and
 every configuration of the workload list (the tiny case, the Llama-3.2-1B
 layers in three modes with quantize-and-pack, the Llama-2-7B QLoRA layers
 forward and transposed, the Llama-3-8B serving layers with bias at M = 1 ..
-1024) under "configs", each against its own roofline.
+1024, the fractional-zero / bf16-scale variant) under "configs", each
+against its own roofline.
 
 Multi-GPU: one process per GPU (torchrun); each rank runs the whole sweep on
 its own GPU (independent problems, no data-path collective), value = bytes

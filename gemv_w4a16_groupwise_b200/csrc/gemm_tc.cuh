@@ -19,7 +19,10 @@
 // units write fp32 partial tiles, which gemm_tail_finalize_kernel adds in
 // slice order (with the bias) and rounds, so the last wave takes about
 // 1 / S of a tile's time instead of a whole one.  Warp roles (704 threads):
-//   warp 0       TMA producer: packed weight tile + activation tile per stage
+//   warp 0       TMA producer: packed weight tile + activation tile per stage,
+//                and, for groupwise scales whose row stride is a multiple of
+//                16 bytes, a box of 8 groups x the tile's rows of S and of Z,
+//                so that the scales arrive with the weights a ring ahead
 //   warp 1       TMEM allocator; lane 0 issues tcgen05.mma and commits
 //   warps 2..17  dequantize packed codes into the bf16 A tile of a stage
 //                (128-byte swizzled UMMA layout).  Two groups of 8 warps take
@@ -63,6 +66,8 @@ struct TcArgs {
     int M, N, K;
     int g, G, sz_row;
     int stages;
+    int stage_bytes;      // tc_stage_bytes(BN), plus the scale / zero boxes when sz_tma
+    int sz_tma;           // scales and zeros come with each stage (TMA boxes)
     int F;                // tiles 0 .. F - 1 are whole work units
     int nslice;           // k slices of each tile from F on (1: no split)
 };
@@ -175,9 +180,12 @@ __device__ __forceinline__ uint4 dequant_word_bf16(uint32_t w, float s, float c_
 template <bool TR, int BN, bool PWG, bool FZ>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap pmap, const __grid_constant__ CUtensorMap bmap,
+                   const __grid_constant__ CUtensorMap smap, const __grid_constant__ CUtensorMap zmap,
                    const TcArgs a) {
     static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 256, "BN");
-    constexpr int kStageBytes = tc_stage_bytes(BN);
+    const int kStageBytes = a.stage_bytes;
+    constexpr int kSzOff = tc_stage_bytes(BN);                  // the stage's scale / zero boxes
+    constexpr int kSzRows = TR ? kTcBK : kTcBM;                 // weight rows of a stage
     constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;          // one accumulator buffer
     constexpr uint32_t kTmemCols = 2 * kAccCols;              // two, a power of two >= 64
     constexpr uint32_t kTxBytes = kTcPBytes + BN * 128;
@@ -256,6 +264,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
             tma_prefetch_desc(&pmap);
             tma_prefetch_desc(&bmap);
+            if (a.sz_tma) {
+                tma_prefetch_desc(&smap);
+                tma_prefetch_desc(&zmap);
+            }
             int s = 0;
             uint32_t round = 0;
             bool ok = true;
@@ -268,12 +280,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         break;
                     }
                     uint8_t* st = base + s * kStageBytes;
-                    mbar_arrive_expect_tx(&tma_full[s], kTxBytes);
+                    mbar_arrive_expect_tx(&tma_full[s], kTxBytes + (a.sz_tma ? 2 * kSzRows * 16 : 0));
                     if (TR)
                         tma_load_2d(st + kTcABytes + BN * 128, &pmap, r0 / 8, kb * kTcBK, &tma_full[s]);
                     else
                         tma_load_2d(st + kTcABytes + BN * 128, &pmap, kb * (kTcBK / 8), r0, &tma_full[s]);
                     tma_load_2d(st + kTcABytes, &bmap, kb * kTcBK, m0, &tma_full[s]);
+                    if (a.sz_tma) {
+                        // groups from the stage's first one, rounded down to a
+                        // multiple of 8 (16 bytes), for the stage's weight rows
+                        const int x0 = (min((TR ? r0 : kb * kTcBK) / a.g, a.G - 1)) & ~7;
+                        const int y0 = TR ? kb * kTcBK : r0;
+                        tma_load_2d(st + kSzOff, &smap, x0, y0, &tma_full[s]);
+                        tma_load_2d(st + kSzOff + kSzRows * 16, &zmap, x0, y0, &tma_full[s]);
+                    }
                     if (++s == NS) {
                         s = 0;
                         ++round;
@@ -388,14 +408,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint32_t phase = static_cast<uint32_t>(grp_id / NS) & 1u;
         float sv[NG], zv[NG], svn[NG], zvn[NG];
         int cr0 = ci < my_units ? tile_r0(ci) : 0;           // output row offset of the current tile
-        if (ci < my_units) load_sz(cr0, ckb, sv, zv);
+        if (ci < my_units && !a.sz_tma) load_sz(cr0, ckb, sv, zv);
         while (ci < my_units) {
             // the next stage of this group, whose scales are fetched now
             int ni = ci, nkb = ckb, nb1 = cb1;
             advance(ni, nkb, nb1, kTcDeqGroups);
             const bool more = ni < my_units;
             const int nr0 = (more && ni != ci) ? tile_r0(ni) : cr0;
-            if (more) load_sz(nr0, nkb, svn, zvn);
+            if (more && !a.sz_tma) load_sz(nr0, nkb, svn, zvn);
             const int r0 = cr0;
             const int n = TR ? ckb * kTcBK + prow : r0 + prow;
             const int kw0 = TR ? r0 / 8 + 4 * pquad : ckb * (kTcBK / 8) + 4 * pquad;
@@ -404,6 +424,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                                                       kErrTimeoutTmaFull));
             if (ok) {
                 uint8_t* st = base + s * kStageBytes;
+                if (a.sz_tma) {
+                    // this stage's boxes: [S rows][8 groups] then [Z rows][8 groups]
+                    const uint16_t* hs = reinterpret_cast<const uint16_t*>(st + kSzOff) + prow * 8;
+                    const uint16_t* hz = hs + kSzRows * 8;
+                    const int x0 = group_of(TR ? r0 : ckb * kTcBK) & ~7;
+#pragma unroll
+                    for (int j = 0; j < NG; ++j) {
+                        const int idx = group_of(8 * (kw0 + j)) - x0;
+                        sv[j] = meta_to_float(hs[idx], mbf);
+                        zv[j] = meta_to_float(hz[idx], mbf);
+                    }
+                }
                 const uint8_t* pk = st + kTcABytes + BN * 128;
                 const uint4 wv = TR ? *reinterpret_cast<const uint4*>(pk + prow * 64 + pquad * 16)
                                     : *reinterpret_cast<const uint4*>(pk + prow * 32 + pquad * 16);
@@ -421,10 +453,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&deq_full[s]);
             }
+            if (!a.sz_tma) {
 #pragma unroll
-            for (int j = 0; j < NG; ++j) {
-                sv[j] = svn[j];
-                zv[j] = zvn[j];
+                for (int j = 0; j < NG; ++j) {
+                    sv[j] = svn[j];
+                    zv[j] = zvn[j];
+                }
             }
             ci = ni;
             ckb = nkb;

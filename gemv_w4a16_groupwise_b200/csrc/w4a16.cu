@@ -849,31 +849,30 @@ size_t gemm_tc_workspace_bytes(int M, int N, int K, int transposed, int sms) {
 }
 
 template <bool TR, int BN, bool PWG, bool FZ>
-w4_status launch_tc(const CUtensorMap& pm, const CUtensorMap& bm, const TcArgs& a, dim3 grid,
-                    size_t smem, cudaStream_t st) {
+w4_status launch_tc(const CUtensorMap& pm, const CUtensorMap& bm, const CUtensorMap& sm, const CUtensorMap& zm,
+                    const TcArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
     const void* fn = reinterpret_cast<const void*>(gemm_tc_kernel<TR, BN, PWG, FZ>);
     if (ensure_smem(fn, smem) != cudaSuccess) return W4_ERR_CUDA;
-    gemm_tc_kernel<TR, BN, PWG, FZ><<<grid, kTcThreads, smem, st>>>(pm, bm, a);
+    gemm_tc_kernel<TR, BN, PWG, FZ><<<grid, kTcThreads, smem, st>>>(pm, bm, sm, zm, a);
     return launch_status();
 }
 
 template <bool TR, bool PWG, bool FZ>
-w4_status launch_tc_bn(int BN, const CUtensorMap& pm, const CUtensorMap& bm, const TcArgs& a,
-                       dim3 grid, size_t smem, cudaStream_t st) {
+w4_status launch_tc_bn(int BN, const CUtensorMap* m, const TcArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
     switch (BN) {
-        case 16: return launch_tc<TR, 16, PWG, FZ>(pm, bm, a, grid, smem, st);
-        case 32: return launch_tc<TR, 32, PWG, FZ>(pm, bm, a, grid, smem, st);
-        case 64: return launch_tc<TR, 64, PWG, FZ>(pm, bm, a, grid, smem, st);
-        case 128: return launch_tc<TR, 128, PWG, FZ>(pm, bm, a, grid, smem, st);
-        default: return launch_tc<TR, 256, PWG, FZ>(pm, bm, a, grid, smem, st);
+        case 16: return launch_tc<TR, 16, PWG, FZ>(m[0], m[1], m[2], m[3], a, grid, smem, st);
+        case 32: return launch_tc<TR, 32, PWG, FZ>(m[0], m[1], m[2], m[3], a, grid, smem, st);
+        case 64: return launch_tc<TR, 64, PWG, FZ>(m[0], m[1], m[2], m[3], a, grid, smem, st);
+        case 128: return launch_tc<TR, 128, PWG, FZ>(m[0], m[1], m[2], m[3], a, grid, smem, st);
+        default: return launch_tc<TR, 256, PWG, FZ>(m[0], m[1], m[2], m[3], a, grid, smem, st);
     }
 }
 
 template <bool TR, bool PWG>
-w4_status launch_tc_fz(bool fz, int BN, const CUtensorMap& pm, const CUtensorMap& bm, const TcArgs& a,
-                       dim3 grid, size_t smem, cudaStream_t st) {
-    return fz ? launch_tc_bn<TR, PWG, true>(BN, pm, bm, a, grid, smem, st)
-              : launch_tc_bn<TR, PWG, false>(BN, pm, bm, a, grid, smem, st);
+w4_status launch_tc_fz(bool fz, int BN, const CUtensorMap* m, const TcArgs& a, dim3 grid, size_t smem,
+                       cudaStream_t st) {
+    return fz ? launch_tc_bn<TR, PWG, true>(BN, m, a, grid, smem, st)
+              : launch_tc_bn<TR, PWG, false>(BN, m, a, grid, smem, st);
 }
 
 // Shapes whose rows TMA cannot stream: the plain CUDA-core kernel.
@@ -908,20 +907,33 @@ w4_status run_gemm_tc(const TcProblem& p, void* ws, size_t ws_bytes, cudaStream_
     const TcPlan plan = plan_tc(p.M, p.N, p.K, p.transposed, di.sms);
     if (plan.ws > ws_bytes || (plan.ws > 0 && ws == nullptr)) return W4_ERR_WORKSPACE;
     const int BN = plan.BN;
-    const int stage = tc_stage_bytes(BN);
+    const bool tr = p.transposed != 0;
+    // scales and zeros ride on each stage as 8-group TMA boxes when the rows
+    // are 16-byte strided and a stage's k range (64, transposed 128) never
+    // leaves the box that starts at its first group rounded down to 8
+    const int L = tr ? 128 : kTcBK;
+    const bool sz_tma = p.G > 1 && p.G % 8 == 0 &&
+                        (p.g % L == 0 || (L % p.g == 0 && L / p.g <= 8));
+    const int sz_rows = tr ? kTcBK : kTcBM;
+    const int stage = tc_stage_bytes(BN) + (sz_tma ? 2 * sz_rows * 16 : 0);
     const size_t fixed = 1024 + 64;
     int stages = static_cast<int>((static_cast<size_t>(di.max_smem_optin) - fixed - 64) / (stage + 24));
     stages = std::min(stages, 8);
     if (stages < 2) return W4_ERR_UNSUPPORTED;
     const size_t smem = fixed + static_cast<size_t>(stages) * stage + static_cast<size_t>(3 * stages + 4) * 8 + 16;
-    const bool tr = p.transposed != 0;
-    CUtensorMap pm, bm;
+    CUtensorMap maps[4];
+    std::memset(maps, 0, sizeof maps);
+    CUtensorMap& pm = maps[0];
+    CUtensorMap& bm = maps[1];
     // packed weights [N, K/8] uint32: box 8 words x 128 rows (forward) or
     // 16 words x 64 rows (transposed); activations [M, K] or dY [M, N] bf16,
     // box 64 x BN with the 128-byte swizzle the MMA descriptors expect
     bool ok = tr ? make_map_2d(&pm, p.packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, p.N, p.K / 8, 64, 16, 0)
                  : make_map_2d(&pm, p.packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, p.N, p.K / 8, 128, 8, 0);
     ok = ok && make_map_2d(&bm, p.A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.M, tr ? p.N : p.K, BN, 64, 128);
+    if (sz_tma)
+        ok = ok && make_map_2d(&maps[2], p.S, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.N, p.G, sz_rows, 8, 0) &&
+             make_map_2d(&maps[3], p.Z, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, p.N, p.G, sz_rows, 8, 0);
     if (!ok) return W4_ERR_CUDA;
     TcArgs a;
     a.S = static_cast<const __half*>(p.S);
@@ -936,6 +948,8 @@ w4_status run_gemm_tc(const TcProblem& p, void* ws, size_t ws_bytes, cudaStream_
     a.sz_row = p.sz_row;
     a.fmt = p.fmt;
     a.stages = stages;
+    a.stage_bytes = stage;
+    a.sz_tma = sz_tma ? 1 : 0;
     a.part = static_cast<float*>(ws);
     a.F = plan.F;
     a.nslice = plan.S;
@@ -946,10 +960,10 @@ w4_status run_gemm_tc(const TcProblem& p, void* ws, size_t ws_bytes, cudaStream_
     const dim3 grid(static_cast<unsigned>(plan.grid));
     const bool pwg = (p.g % 32) != 0;
     const bool fz = (p.fmt & kFmtZeroFloat) != 0;
-    w4_status s = tr ? (pwg ? launch_tc_fz<true, true>(fz, BN, pm, bm, a, grid, smem, st)
-                            : launch_tc_fz<true, false>(fz, BN, pm, bm, a, grid, smem, st))
-                     : (pwg ? launch_tc_fz<false, true>(fz, BN, pm, bm, a, grid, smem, st)
-                            : launch_tc_fz<false, false>(fz, BN, pm, bm, a, grid, smem, st));
+    w4_status s = tr ? (pwg ? launch_tc_fz<true, true>(fz, BN, maps, a, grid, smem, st)
+                            : launch_tc_fz<true, false>(fz, BN, maps, a, grid, smem, st))
+                     : (pwg ? launch_tc_fz<false, true>(fz, BN, maps, a, grid, smem, st)
+                            : launch_tc_fz<false, false>(fz, BN, maps, a, grid, smem, st));
     if (s != W4_OK || plan.F == plan.tiles) return s;
     const long long threads = static_cast<long long>(plan.tiles - plan.F) * BN * (kTcBM / 4);
     launch_pdl(gemm_tail_finalize_kernel, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0, st,
