@@ -344,10 +344,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // takes stages grp_id, grp_id + 2, ...
         const int grp_id = (threadIdx.x - 64) >> 8;
         const int t = (threadIdx.x - 64) & 255;               // 0 .. 255 within the group
-        // forward: row n = r0 + t % 128, words 4h .. 4h+3 of the 8 in a k-block
+        // forward: row n = r0 + t / 2, words 4 (t % 2) .. + 3 of the 8 in a k-block
+        //   (a phase of 8 lanes reads 4 rows' 32 bytes: 128 contiguous bytes, no bank
+        //   conflict; its swizzled 16-byte stores still land in 8 distinct banks)
         // transposed: row n = kb * 64 + t % 64, words 4q .. 4q+3 of the 16 of a k-tile
-        const int prow = TR ? (t & 63) : (t & 127);
-        const int pquad = TR ? (t >> 6) : (t >> 7);
+        const int prow = TR ? (t & 63) : (t >> 1);
+        const int pquad = TR ? (t >> 6) : (t & 1);
         const int W8 = a.K / 8;
         // swizzled 16-byte destinations of this thread's 4 words in the A tile
         uint32_t off[4];
