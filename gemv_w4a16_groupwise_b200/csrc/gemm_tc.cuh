@@ -347,9 +347,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // forward: row n = r0 + t / 2, words 4 (t % 2) .. + 3 of the 8 in a k-block
         //   (a phase of 8 lanes reads 4 rows' 32 bytes: 128 contiguous bytes, no bank
         //   conflict; its swizzled 16-byte stores still land in 8 distinct banks)
-        // transposed: row n = kb * 64 + t % 64, words 4q .. 4q+3 of the 16 of a k-tile
-        const int prow = TR ? (t & 63) : (t >> 1);
-        const int pquad = TR ? (t >> 6) : (t & 1);
+        // transposed: row n = kb * 64 + prow, words 4q .. 4q+3 of the 16 of a k-tile,
+        //   with (prow, q) spread so that a phase of 8 lanes takes 4 rows x 2 quads of
+        //   one 64-k atom: its 16-byte loads meet at most 2 to a bank (4 before) and its
+        //   MN-major stores fall into 8 distinct banks
+        const int prow = TR ? (((t >> 4) << 2) | ((t >> 1) & 3)) : (t >> 1);
+        const int pquad = TR ? ((((t >> 3) & 1) << 1) | (t & 1)) : (t & 1);
         const int W8 = a.K / 8;
         // swizzled 16-byte destinations of this thread's 4 words in the A tile
         uint32_t off[4];
