@@ -18,8 +18,8 @@ transposed / with bias, fused QKV) are timed once each under "rows", and
 every configuration of the workload list (the tiny case, the Llama-3.2-1B
 layers in three modes with quantize-and-pack, the Llama-2-7B QLoRA layers
 forward and transposed, the Llama-3-8B serving layers with bias at M = 1 ..
-1024, the fractional-zero / bf16-scale variant) under "configs", each
-against its own roofline.
+1024, the fractional-zero / bf16-scale variant, act-order weights) under
+"configs", each against its own roofline.
 
 Multi-GPU: one process per GPU (torchrun); each rank runs the whole sweep on
 its own GPU (independent problems, no data-path collective), value = bytes
@@ -381,8 +381,8 @@ def measure_configs(torch, w4, dev, peaks, stream):
     flushed before it): the tiny correctness case, the Llama-3.2-1B layers in
     three quantization modes with quantize-and-pack of each weight, the
     Llama-2-7B QLoRA layers forward and transposed, the Llama-3-8B serving
-    layers with bias at M = 1 .. 1024, and the fractional-zero variant (fp16
-    and bf16 metadata) on decode and training shapes.  Each row reports the
+    layers with bias at M = 1 .. 1024, the fractional-zero variant (fp16
+    and bf16 metadata) and act-order weights on decode and training shapes.  Each row reports the
     fraction of its own roofline (the slower of tensor-core and HBM time)."""
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     gen = torch.Generator(device=dev)
@@ -498,6 +498,22 @@ def measure_configs(torch, w4, dev, peaks, stream):
                 del P, S, Z
             del W
         out["variant_float_zero"] = rows
+        # act-order weights (packed column j = input channel perm[j]): the gather of
+        # X's columns (forward) or the scatter of dX's (transposed) is inside the call
+        rows = []
+        for (N, K, g, Ms) in ((8192, 8192, 128, (1, 4)), (11008, 4096, 64, (2048,))):
+            W = rnd((N, K), 0.02)
+            perm = torch.randperm(K, generator=gen, device=dev).to(torch.int32)
+            P, S, Z = w4.w4_quantize_pack(W, "groupwise", g, perm=perm)
+            for M in Ms:
+                X, dY = rnd((M, K)), rnd((M, N))
+                rows.append(row("act-order fwd", M, N, K, "groupwise", g,
+                                lambda: w4.w4a16_gemm(X, P, S, Z, "groupwise", g, N=N, K=K, perm=perm)))
+                rows.append(row("act-order t", M, N, K, "groupwise", g,
+                                lambda: w4.w4a16_gemm(dY, P, S, Z, "groupwise", g, N=N, K=K, transposed=True,
+                                                      perm=perm), transposed=True))
+            del W, P, S, Z
+        out["variant_act_order"] = rows
         del flush
     torch.cuda.synchronize()
     return out

@@ -15,7 +15,12 @@ Entry points (same names as the C ABI in ``include/w4a16.h``):
   ``transposed=True``), optional bias
 * :func:`w4a16_gemv` -- the same for M <= 4 (TMA-streamed weights, exact
   products on the tensor pipe, fp32 sums)
+* :func:`w4_gather_columns` / :func:`w4_scatter_columns` -- the column
+  permutations of act-order weights (``perm=`` on the calls above)
 * :func:`w4_workspace_bytes`, :func:`w4_device_error`
+
+``packed`` may also be given as its two-per-byte view, uint8 [N, K/2] (the
+same bytes; the even k in the low nibble).
 """
 from __future__ import annotations
 
@@ -81,6 +86,10 @@ def library():
             lib.w4_debug_set_wait_limit.restype = I
             lib.w4_debug_withhold_stage.argtypes = [I]
             lib.w4_debug_withhold_stage.restype = I
+            lib.w4_gather_columns.argtypes = [P, I, I, P, I, P, P]
+            lib.w4_gather_columns.restype = I
+            lib.w4_scatter_columns.argtypes = [P, I, I, P, I, P, P]
+            lib.w4_scatter_columns.restype = I
             _lib = lib
     return _lib
 
@@ -117,6 +126,24 @@ def _check_cuda(t, name, dtype, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
+def _packed_words(packed, N: int, K: int):
+    """The packed codes as int32 [N, K/8]; a uint8 [N, K/2] two-per-byte view is
+    reinterpreted (same bytes), anything else is passed on for the checks."""
+    torch = _torch()
+    if isinstance(packed, torch.Tensor) and packed.dtype == torch.uint8:
+        if tuple(packed.shape) != (N, K // 2) or not packed.is_contiguous():
+            raise ValueError(f"uint8 packed codes must be contiguous [{N}, {K // 2}]")
+        return packed.view(torch.int32)
+    return packed
+
+
+def _check_perm(perm, K: int, dev):
+    torch = _torch()
+    _check_cuda(perm, "perm", torch.int32, (K,))
+    if perm.device != dev:
+        raise ValueError("perm must be on the activations' device")
+
+
 def _stream_ptr(device):
     torch = _torch()
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
@@ -142,15 +169,19 @@ def w4_workspace_bytes(M: int, N: int, K: int, transposed: bool = False) -> int:
 
 
 def w4_quantize_pack(W, mode="groupwise", group_size: int = 128, out=None, zero: str = "int",
-                     meta: str = "fp16"):
+                     meta: str = "fp16", perm=None):
     """Quantize bf16 W [N, K] (CUDA) -> (packed int32 [N, K/8], scales, zeros).
 
     ``zero="float"`` keeps a fractional zero point (the HQQ-style quantizer);
-    ``meta="bf16"`` stores scales and zeros as bf16 instead of fp16.
+    ``meta="bf16"`` stores scales and zeros as bf16 instead of fp16;
+    ``perm`` (int32 [K], a permutation) quantizes W[:, perm] (act-order).
     """
     torch = _torch()
     _check_cuda(W, "W", torch.bfloat16)
     N, K = W.shape
+    if perm is not None:
+        _check_perm(perm, K, W.device)
+        W = w4_gather_columns(W, perm)
     shape = meta_shape(N, K, mode, group_size)
     dev = W.device
     mdt = _meta_dtype(meta)
@@ -173,8 +204,20 @@ def w4_quantize_pack(W, mode="groupwise", group_size: int = 128, out=None, zero:
     return packed, scales, zeros
 
 
-def _matmul(fname, A, packed, scales, zeros, mode, group_size, N, K, bias, transposed, out, zero):
+def _matmul(fname, A, packed, scales, zeros, mode, group_size, N, K, bias, transposed, out, zero,
+            perm=None):
     torch = _torch()
+    packed = _packed_words(packed, N, K)
+    if perm is not None:
+        # act-order: forward gathers X's columns; transposed scatters dX's
+        _check_cuda(A, "A", torch.bfloat16)
+        _check_perm(perm, K, A.device)
+        if not transposed:
+            return _matmul(fname, w4_gather_columns(A, perm), packed, scales, zeros, mode, group_size, N, K,
+                           bias, False, out, zero)
+        bias_p = None if bias is None else w4_gather_columns(bias.view(1, -1), perm).view(-1)
+        part = _matmul(fname, A, packed, scales, zeros, mode, group_size, N, K, bias_p, True, None, zero)
+        return w4_scatter_columns(part, perm, K, out=out)
     _check_cuda(A, "A", torch.bfloat16)
     _check_cuda(packed, "packed", torch.int32, (N, K // 8))
     # the metadata type follows the scales' dtype (fp16 or bf16)
@@ -208,21 +251,64 @@ def _matmul(fname, A, packed, scales, zeros, mode, group_size, N, K, bias, trans
 
 
 def w4a16_gemm(A, packed, scales, zeros, mode="groupwise", group_size: int = 128, *, N: int,
-               K: int, bias=None, transposed: bool = False, out=None, zero: str = "int"):
+               K: int, bias=None, transposed: bool = False, out=None, zero: str = "int", perm=None):
     """Y = A . dequant(W)^T  (A [M, K])  or, transposed, dX = A . dequant(W)  (A [M, N]).
 
     ``zero`` must name the quantizer's zero point ("int" or "float"); bf16 scales
-    and zeros are recognised by their dtype."""
+    and zeros are recognised by their dtype; ``perm`` (int32 [K]) marks act-order
+    weights whose packed column j is input channel perm[j]."""
     return _matmul("w4a16_gemm", A, packed, scales, zeros, mode, group_size, N, K, bias,
-                   transposed, out, zero)
+                   transposed, out, zero, perm)
 
 
 def w4a16_gemv(A, packed, scales, zeros, mode="groupwise", group_size: int = 128, *, N: int,
-               K: int, bias=None, transposed: bool = False, out=None, zero: str = "int"):
+               K: int, bias=None, transposed: bool = False, out=None, zero: str = "int", perm=None):
     """Small-batch (M <= 4) path of :func:`w4a16_gemm`: TMA-streamed weights, exact
     products on the tensor pipe with fp32 sums, forward and transposed."""
     return _matmul("w4a16_gemv", A, packed, scales, zeros, mode, group_size, N, K, bias,
-                   transposed, out, zero)
+                   transposed, out, zero, perm)
+
+
+def w4_gather_columns(A, idx, out=None):
+    """out[m, j] = A[m, idx[j]]: bf16 A [M, C] (CUDA), int32 idx [L] -> bf16 [M, L]."""
+    torch = _torch()
+    _check_cuda(A, "A", torch.bfloat16)
+    _check_cuda(idx, "idx", torch.int32)
+    if A.dim() != 2 or idx.dim() != 1:
+        raise ValueError("A must be 2-D and idx 1-D")
+    M, C = A.shape
+    L = idx.shape[0]
+    if out is None:
+        out = torch.empty((M, L), dtype=torch.bfloat16, device=A.device)
+    else:
+        _check_cuda(out, "out", torch.bfloat16, (M, L))
+    with torch.cuda.device(A.device):
+        st = library().w4_gather_columns(A.data_ptr(), M, C, idx.data_ptr(), L, out.data_ptr(),
+                                         _stream_ptr(A.device))
+    if st != 0:
+        raise W4Error(st, "w4_gather_columns")
+    return out
+
+
+def w4_scatter_columns(A, idx, dst_cols: int, out=None):
+    """out[m, idx[j]] = A[m, j]: bf16 A [M, L], int32 idx [L] (no repeats) -> bf16
+    [M, dst_cols] (a fresh tensor, zero where no index lands, unless `out` is given)."""
+    torch = _torch()
+    _check_cuda(A, "A", torch.bfloat16)
+    _check_cuda(idx, "idx", torch.int32)
+    M, L = A.shape
+    if idx.shape != (L,):
+        raise ValueError(f"idx must have shape ({L},)")
+    if out is None:
+        out = torch.zeros((M, dst_cols), dtype=torch.bfloat16, device=A.device)
+    else:
+        _check_cuda(out, "out", torch.bfloat16, (M, dst_cols))
+    with torch.cuda.device(A.device):
+        st = library().w4_scatter_columns(A.data_ptr(), M, L, idx.data_ptr(), dst_cols, out.data_ptr(),
+                                          _stream_ptr(A.device))
+    if st != 0:
+        raise W4Error(st, "w4_scatter_columns")
+    return out
 
 
 def w4_launch_count() -> int:
@@ -253,6 +339,6 @@ def w4_device_error() -> int:
     """Read and clear the device error word (synchronizes); 0 = no kernel gave up."""
     code = ctypes.c_int(0)
     st = library().w4_device_error(ctypes.byref(code))
-    if st not in (0, 6):
+    if st not in (0, 1, 6) or (st == 1 and code.value == 0):
         raise W4Error(st, "w4_device_error")
     return int(code.value)

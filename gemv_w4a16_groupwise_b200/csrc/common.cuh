@@ -22,6 +22,7 @@ enum DeviceError : unsigned int {
     kErrTimeoutDequant = 2,     // the MMA issuer waited too long for dequantized tiles
     kErrTimeoutEmpty = 3,       // the producer waited too long for a free stage
     kErrTimeoutAccum = 4,       // the epilogue waited too long for the accumulator
+    kErrBadIndex = 5,           // a column index of a gather / scatter was out of range
 };
 
 // Debug controls, set from the host (w4_debug_set_wait_limit,

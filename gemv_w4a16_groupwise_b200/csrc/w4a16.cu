@@ -16,6 +16,7 @@
 #include "gemv_mma.cuh"
 #include "gemv_q8.cuh"
 #include "gemv_t_mma.cuh"
+#include "permute.cuh"
 #include "quantize.cuh"
 #include "w4a16.h"
 
@@ -1204,7 +1205,28 @@ w4_status w4_device_error(int* code) {
     if (cudaMemcpyFromSymbol(&v, w4::g_error_word, sizeof v) != cudaSuccess) return W4_ERR_CUDA;
     if (cudaMemcpyToSymbol(w4::g_error_word, &zero, sizeof zero) != cudaSuccess) return W4_ERR_CUDA;
     *code = static_cast<int>(v);
+    if (v == w4::kErrBadIndex) return W4_ERR_INVALID_ARG;
     return v ? W4_ERR_TIMEOUT : W4_OK;
+}
+
+w4_status w4_gather_columns(const void* A, int M, int src_cols, const int32_t* idx, int L, void* out,
+                            void* stream) {
+    if (M <= 0 || src_cols <= 0 || L <= 0 || !A || !idx || !out) return W4_ERR_INVALID_ARG;
+    const long long total = static_cast<long long>(M) * L;
+    const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 148 * 16));
+    w4::gather_columns_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint16_t*>(A), M, src_cols, idx, L, static_cast<uint16_t*>(out));
+    return launch_status();
+}
+
+w4_status w4_scatter_columns(const void* A, int M, int L, const int32_t* idx, int dst_cols, void* out,
+                             void* stream) {
+    if (M <= 0 || dst_cols <= 0 || L <= 0 || !A || !idx || !out) return W4_ERR_INVALID_ARG;
+    const long long total = static_cast<long long>(M) * L;
+    const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 148 * 16));
+    w4::scatter_columns_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint16_t*>(A), M, L, idx, dst_cols, static_cast<uint16_t*>(out));
+    return launch_status();
 }
 
 }  // extern "C"

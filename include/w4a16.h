@@ -166,14 +166,49 @@ w4_status w4a16_gemv(const void *A, int M, int N, int K, const uint32_t *packed,
                      const void *bias, int transposed, void *Y,
                      void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Act-order: weights quantized in a permuted input-channel order (the GPTQ
+ * "desc_act" variant that TensorRT-LLM "Modify small-batched weight only
+ * quantization" names beside channel-wise and group-wise AWQ/GPTQ).  When
+ * packed column j holds input channel perm[j] (perm a permutation of
+ * [0, K)), the products are
+ *     forward     Y = X[:, perm] . w_hat^T:  gather X's columns, then the matmul;
+ *     transposed  dX[:, perm] = dY . w_hat:  the matmul (with bias[perm] when a
+ *                                            bias is given), then scatter.
+ * The packed layout itself is unchanged; quantizing W[:, perm] gives it.
+ *
+ * w4_gather_columns -- out[m, j] = A[m, idx[j]] for m < M, j < L.
+ *   A: bf16 [M, src_cols] row-major; idx: int32 [L] (device); out: bf16
+ *   [M, L].  An idx[j] outside [0, src_cols) gives 0 there and records
+ *   code 5 in the device error word (w4_device_error then returns
+ *   W4_ERR_INVALID_ARG).
+ * w4_scatter_columns -- out[m, idx[j]] = A[m, j] for m < M, j < L.
+ *   A: bf16 [M, L]; out: bf16 [M, dst_cols]; idx must not repeat (a
+ *   repeated index is a race); an index outside [0, dst_cols) is skipped
+ *   and recorded as above.  Columns of out that no idx names are left as
+ *   they are.
+ * Both are asynchronous on `stream`; M, L and the column counts must be
+ * > 0 and the pointers non-NULL (W4_ERR_INVALID_ARG otherwise).
+ *
+ * Two-per-byte view: the packed uint32 [N, K/8] array is byte-identical to
+ * uint8 [N, K/2] with two codes per byte, the even k in the low nibble, so a
+ * caller holding that byte layout passes its pointer as `packed` unchanged.
+ */
+w4_status w4_gather_columns(const void *A, int M, int src_cols, const int32_t *idx, int L,
+                            void *out, void *stream);
+w4_status w4_scatter_columns(const void *A, int M, int L, const int32_t *idx, int dst_cols,
+                             void *out, void *stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *w4_status_string(int status);
 
 /*
  * w4_device_error -- read and clear the device-side error word of the
  * current device.  Kernels whose waits are bounded set it instead of
- * hanging; *code receives 0 when no kernel gave up.  Synchronizes the
- * device.  Returns W4_ERR_TIMEOUT when *code != 0, W4_ERR_CUDA on a CUDA
+ * hanging (codes 1..4: which wait gave up); the column gather / scatter set
+ * code 5 for an index out of range; *code receives 0 when nothing was
+ * recorded.  Synchronizes the device.  Returns W4_ERR_INVALID_ARG for code 5,
+ * W4_ERR_TIMEOUT for the other non-zero codes, W4_ERR_CUDA on a CUDA
  * failure, W4_OK otherwise.
  */
 w4_status w4_device_error(int *code);

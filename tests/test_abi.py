@@ -50,6 +50,9 @@ def test_status_strings_and_host_validation():
     assert lib.w4a16_gemm(*args(4, 64, 252, 2, 64)) == 1
     assert lib.w4a16_gemm(*args(4, 64, 256, 2, 48)) == 1
     assert lib.w4a16_gemm(*args(4, 64, 256, 9, 64)) == 1
+    assert lib.w4a16_gemm(*args(4, 64, 256, 2 | 0x40, 64)) == 1      # unknown format flag
+    assert lib.w4_gather_columns(fake, 0, 8, fake, 8, fake, None) == 1
+    assert lib.w4_scatter_columns(fake, 4, 8, None, 8, fake, None) == 1
     assert lib.w4a16_gemv(*args(4, 64, 256, 2, 64)[:0] + (None, 4, 64, 256, fake, fake, fake, 2, 64,
                                                            None, 0, fake, None, 0, None)) == 1
     assert lib.w4_quantize_pack(fake, 64, 250, 1, 0, fake, fake, fake, None, 0, None) == 1
