@@ -90,6 +90,8 @@ def library():
             lib.w4_gather_columns.restype = I
             lib.w4_scatter_columns.argtypes = [P, I, I, P, I, P, P]
             lib.w4_scatter_columns.restype = I
+            lib.w4_invert_permutation.argtypes = [P, I, P, P]
+            lib.w4_invert_permutation.restype = I
             _lib = lib
     return _lib
 
@@ -217,7 +219,8 @@ def _matmul(fname, A, packed, scales, zeros, mode, group_size, N, K, bias, trans
                            bias, False, out, zero)
         bias_p = None if bias is None else w4_gather_columns(bias.view(1, -1), perm).view(-1)
         part = _matmul(fname, A, packed, scales, zeros, mode, group_size, N, K, bias_p, True, None, zero)
-        return w4_scatter_columns(part, perm, K, out=out)
+        # dX[:, perm[j]] = part[:, j]: a gather by the inverse permutation
+        return w4_gather_columns(part, w4_invert_permutation(perm), out=out)
     _check_cuda(A, "A", torch.bfloat16)
     _check_cuda(packed, "packed", torch.int32, (N, K // 8))
     # the metadata type follows the scales' dtype (fp16 or bf16)
@@ -288,6 +291,19 @@ def w4_gather_columns(A, idx, out=None):
     if st != 0:
         raise W4Error(st, "w4_gather_columns")
     return out
+
+
+def w4_invert_permutation(perm, out=None):
+    """inv [n] with inv[perm[j]] = j (int32, CUDA; perm a permutation of [0, n))."""
+    torch = _torch()
+    _check_cuda(perm, "perm", torch.int32)
+    n = perm.shape[0]
+    inv = torch.empty_like(perm) if out is None else out
+    with torch.cuda.device(perm.device):
+        st = library().w4_invert_permutation(perm.data_ptr(), n, inv.data_ptr(), _stream_ptr(perm.device))
+    if st != 0:
+        raise W4Error(st, "w4_invert_permutation")
+    return inv
 
 
 def w4_scatter_columns(A, idx, dst_cols: int, out=None):

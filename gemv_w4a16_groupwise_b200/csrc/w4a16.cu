@@ -1209,23 +1209,55 @@ w4_status w4_device_error(int* code) {
     return v ? W4_ERR_TIMEOUT : W4_OK;
 }
 
+// Rows up to this size are staged in shared memory by the column gather /
+// scatter (two blocks per SM still fit).
+constexpr size_t kRowStageBytes = 96u << 10;
+
 w4_status w4_gather_columns(const void* A, int M, int src_cols, const int32_t* idx, int L, void* out,
                             void* stream) {
     if (M <= 0 || src_cols <= 0 || L <= 0 || !A || !idx || !out) return W4_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t row_bytes = (static_cast<size_t>(src_cols) * 2 + 15) & ~static_cast<size_t>(15);
+    if (row_bytes <= kRowStageBytes) {
+        if (ensure_smem(reinterpret_cast<const void*>(w4::gather_rows_kernel), row_bytes) != cudaSuccess)
+            return W4_ERR_CUDA;
+        const dim3 grid((L + w4::kGatherChunk - 1) / w4::kGatherChunk, std::min(M, 65535));
+        launch_pdl(w4::gather_rows_kernel, grid, dim3(512), row_bytes, st, static_cast<const uint16_t*>(A), M,
+                   src_cols, idx, L, static_cast<uint16_t*>(out));
+        return launch_status();
+    }
     const long long total = static_cast<long long>(M) * L;
     const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 148 * 16));
-    w4::gather_columns_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint16_t*>(A), M, src_cols, idx, L, static_cast<uint16_t*>(out));
+    w4::gather_columns_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint16_t*>(A), M, src_cols, idx, L,
+                                                      static_cast<uint16_t*>(out));
+    return launch_status();
+}
+
+w4_status w4_invert_permutation(const int32_t* perm, int n, int32_t* inv, void* stream) {
+    if (n <= 0 || !perm || !inv) return W4_ERR_INVALID_ARG;
+    const int blocks = std::min((n + 255) / 256, device_info(current_device()).sms * 4);
+    launch_pdl(w4::invert_permutation_kernel, dim3(blocks), dim3(256), 0, static_cast<cudaStream_t>(stream), perm,
+               n, inv);
     return launch_status();
 }
 
 w4_status w4_scatter_columns(const void* A, int M, int L, const int32_t* idx, int dst_cols, void* out,
                              void* stream) {
     if (M <= 0 || dst_cols <= 0 || L <= 0 || !A || !idx || !out) return W4_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t row_bytes = (static_cast<size_t>(dst_cols) * 2 + 15) & ~static_cast<size_t>(15);
+    if (row_bytes <= kRowStageBytes) {
+        if (ensure_smem(reinterpret_cast<const void*>(w4::scatter_rows_kernel), row_bytes) != cudaSuccess)
+            return W4_ERR_CUDA;
+        const int blocks = std::min(M, device_info(current_device()).sms * 4);
+        launch_pdl(w4::scatter_rows_kernel, dim3(blocks), dim3(512), row_bytes, st, static_cast<const uint16_t*>(A),
+                   M, L, idx, dst_cols, static_cast<uint16_t*>(out));
+        return launch_status();
+    }
     const long long total = static_cast<long long>(M) * L;
     const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 148 * 16));
-    w4::scatter_columns_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint16_t*>(A), M, L, idx, dst_cols, static_cast<uint16_t*>(out));
+    w4::scatter_columns_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint16_t*>(A), M, L, idx, dst_cols,
+                                                       static_cast<uint16_t*>(out));
     return launch_status();
 }
 

@@ -174,7 +174,9 @@ w4_status w4a16_gemv(const void *A, int M, int N, int K, const uint32_t *packed,
  * [0, K)), the products are
  *     forward     Y = X[:, perm] . w_hat^T:  gather X's columns, then the matmul;
  *     transposed  dX[:, perm] = dY . w_hat:  the matmul (with bias[perm] when a
- *                                            bias is given), then scatter.
+ *                                            bias is given), then the columns
+ *                                            put back (a gather by the inverse
+ *                                            permutation).
  * The packed layout itself is unchanged; quantizing W[:, perm] gives it.
  *
  * w4_gather_columns -- out[m, j] = A[m, idx[j]] for m < M, j < L.
@@ -198,6 +200,13 @@ w4_status w4_gather_columns(const void *A, int M, int src_cols, const int32_t *i
                             void *out, void *stream);
 w4_status w4_scatter_columns(const void *A, int M, int L, const int32_t *idx, int dst_cols,
                              void *out, void *stream);
+/*
+ * w4_invert_permutation -- inv[perm[j]] = j for j < n: int32 [n] device
+ * arrays; perm must be a permutation of [0, n) (an entry outside it is
+ * skipped and recorded as code 5).  A scatter by perm of a whole row is then
+ * the gather by inv, whose writes are contiguous.  Asynchronous on `stream`.
+ */
+w4_status w4_invert_permutation(const int32_t *perm, int n, int32_t *inv, void *stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *w4_status_string(int status);

@@ -42,6 +42,17 @@ def test_gather_scatter_bit_exact(cuda_device, M, L, C):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("n", [1, 777, 4096, 28672])
+def test_invert_permutation(cuda_device, n):
+    import torch
+    w4 = lib()
+    perm = _perm(n, n)
+    inv = w4.w4_invert_permutation(torch.from_numpy(perm).to(cuda_device)).cpu().numpy()
+    assert (inv[perm] == np.arange(n)).all()
+    assert w4.w4_device_error() == 0
+
+
+@pytest.mark.gpu
 def test_out_of_range_index_is_reported_not_read(cuda_device):
     import torch
     w4 = lib()
