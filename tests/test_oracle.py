@@ -567,3 +567,30 @@ def test_variant_matmul_one_hot_and_adjoint(zero, meta):
     rhs = float(np.sum(bf16_value(X) * x64))
     assert abs(lhs - rhs) <= 1e-9 * (abs(lhs) + 1.0)
     assert np.allclose(y64, bf16_value(X) @ wh.T, rtol=1e-12, atol=1e-12)
+
+
+def test_act_order_reading_reduces_to_the_unpermuted_product():
+    """Act-order: packed column j holds input channel perm[j].  Quantizing W[:, perm] and
+    multiplying X[:, perm] equals the plain product with the dequantized weights put back in
+    channel order (w_full[:, perm[j]] = w_hat[:, j]); the transposed product lands in
+    dX[:, perm]."""
+    N, K, g = 48, 256, 32
+    W = synth.weights(N, K, 13)
+    X = synth.activations(3, K, 13)
+    dY = synth.grads(3, N, 13)
+    perm = np.random.default_rng(13).permutation(K)
+    p, s, z = oracle.quantize_pack(W[:, perm], "groupwise", g)
+    wh = oracle.dequant(p, s, z, "groupwise", g, K)
+    w_full = np.empty_like(wh)
+    w_full[:, perm] = wh
+    y64, _ = oracle.linear(X[:, perm], p, s, z, "groupwise", g, N, K)
+    assert np.allclose(y64, bf16_value(X) @ w_full.T, rtol=1e-12, atol=1e-12)
+    x64p, _ = oracle.linear_t(dY, p, s, z, "groupwise", g, N, K)
+    x64 = np.empty_like(x64p)
+    x64[:, perm] = x64p
+    assert np.allclose(x64, bf16_value(dY) @ w_full, rtol=1e-12, atol=1e-12)
+    # with the identity permutation it is the ordinary layer
+    p0, s0, z0 = oracle.quantize_pack(W, "groupwise", g)
+    pi = np.arange(K)
+    pi_p, pi_s, pi_z = oracle.quantize_pack(W[:, pi], "groupwise", g)
+    assert (pi_p == p0).all() and (pi_s == s0).all() and (pi_z == z0).all()
