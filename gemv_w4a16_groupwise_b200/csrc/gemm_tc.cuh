@@ -22,13 +22,20 @@
 //   warp 0       TMA producer: packed weight tile + activation tile per stage,
 //                and, for groupwise scales whose row stride is a multiple of
 //                16 bytes, a box of 8 groups x the tile's rows of S and of Z,
-//                so that the scales arrive with the weights a ring ahead
+//                so that the scales arrive with the weights a ring ahead.  The
+//                weights (with their scales) complete one barrier and the
+//                activation tile another, so the dequantization of a stage does
+//                not wait for the activation bytes, which only the MMA reads
 //   warp 1       TMEM allocator; lane 0 issues tcgen05.mma and commits
 //   warps 2..17  dequantize packed codes into the bf16 A tile of a stage
 //                (128-byte swizzled UMMA layout).  Two groups of 8 warps take
-//                alternate stages, so two stages are being dequantized at any
-//                time and the tensor pipe is not left waiting on one stage's
-//                dequantization latency.
+//                alternate stages, four packed words per thread, so two
+//                stages are being dequantized at any time: a warp's share of
+//                a stage is a chain of dependent steps (wait, scale and code
+//                loads, arithmetic, stores, proxy fence, arrival) whose
+//                latency hardly depends on how many words it converts, so
+//                one group of 16 warps on every stage (kTcDeqGroups = 1, two
+//                words per thread) measured 25 % slower.
 //   warps 18..21 epilogue: TMEM -> registers, fp32 bias, one bf16 rounding,
 //                store (warp w reads the TMEM lanes 32 (w % 4) .. + 31).
 // Every mbarrier wait is bounded; a wait that runs out records the reason in
@@ -48,11 +55,15 @@
 
 namespace w4 {
 
-constexpr int kTcDeqGroups = 2;                      // dequantizing warp groups (8 warps each)
+constexpr int kTcDeqWarps = 16;                      // dequantizing warps
+constexpr int kTcDeqGroups = 2;                      // groups of them that take alternate stages
 constexpr int kTcEpiWarps = 4;
-constexpr int kTcThreads = 64 + kTcDeqGroups * 256 + kTcEpiWarps * 32;
+constexpr int kTcThreads = 64 + kTcDeqWarps * 32 + kTcEpiWarps * 32;
 constexpr int kTcBM = 128;     // MMA M (weight rows per tile)
 constexpr int kTcBK = 64;      // reduction depth per pipeline stage
+constexpr int kTcDeqGroupThreads = kTcDeqWarps * 32 / kTcDeqGroups;
+constexpr int kTcWpt = kTcBM * kTcBK / 8 / kTcDeqGroupThreads;   // packed words per thread and stage
+static_assert(kTcWpt == 2 || kTcWpt == 4, "dequantization mapping");
 constexpr int kTcABytes = kTcBM * kTcBK * 2;   // 16 KB dequantized tile
 constexpr int kTcPBytes = kTcBM * kTcBK / 2;   // 4 KB packed tile
 
@@ -188,14 +199,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr int kSzRows = TR ? kTcBK : kTcBM;                 // weight rows of a stage
     constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;          // one accumulator buffer
     constexpr uint32_t kTmemCols = 2 * kAccCols;              // two, a power of two >= 64
-    constexpr uint32_t kTxBytes = kTcPBytes + BN * 128;
+    constexpr uint32_t kBTxBytes = BN * 128;
     constexpr uint32_t kIdesc = umma_idesc_bf16(BN, TR);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int NS = a.stages;
+    // tma_full: the stage's packed weights (and scale / zero boxes), which the
+    // dequantizing warps wait for; b_full: its activation tile, which only
+    // the MMA needs.  Separate barriers let the dequantization start as soon
+    // as its 8 KB land, while the larger activation tile is still arriving.
     uint64_t* tma_full = reinterpret_cast<uint64_t*>(base + NS * kStageBytes);
-    uint64_t* deq_full = tma_full + NS;
+    uint64_t* b_full = tma_full + NS;
+    uint64_t* deq_full = b_full + NS;
     uint64_t* empty = deq_full + NS;
     uint64_t* acc_full = empty + NS;          // [2] an accumulator buffer holds a finished tile
     uint64_t* acc_empty = acc_full + 2;       // [2] the epilogue has drained a buffer
@@ -237,7 +253,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&tma_full[s], 1);
-            mbar_init(&deq_full[s], 8);
+            mbar_init(&b_full[s], 1);
+            mbar_init(&deq_full[s], kTcDeqWarps / kTcDeqGroups);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -280,12 +297,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         break;
                     }
                     uint8_t* st = base + s * kStageBytes;
-                    mbar_arrive_expect_tx(&tma_full[s], kTxBytes + (a.sz_tma ? 2 * kSzRows * 16 : 0));
+                    mbar_arrive_expect_tx(&tma_full[s], kTcPBytes + (a.sz_tma ? 2 * kSzRows * 16 : 0));
                     if (TR)
                         tma_load_2d(st + kTcABytes + BN * 128, &pmap, r0 / 8, kb * kTcBK, &tma_full[s]);
                     else
                         tma_load_2d(st + kTcABytes + BN * 128, &pmap, kb * (kTcBK / 8), r0, &tma_full[s]);
-                    tma_load_2d(st + kTcABytes, &bmap, kb * kTcBK, m0, &tma_full[s]);
                     if (a.sz_tma) {
                         // groups from the stage's first one, rounded down to a
                         // multiple of 8 (16 bytes), for the stage's weight rows
@@ -294,6 +310,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         tma_load_2d(st + kSzOff, &smap, x0, y0, &tma_full[s]);
                         tma_load_2d(st + kSzOff + kSzRows * 16, &zmap, x0, y0, &tma_full[s]);
                     }
+                    mbar_arrive_expect_tx(&b_full[s], kBTxBytes);
+                    tma_load_2d(st + kTcABytes, &bmap, kb * kTcBK, m0, &b_full[s]);
                     if (++s == NS) {
                         s = 0;
                         ++round;
@@ -316,8 +334,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc_fence_after();
                 const uint32_t acc = tmem_d + static_cast<uint32_t>(buf) * kAccCols;
                 for (int kb = w.kb0; kb < w.kb1; ++kb) {
-                    ok = mbar_wait_bounded(&tma_full[s], phase, abort_flag, kErrTimeoutTmaFull) &&
-                         mbar_wait_bounded(&deq_full[s], phase, abort_flag, kErrTimeoutDequant);
+                    // deq_full implies tma_full: every dequantizing warp waited for it
+                    ok = mbar_wait_bounded(&deq_full[s], phase, abort_flag, kErrTimeoutDequant) &&
+                         mbar_wait_bounded(&b_full[s], phase, abort_flag, kErrTimeoutTmaFull);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(base + s * kStageBytes);
@@ -338,32 +357,45 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 umma_commit(&acc_full[buf]);   // also tracks any MMA issued before an abort
             }
         }
-    } else if (warp < 2 + 8 * kTcDeqGroups) {
+    } else if (warp < 2 + kTcDeqWarps) {
         // ------------------------------------------------ dequantize
         // Stages are numbered across the CTA's units, in order; group grp_id
-        // takes stages grp_id, grp_id + 2, ...
-        const int grp_id = (threadIdx.x - 64) >> 8;
-        const int t = (threadIdx.x - 64) & 255;               // 0 .. 255 within the group
-        // forward: row n = r0 + t / 2, words 4 (t % 2) .. + 3 of the 8 in a k-block
-        //   (a phase of 8 lanes reads 4 rows' 32 bytes: 128 contiguous bytes, no bank
-        //   conflict; its swizzled 16-byte stores still land in 8 distinct banks)
-        // transposed: row n = kb * 64 + prow, words 4q .. 4q+3 of the 16 of a k-tile,
-        //   with (prow, q) spread so that a phase of 8 lanes takes 4 rows x 2 quads of
-        //   one 64-k atom: its 16-byte loads meet at most 2 to a bank (4 before) and its
-        //   MN-major stores fall into 8 distinct banks
-        const int prow = TR ? (((t >> 4) << 2) | ((t >> 1) & 3)) : (t >> 1);
-        const int pquad = TR ? ((((t >> 3) & 1) << 1) | (t & 1)) : (t & 1);
+        // takes stages grp_id, grp_id + kTcDeqGroups, ...  Each thread of a
+        // group dequantizes kTcWpt packed words (8 codes each) of one weight row.
+        const int grp_id = (threadIdx.x - 64) / kTcDeqGroupThreads;
+        const int t = (threadIdx.x - 64) % kTcDeqGroupThreads;
+        int prow, pw;          // the thread's row in the stage and its first word in that row
+        if (kTcWpt == 4) {
+            // forward: row t / 2, words 4 (t % 2) .. + 3 of the 8 in a k-block (a phase of
+            //   8 lanes reads 4 rows' 32 bytes: 128 contiguous bytes, no bank conflict; its
+            //   swizzled 16-byte stores still land in 8 distinct banks)
+            // transposed: words 4q .. 4q+3 of the 16 of a k-tile, with (row, q) spread so
+            //   that a phase of 8 lanes takes 4 rows x 2 quads of one 64-k atom: its 16-byte
+            //   loads meet at most 2 to a bank and its MN-major stores fall into 8 distinct banks
+            prow = TR ? (((t >> 4) << 2) | ((t >> 1) & 3)) : (t >> 1);
+            pw = 4 * (TR ? ((((t >> 3) & 1) << 1) | (t & 1)) : (t & 1));
+        } else {
+            // forward: row t / 4, words 2 (t % 4), + 1 (a half warp reads 4 rows' 32 bytes,
+            //   128 contiguous bytes; 8 lanes store 2 rows x 4 chunks of one parity, which
+            //   the swizzle puts in 8 distinct banks)
+            // transposed: lane = (row bit 1, atom, row bit 0, pair 0..3), 4 rows per warp: a
+            //   half warp reads 2 rows' 64 bytes (128 contiguous bytes); 8 lanes store 2 rows
+            //   x 4 chunks of one atom, again 8 distinct banks
+            const int l = t & 31;
+            prow = TR ? ((t >> 5) * 4 + ((l >> 4) & 1) * 2 + ((l >> 2) & 1)) : (t >> 2);
+            pw = TR ? (((l >> 3) & 1) * 8 + (l & 3) * 2) : 2 * (t & 3);
+        }
         const int W8 = a.K / 8;
-        // swizzled 16-byte destinations of this thread's 4 words in the A tile
-        uint32_t off[4];
+        // swizzled 16-byte destinations of this thread's words in the A tile
+        uint32_t off[kTcWpt];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kTcWpt; ++j) {
             if (TR) {
-                const int kk = 32 * pquad + 8 * j;        // k within the 128-wide tile
+                const int kk = 8 * (pw + j);               // k within the 128-wide tile
                 const int atom = kk >> 6, c = (kk & 63) >> 3;
                 off[j] = atom * 8192 + (prow >> 3) * 1024 + (prow & 7) * 128 + ((c ^ (prow & 7)) << 4);
             } else {
-                const int c = 4 * pquad + j;               // 16-byte chunk within the row
+                const int c = pw + j;                      // 16-byte chunk within the row
                 off[j] = prow * 128 + ((c ^ (prow & 7)) << 4);
             }
         }
@@ -373,15 +405,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool mbf = (a.fmt & kFmtMetaBf16) != 0;
         constexpr bool fz = FZ;     // a.fmt & kFmtZeroFloat, as a template argument
         // Scale / zero of one stage (tile i, block kb); with g a multiple of
-        // 32 the thread's 4 words share one group.
-        constexpr int NG = PWG ? 4 : 1;
+        // 32 the thread's words share one group.
+        constexpr int NG = PWG ? kTcWpt : 1;
         auto tile_r0 = [&](int i) { return (unit_of(i).t / tiles_m) * kTcBM; };
         auto load_sz = [&](int r0, int kb, float (&sv)[NG], float (&zv)[NG]) {
             const int n = TR ? kb * kTcBK + prow : r0 + prow;
             const int nc = min(n, a.N - 1);
             const __half* sp = a.S + static_cast<size_t>(nc) * a.sz_row;
             const __half* zp = a.Z + static_cast<size_t>(nc) * a.sz_row;
-            const int kw0 = TR ? r0 / 8 + 4 * pquad : kb * (kTcBK / 8) + 4 * pquad;
+            const int kw0 = TR ? r0 / 8 + pw : kb * (kTcBK / 8) + pw;
 #pragma unroll
             for (int j = 0; j < NG; ++j) {
                 const int grp = group_of(8 * (kw0 + j));
@@ -423,7 +455,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (more && !a.sz_tma) load_sz(nr0, nkb, svn, zvn);
             const int r0 = cr0;
             const int n = TR ? ckb * kTcBK + prow : r0 + prow;
-            const int kw0 = TR ? r0 / 8 + 4 * pquad : ckb * (kTcBK / 8) + 4 * pquad;
+            const int kw0 = TR ? r0 / 8 + pw : ckb * (kTcBK / 8) + pw;
             const bool row_ok = n < a.N;
             const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&tma_full[s], phase, abort_flag,
                                                                       kErrTimeoutTmaFull));
@@ -441,12 +473,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         zv[j] = meta_to_float(hz[idx], mbf);
                     }
                 }
-                const uint8_t* pk = st + kTcABytes + BN * 128;
-                const uint4 wv = TR ? *reinterpret_cast<const uint4*>(pk + prow * 64 + pquad * 16)
-                                    : *reinterpret_cast<const uint4*>(pk + prow * 32 + pquad * 16);
+                const uint8_t* pk = st + kTcABytes + BN * 128 + prow * (TR ? 64 : 32) + pw * 4;
+                uint32_t wv[kTcWpt];
+                if constexpr (kTcWpt == 4) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(pk);
+                    wv[0] = v.x;
+                    wv[1] = v.y;
+                    wv[2] = v.z;
+                    wv[3] = v.w;
+                } else {
+                    const uint2 v = *reinterpret_cast<const uint2*>(pk);
+                    wv[0] = v.x;
+                    wv[1] = v.y;
+                }
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t w = (j == 0) ? wv.x : (j == 1) ? wv.y : (j == 2) ? wv.z : wv.w;
+                for (int j = 0; j < kTcWpt; ++j) {
+                    const uint32_t w = wv[j];
                     const float sj = sv[PWG ? j : 0], zj = zv[PWG ? j : 0];
                     uint4 out = make_uint4(0u, 0u, 0u, 0u);
                     if (row_ok && (kw0 + j) < W8)

@@ -918,10 +918,10 @@ w4_status run_gemm_tc(const TcProblem& p, void* ws, size_t ws_bytes, cudaStream_
     const int sz_rows = tr ? kTcBK : kTcBM;
     const int stage = tc_stage_bytes(BN) + (sz_tma ? 2 * sz_rows * 16 : 0);
     const size_t fixed = 1024 + 64;
-    int stages = static_cast<int>((static_cast<size_t>(di.max_smem_optin) - fixed - 64) / (stage + 24));
+    int stages = static_cast<int>((static_cast<size_t>(di.max_smem_optin) - fixed - 64) / (stage + 32));
     stages = std::min(stages, 8);
     if (stages < 2) return W4_ERR_UNSUPPORTED;
-    const size_t smem = fixed + static_cast<size_t>(stages) * stage + static_cast<size_t>(3 * stages + 4) * 8 + 16;
+    const size_t smem = fixed + static_cast<size_t>(stages) * stage + static_cast<size_t>(4 * stages + 4) * 8 + 16;
     CUtensorMap maps[4];
     std::memset(maps, 0, sizeof maps);
     CUtensorMap& pm = maps[0];
