@@ -328,6 +328,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
                    const __grid_constant__ CUtensorMap zmap, const GemvQ8Args a) {
     static_assert(M >= 1 && M <= 4, "M");
     constexpr int NSET = (M + 1) / 2;
+    // the test hook that withholds a stage (-1 unless a test injects a lost
+    // stage) is set by the host before the launch: read it first thing, so
+    // that its global-memory latency overlaps the set-up instead of delaying
+    // the producer's first copy
+    const int withhold = threadIdx.x >= kQW * 32 ? *reinterpret_cast<volatile int*>(&g_withhold_stage) : -1;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int NS = a.stages;
@@ -379,7 +384,6 @@ __global__ void __launch_bounds__(kQThreads, 1)
         int s = 0, it = 0;
         uint32_t round = 0;
         bool alive = true;
-        const int withhold = g_withhold_stage;     // -1 unless a test injects a lost stage
         for (int c = 0; c < nch && alive; ++c) {
             const int r0 = chunk_lo(c), rc = chunk_lo(c + 1) - r0;
             for (int ks = 0; ks < a.nks && alive; ++ks) {

@@ -89,6 +89,11 @@ __global__ void __launch_bounds__(kTMThreads, 1)
     static_assert(M >= 1 && M <= 4, "M");
     static_assert(KW == 128 || KW == 64, "KW");
     static_assert(SZ == kSzConst || SZ == kSzTma2d || SZ == kSzTma1d, "scale / zero path");
+    // the test hook that withholds a stage (-1 unless a test injects a lost
+    // stage) is set by the host before the launch: read it first thing, so
+    // that its global-memory latency overlaps the set-up instead of delaying
+    // the producer's first copy
+    const int withhold = threadIdx.x >= kTMW * 32 ? *reinterpret_cast<volatile int*>(&g_withhold_stage) : -1;
     constexpr int NSET = (M + 1) / 2;
     constexpr int NT = KW / 16;                   // k-tiles per warp
     constexpr int NWD = KW / 64;                  // packed words per row and lane
@@ -143,7 +148,6 @@ __global__ void __launch_bounds__(kTMThreads, 1)
         // that a last stage carries meet c = 0
         int s = 0;
         uint32_t round = 0;
-        const int withhold = g_withhold_stage;     // -1 unless a test injects a lost stage
         for (int b = 0; b < nst; ++b) {
             if (round > 0) {
                 const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&empty[s], (round - 1) & 1u, abort_flag,

@@ -984,23 +984,17 @@ static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / 
 
 // Device address of the scratch array on the current device.  Host code
 // cannot pass &g_noalloc_scratch to a kernel (that name is a host-side
-// stand-in), so the first call on each device looks the address up with
-// that device current and caches it.
+// stand-in), so every call looks the address up with the device current
+// (the lookup allocates nothing).  It is not cached: after cudaDeviceReset,
+// or a primary context torn down and created again, the module is loaded
+// anew and the array may sit at another address.
 w4_status noalloc_scratch(void** out) {
-    static std::mutex mu;
-    static void* ptrs[64] = {};
-    const int dev = current_device();
-    if (dev < 0 || dev >= 64) return W4_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!ptrs[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
-            cudaGetLastError();
-            return W4_ERR_CUDA;
-        }
-        ptrs[dev] = p;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+        g_last_cuda_error = cudaGetLastError();
+        return W4_ERR_CUDA;
     }
-    *out = ptrs[dev];
+    *out = p;
     return W4_OK;
 }
 
