@@ -1021,6 +1021,36 @@ size_t w4_quantize_workspace_bytes(int N, int K, int mode) {
     return (mode & kModeBaseMask) == W4_MODE_GLOBAL ? 1024 * sizeof(float2) : 0;
 }
 
+}  // extern "C"
+
+namespace {
+// The segmented quantizer with its format flags as a template argument.
+template <int LPG, int WPT>
+void launch_quantize_segmented(int fmt, int blocks, cudaStream_t st, const uint16_t* w, long long total_words,
+                               uint32_t* packed, uint16_t* sc, uint16_t* ze) {
+    using w4::kFmtMetaBf16;
+    using w4::kFmtZeroFloat;
+    switch (fmt & (kFmtZeroFloat | kFmtMetaBf16)) {
+        case 0:
+            w4::quantize_segmented_kernel<LPG, WPT, 0><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze);
+            break;
+        case kFmtZeroFloat:
+            w4::quantize_segmented_kernel<LPG, WPT, kFmtZeroFloat><<<blocks, 256, 0, st>>>(w, total_words, packed,
+                                                                                          sc, ze);
+            break;
+        case kFmtMetaBf16:
+            w4::quantize_segmented_kernel<LPG, WPT, kFmtMetaBf16><<<blocks, 256, 0, st>>>(w, total_words, packed,
+                                                                                         sc, ze);
+            break;
+        default:
+            w4::quantize_segmented_kernel<LPG, WPT, kFmtZeroFloat | kFmtMetaBf16>
+                <<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze);
+    }
+}
+}  // namespace
+
+extern "C" {
+
 w4_status w4_quantize_pack(const void* W, int N, int K, int mode, int group_size, uint32_t* packed,
                            void* scales, void* zeros, void* workspace, size_t workspace_bytes,
                            void* stream) {
@@ -1076,13 +1106,13 @@ w4_status w4_quantize_pack(const void* W, int N, int K, int mode, int group_size
     const int wpt = lpg >= 2 ? 2 : 1;
     const int blocks = static_cast<int>((total_words / wpt + 255) / 256);
     switch (lpg) {
-        case 1: quantize_segmented_kernel<1, 1><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
-        case 2: quantize_segmented_kernel<1, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
-        case 4: quantize_segmented_kernel<2, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
-        case 8: quantize_segmented_kernel<4, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
-        case 16: quantize_segmented_kernel<8, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
-        case 32: quantize_segmented_kernel<16, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
-        case 64: quantize_segmented_kernel<32, 2><<<blocks, 256, 0, st>>>(w, total_words, packed, sc, ze, fmt); break;
+        case 1: launch_quantize_segmented<1, 1>(fmt, blocks, st, w, total_words, packed, sc, ze); break;
+        case 2: launch_quantize_segmented<1, 2>(fmt, blocks, st, w, total_words, packed, sc, ze); break;
+        case 4: launch_quantize_segmented<2, 2>(fmt, blocks, st, w, total_words, packed, sc, ze); break;
+        case 8: launch_quantize_segmented<4, 2>(fmt, blocks, st, w, total_words, packed, sc, ze); break;
+        case 16: launch_quantize_segmented<8, 2>(fmt, blocks, st, w, total_words, packed, sc, ze); break;
+        case 32: launch_quantize_segmented<16, 2>(fmt, blocks, st, w, total_words, packed, sc, ze); break;
+        case 64: launch_quantize_segmented<32, 2>(fmt, blocks, st, w, total_words, packed, sc, ze); break;
         default: {
             const long long groups = total_words / lpg;
             const int gblocks = static_cast<int>((groups + 7) / 8);
