@@ -118,7 +118,7 @@ def _check_cuda(t, name, dtype, shape=None):
     torch = _torch()
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if t.device.type != "cuda":
+    if not t.is_cuda:
         raise ValueError(f"{name} must live on a CUDA device (no CPU path exists)")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
@@ -146,9 +146,60 @@ def _check_perm(perm, K: int, dev):
         raise ValueError("perm must be on the activations' device")
 
 
-def _stream_ptr(device):
+def _device_index(device) -> int:
     torch = _torch()
-    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    if isinstance(device, int):
+        return device
+    return device.index if device.index is not None else torch.cuda.current_device()
+
+
+def _stream_ptr(device):
+    """The current stream of `device` as a raw handle.  PyTorch's own raw
+    accessor (what its compiled kernels use) costs a tenth of building the
+    Stream object; the public call is the fallback."""
+    torch = _torch()
+    idx = _device_index(device)
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    if raw is not None:
+        return ctypes.c_void_p(raw(idx))
+    return ctypes.c_void_p(torch.cuda.current_stream(idx).cuda_stream)
+
+
+class _OnDevice:
+    """Make `idx` the current device for a library call and restore the
+    previous one, switching only when they differ (the library launches on
+    the current device)."""
+
+    __slots__ = ("idx", "prev", "_get", "_set")
+
+    def __init__(self, device):
+        torch = _torch()
+        self.idx = _device_index(device)
+        self._get = getattr(torch._C, "_cuda_getDevice", None)
+        self._set = getattr(torch._C, "_cuda_setDevice", None)
+        self.prev = None
+
+    def __enter__(self):
+        if self._get is None or self._set is None:
+            self.prev = _torch().cuda.device(self.idx)
+            self.prev.__enter__()
+            return self
+        self.prev = self._get()
+        if self.prev != self.idx:
+            self._set(self.idx)
+        return self
+
+    def __exit__(self, *exc):
+        if self._get is None or self._set is None:
+            return self.prev.__exit__(*exc)
+        if self.prev != self.idx:
+            self._set(self.prev)
+        return False
+
+
+# w4_workspace_bytes by (device, M, N, K, transposed): a pure function of
+# the shape and the device's SM count
+_ws_cache: dict = {}
 
 
 def meta_shape(N: int, K: int, mode, group_size: int):
@@ -240,14 +291,20 @@ def _matmul(fname, A, packed, scales, zeros, mode, group_size, N, K, bias, trans
         out = torch.empty((M, out_len), dtype=torch.bfloat16, device=dev)
     else:
         _check_cuda(out, "out", torch.bfloat16, (M, out_len))
-    nws = w4_workspace_bytes(M, N, K, transposed)
-    ws = torch.empty(nws, dtype=torch.uint8, device=dev) if nws else None
-    with torch.cuda.device(dev):
+    with _OnDevice(dev) as on:
+        key = (on.idx, M, N, K, bool(transposed))
+        nws = _ws_cache.get(key)
+        if nws is None:
+            nws = w4_workspace_bytes(M, N, K, transposed)
+            if len(_ws_cache) > 4096:
+                _ws_cache.clear()
+            _ws_cache[key] = nws
+        ws = torch.empty(nws, dtype=torch.uint8, device=dev) if nws else None
         st = getattr(library(), fname)(
             A.data_ptr(), M, N, K, packed.data_ptr(), scales.data_ptr(), zeros.data_ptr(),
             _mode(mode, zero, meta), int(group_size), None if bias is None else bias.data_ptr(),
             int(bool(transposed)), out.data_ptr(), None if ws is None else ws.data_ptr(), nws,
-            _stream_ptr(dev))
+            _stream_ptr(on.idx))
     if st != 0:
         raise W4Error(st, fname)
     return out
