@@ -19,6 +19,9 @@ Entry points (same names as the C ABI in ``include/w4a16.h``):
   permutations of act-order weights (``perm=`` on the calls above)
 * :func:`w4_workspace_bytes`, :func:`w4_device_error`
 
+:mod:`gemv_w4a16_groupwise_b200.tp` shards one layer over torch.distributed
+ranks (column-parallel over N, row-parallel over K) on top of these calls.
+
 ``packed`` may also be given as its two-per-byte view, uint8 [N, K/2] (the
 same bytes; the even k in the low nibble).
 """
